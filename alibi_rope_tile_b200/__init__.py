@@ -1,0 +1,210 @@
+"""B200 (sm_100a) attention core: a thin ctypes binding of ``libattn_rope_tile.so``.
+
+The functions here carry the C ABI's names (``include/attn_rope_tile.h``) and only
+marshal arguments: they read shapes, dtypes and data pointers from torch CUDA tensors,
+allocate outputs with torch when the caller gives none, pass the current torch stream,
+and raise ``AttnError`` on a non-zero status. Every step of the computation runs in the
+library's CUDA kernels; there is no fallback of any kind. If the library has not been
+built, the first call raises ``RuntimeError`` (build it with
+``python -m alibi_rope_tile_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn_rope_tile.so")
+
+ATTN_F32, ATTN_BF16 = 0, 1
+STATUS = {0: "ATTN_OK", -1: "ATTN_ERR_ARG", -2: "ATTN_ERR_ALIGN", -3: "ATTN_ERR_UNSUPPORTED",
+          -4: "ATTN_ERR_CUDA", -5: "ATTN_ERR_TIMEOUT", -6: "ATTN_ERR_WORKSPACE",
+          -7: "ATTN_ERR_DEVICE_ARG"}
+
+_P, _I, _L, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_size_t
+_FP = ctypes.POINTER(ctypes.c_float)
+
+# (name, restype, argtypes) of every exported entry point
+SIGNATURES = {
+    "attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _F, _I, _I, _FP, _I, _P]),
+    "attn_decode_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _FP, _I, _P, _S,
+                         _P]),
+    "attn_kv_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_block_workspace_size": (_S, [_I, _I, _I, _I, _I, _I, _I]),
+    "attn_block": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _L, _F, _I, _I, _FP, _I,
+                        _P, _S, _P]),
+    "attn_alibi_slopes": (None, [_I, _FP]),
+    "attn_sync_status": (_I, [_P]),
+    "attn_last_error": (_I, [ctypes.c_char_p, _S]),
+    "attn_version": (ctypes.c_char_p, []),
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (loaded on first use; raises if it is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                               "(run python -m alibi_rope_tile_b200.build)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        buf = ctypes.create_string_buffer(512)
+        lib().attn_last_error(buf, 512)
+        raise AttnError(status, buf.value.decode(errors="replace"))
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return ATTN_F32
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None) -> int:
+    if t is None:
+        return 0
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _slopes(slopes, H: int):
+    if slopes is None:
+        return None
+    vals = [float(x) for x in (slopes.tolist() if hasattr(slopes, "tolist") else slopes)]
+    if len(vals) != H:
+        raise ValueError(f"alibi_slopes needs {H} values, got {len(vals)}")
+    return (ctypes.c_float * H)(*vals)
+
+
+def alibi_slopes(H: int) -> list:
+    """The library's ALiBi schedule 2^(-8(h+1)/H) (computed by attn_alibi_slopes)."""
+    buf = (ctypes.c_float * H)()
+    lib().attn_alibi_slopes(H, buf)
+    return list(buf)
+
+
+def attn_prefill(q, k, v, out=None, lse=None, *, pos0: int = 0, rope_base: float = 0.0,
+                 causal: bool = True, window: int = 0, alibi_slopes: Optional[Sequence] = None,
+                 stream=None):
+    """q [B,T,H,hd], k/v [B,T,KV,hd] (CUDA, fp32 or bf16) -> out [B,T,H,hd] (and lse [B,H,T])."""
+    B, T, H, hd = q.shape
+    KV = k.shape[2]
+    if k.shape != (B, T, KV, hd) or v.shape != k.shape:
+        raise ValueError(f"k and v must be [B,T,KV,hd] matching q {tuple(q.shape)}")
+    dt = q.dtype
+    if out is None:
+        out = torch.empty_like(q)
+    st = lib().attn_prefill(_dev(q, "q"), _dev(k, "k", dt), _dev(v, "v", dt), _dev(out, "out", dt),
+                            _dev(lse, "lse", torch.float32), B, T, H, KV, hd, int(pos0),
+                            float(rope_base), int(bool(causal)), int(window),
+                            _slopes(alibi_slopes, H), _dtype(q), _stream(stream))
+    _check(st)
+    return out
+
+
+def attn_decode_workspace_size(B: int, H: int, KV: int, hd: int, Lmax: int) -> int:
+    return int(lib().attn_decode_workspace_size(B, H, KV, hd, Lmax))
+
+
+def attn_decode(q, kcache, vcache, seqlens, qpos, out=None, lse=None, workspace=None, *,
+                rope_base: float = 0.0, window: int = 0, alibi_slopes=None, stream=None):
+    """q [B,H,hd] (not rotated), caches [B,Lmax,KV,hd], seqlens/qpos [B] int32 -> out [B,H,hd]."""
+    B, H, hd = q.shape
+    _, Lmax, KV, _ = kcache.shape
+    dt = q.dtype
+    if out is None:
+        out = torch.empty_like(q)
+    need = attn_decode_workspace_size(B, H, KV, hd, Lmax)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib().attn_decode(_dev(q, "q"), _dev(kcache, "kcache", dt), _dev(vcache, "vcache", dt),
+                           _dev(seqlens, "seqlens", torch.int32), _dev(qpos, "qpos", torch.int32),
+                           _dev(out, "out", dt), _dev(lse, "lse", torch.float32), B, H, KV, hd, Lmax,
+                           float(rope_base), int(window), _slopes(alibi_slopes, H), _dtype(q),
+                           _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                           _stream(stream))
+    _check(st)
+    return out
+
+
+def attn_kv_append(k_new, v_new, kcache, vcache, pos, *, rope_base: float = 0.0, stream=None):
+    """Write k_new (rotated at pos[b]) and v_new [B,KV,hd] into cache slot pos[b]."""
+    B, KV, hd = k_new.shape
+    Lmax = kcache.shape[1]
+    dt = k_new.dtype
+    st = lib().attn_kv_append(_dev(k_new, "k_new"), _dev(v_new, "v_new", dt),
+                              _dev(kcache, "kcache", dt), _dev(vcache, "vcache", dt),
+                              _dev(pos, "pos", torch.int32), B, KV, hd, Lmax, float(rope_base),
+                              _dtype(k_new), _stream(stream))
+    _check(st)
+
+
+def attn_block_workspace_size(B, T, d, H, KV, hd, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else (ATTN_F32 if dtype == torch.float32 else ATTN_BF16)
+    return int(lib().attn_block_workspace_size(B, T, d, H, KV, hd, code))
+
+
+def attn_block(x, Wq, Wk, Wv, Wo, out=None, workspace=None, *, H: int, KV: int, pos0: int = 0,
+               rope_base: float = 0.0, causal: bool = True, window: int = 0, alibi_slopes=None,
+               stream=None):
+    """x [B,T,d] -> out [B,T,d] = attention(x Wq, x Wk, x Wv) Wo (weights [in, out])."""
+    B, T, d = x.shape
+    hd = Wq.shape[1] // H
+    dt = x.dtype
+    if out is None:
+        out = torch.empty_like(x)
+    need = attn_block_workspace_size(B, T, d, H, KV, hd, dt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    st = lib().attn_block(_dev(x, "x"), _dev(Wq, "Wq", dt), _dev(Wk, "Wk", dt), _dev(Wv, "Wv", dt),
+                          _dev(Wo, "Wo", dt), _dev(out, "out", dt), B, T, d, H, KV, hd, int(pos0),
+                          float(rope_base), int(bool(causal)), int(window), _slopes(alibi_slopes, H),
+                          _dtype(x), _dev(workspace, "workspace"),
+                          workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st)
+    return out
+
+
+def attn_sync_status(stream=None) -> int:
+    """Synchronise and read (then clear) the device error word; raises AttnError if set."""
+    st = lib().attn_sync_status(_stream(stream))
+    _check(st)
+    return st
+
+
+def attn_version() -> str:
+    return lib().attn_version().decode()

@@ -1,0 +1,314 @@
+// Host side of the C ABI declared in include/attn_rope_tile.h: argument checks, the
+// per-call rotary/ALiBi tables, dispatch to the kernels, and error reporting. No entry
+// point allocates device memory.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "attn_rope_tile.h"
+#include "kernels.h"
+
+using namespace attn;
+
+namespace {
+
+thread_local char g_msg[512] = "no error";
+thread_local int g_last = ATTN_OK;
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  g_last = code;
+  return code;
+}
+
+int ok() {
+  g_last = ATTN_OK;
+  return ATTN_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(ATTN_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+// Per-device status word written by kernels that find a bad device-resident argument or
+// give up on a bounded wait. Host code reaches it through cudaGetSymbolAddress.
+__device__ int g_attn_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
+int* g_status_ptr[kMaxDevices] = {};
+
+int* device_status(int* err) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *err = cuda_fail(e == cudaSuccess ? cudaErrorInvalidDevice : e, "cudaGetDevice");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_attn_device_status);
+    if (e != cudaSuccess) {
+      *err = cuda_fail(e, "cudaGetSymbolAddress(status word)");
+      return nullptr;
+    }
+    g_status_ptr[dev] = static_cast<int*>(ptr);
+  }
+  return g_status_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(int dtype) { return dtype == ATTN_F32 ? 4 : 2; }
+
+RopeFreqs make_rope(int hd, float base) {
+  RopeFreqs r;
+  std::memset(&r, 0, sizeof(r));
+  r.on = base > 0.f;
+  if (!r.on) return r;
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int c = 0; c < hd / 2; ++c) {
+    const double w = std::pow((double)base, -2.0 * c / hd) / two_pi;  // turns per position
+    const float hi = (float)w;
+    r.hi[c] = hi;
+    r.lo[c] = (float)(w - (double)hi);
+  }
+  return r;
+}
+
+int make_alibi(int H, const float* slopes, Alibi* a) {
+  std::memset(a, 0, sizeof(*a));
+  if (!slopes) return ATTN_OK;
+  if (H > ATTN_MAX_ALIBI_HEADS)
+    return fail(ATTN_ERR_UNSUPPORTED, "ALiBi supports at most %d heads (got %d)",
+                ATTN_MAX_ALIBI_HEADS, H);
+  a->on = 1;
+  for (int h = 0; h < H; ++h) {
+    if (!std::isfinite(slopes[h])) return fail(ATTN_ERR_ARG, "alibi_slopes[%d] is not finite", h);
+    a->slope[h] = slopes[h];
+  }
+  return ATTN_OK;
+}
+
+int check_common(int H, int KV, int hd, int dtype, float rope_base) {
+  if (dtype != ATTN_F32 && dtype != ATTN_BF16) return fail(ATTN_ERR_ARG, "dtype %d is not ATTN_F32/ATTN_BF16", dtype);
+  if (H < 1 || KV < 1) return fail(ATTN_ERR_ARG, "H=%d and KV=%d must be >= 1", H, KV);
+  if (H % KV) return fail(ATTN_ERR_ARG, "H=%d is not a multiple of KV=%d", H, KV);
+  if (hd < 2 || hd > ATTN_MAX_HD || (hd & 1))
+    return fail(ATTN_ERR_ARG, "hd=%d must be even and in [2, %d]", hd, ATTN_MAX_HD);
+  if (!std::isfinite(rope_base)) return fail(ATTN_ERR_ARG, "rope_base is not finite");
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int T,
+                 int H, int KV, int hd, long long pos0, float rope_base, int causal, int window,
+                 const float* alibi_slopes, int dtype, void* stream) {
+  int st = check_common(H, KV, hd, dtype, rope_base);
+  if (st) return st;
+  if (!q || !k || !v || !out) return fail(ATTN_ERR_ARG, "q, k, v and out must not be NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (lse && !aligned16(lse)))
+    return fail(ATTN_ERR_ALIGN, "q, k, v, out and lse must be 16-byte aligned");
+  if (B < 1 || T < 1) return fail(ATTN_ERR_ARG, "B=%d and T=%d must be >= 1", B, T);
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
+  if (window < 0) window = 0;
+  if (window > 0 && !causal) return fail(ATTN_ERR_ARG, "a window requires the causal mask");
+  if (pos0 < 0 || pos0 + (long long)T >= (1LL << 24))
+    return fail(ATTN_ERR_ARG, "positions pos0..pos0+T-1 must lie in [0, 2^24)");
+  if ((long long)B * T * H * hd >= (1LL << 40)) return fail(ATTN_ERR_ARG, "tensor too large");
+
+  PrefillParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.k = k; p.v = v; p.out = out; p.lse = lse;
+  p.B = B; p.T = T; p.H = H; p.KV = KV; p.hd = hd;
+  p.pos0 = (int)pos0; p.causal = causal; p.window = window;
+  p.scale = (float)(1.0 / std::sqrt((double)hd));
+  p.rope = make_rope(hd, rope_base);
+  if ((st = make_alibi(H, alibi_slopes, &p.alibi))) return st;
+  int err = 0;
+  p.status = device_status(&err);
+  if (!p.status) return err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = prefill_tc_supported(p, dtype) ? launch_prefill_tc(p, s)
+                                                 : launch_prefill_simt(p, dtype, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attn_prefill launch");
+  return ok();
+}
+
+size_t attn_decode_workspace_size(int B, int H, int KV, int hd, int Lmax) {
+  if (B < 1 || H < 1 || KV < 1 || H % KV || hd < 2 || hd > ATTN_MAX_HD || Lmax < 1) return 0;
+  return decode_workspace_bytes(B, H, KV, hd, Lmax);
+}
+
+int attn_decode(const void* q, const void* kcache, const void* vcache, const int* seqlens,
+                const int* qpos, void* out, float* lse, int B, int H, int KV, int hd, int Lmax,
+                float rope_base, int window, const float* alibi_slopes, int dtype, void* workspace,
+                size_t ws_bytes, void* stream) {
+  int st = check_common(H, KV, hd, dtype, rope_base);
+  if (st) return st;
+  if (!q || !kcache || !vcache || !seqlens || !qpos || !out)
+    return fail(ATTN_ERR_ARG, "q, kcache, vcache, seqlens, qpos and out must not be NULL");
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out) ||
+      (lse && !aligned16(lse)) || (workspace && !aligned16(workspace)))
+    return fail(ATTN_ERR_ALIGN, "q, caches, out, lse and workspace must be 16-byte aligned");
+  if (B < 1 || Lmax < 1) return fail(ATTN_ERR_ARG, "B=%d and Lmax=%d must be >= 1", B, Lmax);
+  if (Lmax >= (1 << 24)) return fail(ATTN_ERR_ARG, "Lmax must be below 2^24");
+  const int G = H / KV;
+  if (!(hd == 8 || hd == 16 || hd == 32 || hd == 64 || hd == 128 || hd == 256))
+    return fail(ATTN_ERR_UNSUPPORTED, "decode supports hd in {8,16,32,64,128,256} (got %d)", hd);
+  if (!(G == 1 || G == 2 || G == 4 || G == 8 || G == 16 || G == 32))
+    return fail(ATTN_ERR_UNSUPPORTED, "decode supports H/KV in {1,2,4,8,16,32} (got %d)", G);
+  if ((size_t)8 * G * (hd + 2) * sizeof(float) > 200 * 1024)
+    return fail(ATTN_ERR_UNSUPPORTED, "decode: H/KV * hd too large for shared memory");
+  if (window < 0) window = 0;
+  const size_t need = decode_workspace_bytes(B, H, KV, hd, Lmax);
+  if (!workspace || ws_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "decode needs %zu bytes of workspace (got %zu)", need, ws_bytes);
+
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.kcache = kcache; p.vcache = vcache; p.seqlens = seqlens; p.qpos = qpos;
+  p.out = out; p.lse = lse;
+  p.B = B; p.H = H; p.KV = KV; p.hd = hd; p.Lmax = Lmax; p.window = window;
+  p.scale = (float)(1.0 / std::sqrt((double)hd));
+  p.rope = make_rope(hd, rope_base);
+  if ((st = make_alibi(H, alibi_slopes, &p.alibi))) return st;
+  int err = 0;
+  p.status = device_status(&err);
+  if (!p.status) return err;
+  cudaError_t e = launch_decode(p, dtype, workspace, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_decode launch");
+  return ok();
+}
+
+int attn_kv_append(const void* k_new, const void* v_new, void* kcache, void* vcache, const int* pos,
+                   int B, int KV, int hd, int Lmax, float rope_base, int dtype, void* stream) {
+  int st = check_common(KV, KV, hd, dtype, rope_base);
+  if (st) return st;
+  if (!k_new || !v_new || !kcache || !vcache || !pos)
+    return fail(ATTN_ERR_ARG, "k_new, v_new, kcache, vcache and pos must not be NULL");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kcache) || !aligned16(vcache))
+    return fail(ATTN_ERR_ALIGN, "k_new, v_new and the caches must be 16-byte aligned");
+  if (B < 1 || Lmax < 1 || Lmax >= (1 << 24)) return fail(ATTN_ERR_ARG, "B >= 1 and 1 <= Lmax < 2^24");
+  AppendParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.k_new = k_new; p.v_new = v_new; p.kcache = kcache; p.vcache = vcache; p.pos = pos;
+  p.B = B; p.KV = KV; p.hd = hd; p.Lmax = Lmax;
+  p.rope = make_rope(hd, rope_base);
+  int err = 0;
+  p.status = device_status(&err);
+  if (!p.status) return err;
+  cudaError_t e = launch_kv_append(p, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_kv_append launch");
+  return ok();
+}
+
+namespace {
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+struct BlockLayout {
+  size_t q, k, v, ctx, total;
+};
+BlockLayout block_layout(int B, int T, int H, int KV, int hd, int dtype) {
+  const size_t es = elem_size(dtype);
+  BlockLayout L;
+  const size_t nq = (size_t)B * T * H * hd * es, nk = (size_t)B * T * KV * hd * es;
+  L.q = 0;
+  L.k = L.q + round256(nq);
+  L.v = L.k + round256(nk);
+  L.ctx = L.v + round256(nk);
+  L.total = L.ctx + round256(nq);
+  return L;
+}
+cudaError_t gemm(const void* A, const void* W, void* C, int M, int N, int K, int dtype, cudaStream_t s) {
+  if (gemm_tc_supported(M, N, K, dtype)) return launch_gemm_tc(A, W, C, M, N, K, s);
+  return launch_gemm_simt(A, W, C, M, N, K, dtype, s);
+}
+}  // namespace
+
+size_t attn_block_workspace_size(int B, int T, int d, int H, int KV, int hd, int dtype) {
+  if (B < 1 || T < 1 || d < 1 || H < 1 || KV < 1 || H % KV || hd < 2 ||
+      (dtype != ATTN_F32 && dtype != ATTN_BF16))
+    return 0;
+  return block_layout(B, T, H, KV, hd, dtype).total;
+}
+
+int attn_block(const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wo,
+               void* out, int B, int T, int d, int H, int KV, int hd, long long pos0,
+               float rope_base, int causal, int window, const float* alibi_slopes, int dtype,
+               void* workspace, size_t ws_bytes, void* stream) {
+  int st = check_common(H, KV, hd, dtype, rope_base);
+  if (st) return st;
+  if (!x || !Wq || !Wk || !Wv || !Wo || !out)
+    return fail(ATTN_ERR_ARG, "x, Wq, Wk, Wv, Wo and out must not be NULL");
+  if (!aligned16(x) || !aligned16(Wq) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(Wo) ||
+      !aligned16(out) || (workspace && !aligned16(workspace)))
+    return fail(ATTN_ERR_ALIGN, "x, weights, out and workspace must be 16-byte aligned");
+  if (B < 1 || T < 1 || d < 1) return fail(ATTN_ERR_ARG, "B, T and d must be >= 1");
+  const size_t need = attn_block_workspace_size(B, T, d, H, KV, hd, dtype);
+  if (!workspace || ws_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "block needs %zu bytes of workspace (got %zu)", need, ws_bytes);
+  const BlockLayout L = block_layout(B, T, H, KV, hd, dtype);
+  char* ws = static_cast<char*>(workspace);
+  void *q = ws + L.q, *k = ws + L.k, *v = ws + L.v, *ctx = ws + L.ctx;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int M = B * T;
+  cudaError_t e;
+  if ((e = gemm(x, Wq, q, M, H * hd, d, dtype, s)) != cudaSuccess) return cuda_fail(e, "block Wq GEMM");
+  if ((e = gemm(x, Wk, k, M, KV * hd, d, dtype, s)) != cudaSuccess) return cuda_fail(e, "block Wk GEMM");
+  if ((e = gemm(x, Wv, v, M, KV * hd, d, dtype, s)) != cudaSuccess) return cuda_fail(e, "block Wv GEMM");
+  st = attn_prefill(q, k, v, ctx, nullptr, B, T, H, KV, hd, pos0, rope_base, causal, window,
+                    alibi_slopes, dtype, stream);
+  if (st) return st;
+  if ((e = gemm(ctx, Wo, out, M, d, H * hd, dtype, s)) != cudaSuccess) return cuda_fail(e, "block Wo GEMM");
+  return ok();
+}
+
+void attn_alibi_slopes(int H, float* host_out) {
+  if (!host_out || H < 1) return;
+  for (int h = 0; h < H; ++h) host_out[h] = (float)std::pow(2.0, -8.0 * (h + 1.0) / H);
+}
+
+int attn_sync_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_sync_status: stream synchronise");
+  int err = 0;
+  int* ptr = device_status(&err);
+  if (!ptr) return err;
+  int word = 0;
+  if ((e = cudaMemcpy(&word, ptr, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "attn_sync_status: read");
+  if (word != 0) {
+    const int zero = 0;
+    if ((e = cudaMemcpy(ptr, &zero, sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess)
+      return cuda_fail(e, "attn_sync_status: clear");
+  }
+  if (word == DEV_TIMEOUT) return fail(ATTN_ERR_TIMEOUT, "a device-side wait gave up");
+  if (word == DEV_BAD_ARG)
+    return fail(ATTN_ERR_DEVICE_ARG, "a device-resident length or position was out of range");
+  return ok();
+}
+
+int attn_last_error(char* buf, size_t n) {
+  if (buf && n) {
+    std::strncpy(buf, g_msg, n - 1);
+    buf[n - 1] = '\0';
+  }
+  return g_last;
+}
+
+const char* attn_version(void) { return "alibi_rope_tile_b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

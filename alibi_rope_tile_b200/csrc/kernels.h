@@ -1,0 +1,76 @@
+// Host-side launchers of the attention-core kernels (internal; the C ABI is in
+// include/attn_rope_tile.h). Every launcher is asynchronous on the given stream and
+// returns the launch's cudaError_t.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "common.cuh"
+
+namespace attn {
+
+struct PrefillParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;       // [B,H,T] or nullptr
+  int B, T, H, KV, hd;
+  int pos0;         // position of row 0 (pos0 + T < 2^24)
+  int causal, window;
+  float scale;      // 1/sqrt(hd)
+  int* status;      // device error word
+  RopeFreqs rope;
+  Alibi alibi;
+};
+
+// CUDA-core flash prefill: fp32 or bf16 elements, any even hd <= 256.
+cudaError_t launch_prefill_simt(const PrefillParams& p, int dtype, cudaStream_t s);
+
+// Tensor-core (tcgen05 + TMEM + TMA) prefill: bf16, hd in {64, 128}.
+bool prefill_tc_supported(const PrefillParams& p, int dtype);
+cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t s);
+
+struct DecodeParams {
+  const void* q;        // [B,H,hd]
+  const void* kcache;   // [B,Lmax,KV,hd]
+  const void* vcache;
+  const int* seqlens;   // [B]
+  const int* qpos;      // [B]
+  void* out;            // [B,H,hd]
+  float* lse;           // [B,H] or nullptr
+  int B, H, KV, hd, Lmax;
+  int window;
+  float scale;
+  int* status;
+  RopeFreqs rope;
+  Alibi alibi;
+};
+
+// Split-KV geometry: keys per split and number of splits for these sizes.
+int decode_chunk(int B, int KV, int Lmax);
+size_t decode_workspace_bytes(int B, int H, int KV, int hd, int Lmax);
+cudaError_t launch_decode(const DecodeParams& p, int dtype, void* workspace, cudaStream_t s);
+
+struct AppendParams {
+  const void* k_new;
+  const void* v_new;
+  void* kcache;
+  void* vcache;
+  const int* pos;
+  int B, KV, hd, Lmax;
+  int* status;
+  RopeFreqs rope;
+};
+cudaError_t launch_kv_append(const AppendParams& p, int dtype, cudaStream_t s);
+
+// C[M,N] = A[M,K] @ W[K,N], row-major, fp32 accumulation, output in the input dtype.
+cudaError_t launch_gemm_simt(const void* A, const void* W, void* C, int M, int N, int K, int dtype,
+                             cudaStream_t s);
+// Tensor-core (tcgen05) version for bf16 when M, N, K fit its tiles.
+bool gemm_tc_supported(int M, int N, int K, int dtype);
+cudaError_t launch_gemm_tc(const void* A, const void* W, void* C, int M, int N, int K,
+                           cudaStream_t s);
+
+}  // namespace attn

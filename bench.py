@@ -1,0 +1,338 @@
+"""Benchmark of the attention core on B200: causal GQA prefill TFLOP/s and decode HBM GB/s.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  * prefill of the GQA workload (B=2, T=4096, H=32, KV=8, hd=128, causal, RoPE base 5e5):
+    RoPE on load, QK^T, mask, online softmax, PV, epilogue;
+  * one decode step of the KV-cache workload (batch 64, H=32, KV=8, hd=128, cache lengths
+    uniform in [1024, 8192]): split-KV partials and the log-sum-exp merge.
+``value`` is the prefill TFLOP/s (causal FLOPs counted: 4*B*H*hd*allowed pairs); the decode
+GB/s rides along under ``decode``. Kernels are timed with CUDA events on the stream they
+are launched on; L2 is flushed (a 256 MiB memset, outside the timed events) before every
+step. ``e2e`` times the same call with the step's inputs copied from pinned host memory and
+its output copied back, all inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank runs its own replica of the step (the path
+shards into independent problems; there is no data-path collective): value = all ranks'
+FLOPs / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+METRIC = "causal GQA prefill TFLOP/s and decode HBM GB/s on 1 B200, % of roofline"
+PREFILL = workloads.GQA
+DECODE = workloads.DECODE_GQA
+# Algorithmic bytes and launches, stated once (see the design notes):
+#   decode bytes = cache rows read (K and V) + q + out; prefill FLOPs = PREFILL.flops.
+PREFILL_LAUNCHES = 1
+DECODE_LAUNCHES = 2
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    return dict(PEAKS_FALLBACK)
+
+
+def decode_bytes(seqlens, w) -> int:
+    rows = int(seqlens.sum())
+    elt = 2
+    return rows * 2 * w.KV * w.hd * elt + 2 * w.B * w.H * w.hd * elt
+
+
+def dist_setup(n):
+    rank, world = int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+    if world != n and n > 1:
+        raise SystemExit(f"--gpus {n} but WORLD_SIZE={world}: launch with torchrun")
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", 0))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={device_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_tflops(budget_s: float = 12.0):
+    """The fp64 oracle on a bounded sample of the prefill workload (rows of the first
+    sequence, the four query heads of key/value head 0), as TFLOP/s of causal FLOPs."""
+    from oracle import attention as A
+    w = PREFILL
+    q, k, v = workloads.prefill_inputs(w)
+    q, k, v = q[:1, :, :4], k[:1, :, :1], v[:1, :, :1]
+    rows_all = torch.arange(w.T).numpy()
+    flops = done = 0
+    t0 = time.perf_counter()
+    chunk = 512
+    while time.perf_counter() - t0 < budget_s and done < w.T:
+        rows = rows_all[w.T - done - chunk: w.T - done] if done + chunk <= w.T else rows_all[:w.T - done]
+        A.attention(q, k, v, rope_base=w.rope_base, causal=True, rows=rows)
+        flops += 4 * 4 * w.hd * int((rows + 1).sum())
+        done += len(rows)
+    dt = time.perf_counter() - t0
+    sample = (f"GQA prefill, batch 0, query heads 0-3 (key/value head 0), last {done} of "
+              f"{w.T} rows, full key range, fp64 numpy/OpenBLAS")
+    return flops / dt / 1e12, dt, sample
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 CPU oracle, as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample_tflops(min(per_step, 3.0))
+    vals, secs, sample = [], 0.0, ""
+    for _ in range(args.steps):
+        v, dt, sample = oracle_sample_tflops(per_step)
+        vals.append(v)
+        secs += dt
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * secs / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": PREFILL.name, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world):
+    import alibi_rope_tile_b200 as art
+    art.lib()
+    dev = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+    w, dw = PREFILL, DECODE
+
+    q, k, v = workloads.prefill_inputs(w)
+    dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
+    dout = torch.empty_like(dq)
+    dq_, dkc, dvc, dsl, dqp = workloads.decode_inputs(dw)
+    dbytes = decode_bytes(dsl, dw)
+    ddq, dkc, dvc, dsl, dqp = dq_.cuda(), dkc.cuda(), dvc.cuda(), dsl.cuda(), dqp.cuda()
+    ddout = torch.empty_like(ddq)
+    ws = torch.empty(art.attn_decode_workspace_size(dw.B, dw.H, dw.KV, dw.hd, dw.Lmax),
+                     dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def prefill():
+        art.attn_prefill(dq, dk, dv, dout, rope_base=w.rope_base, causal=True, window=w.window)
+
+    def decode():
+        art.attn_decode(ddq, dkc, dvc, dsl, dqp, ddout, workspace=ws, rope_base=dw.rope_base)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        prefill()
+        decode()
+    torch.cuda.synchronize()
+    art.attn_sync_status()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = Clocks(dev)
+    time.sleep(0.3)
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_begin.record(stream)
+    for s in range(args.steps):
+        flush.zero_()
+        ev[s][0].record(stream)
+        prefill()
+        ev[s][1].record(stream)
+        ev[s][2].record(stream)
+        decode()
+        ev[s][3].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    art.attn_sync_status()
+    p_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
+    d_ms = [ev[s][2].elapsed_time(ev[s][3]) for s in range(args.steps)]
+    p_tot = max_over_ranks(sum(p_ms), world)
+    d_tot = max_over_ranks(sum(d_ms), world)
+    region_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
+
+    # end to end: pinned host inputs -> device -> prefill -> host output, every step
+    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
+        prefill()
+        hout.copy_(dout, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for _ in range(args.steps):
+        dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
+        prefill()
+        hout.copy_(dout, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+
+    pk = peaks()
+    flops_step = w.flops
+    tflops = world * flops_step * args.steps / (p_tot * 1e-3) / 1e12
+    per_launch_ms = p_tot / args.steps
+    achieved = flops_step / (per_launch_ms * 1e-3) / 1e12
+    d_gbs = world * dbytes * args.steps / (d_tot * 1e-3) / 1e9
+    d_per = d_tot / args.steps
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        with open(prof) as f:
+            traffic = json.load(f).get("prefill_tc")
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        val, dt, sample = oracle_sample_tflops()
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": sample, "seconds": round(dt, 2)}
+    line = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": (p_tot + d_tot) / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "decode_workload": dw.name, "parallelism": f"replicas{world}",
+                   "l2": "flushed: 256 MiB memset before every step, outside the kernel events",
+                   "timed_region_ms": region_ms},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
+                     "peak_source": f"{pk.get('source')} burst bf16 dense"},
+        "decode": {"value": d_gbs, "unit": "GB/s", "ms": d_per, "bytes": dbytes,
+                   "roofline": {"bound": "hbm", "achieved": dbytes / (d_per * 1e-3) / 1e9,
+                                "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                "frac": dbytes / (d_per * 1e-3) / 1e9 / pk["hbm_gbs"],
+                                "traffic": None, "peak_source": f"{pk.get('source')} copy"}},
+        "e2e": {"value": world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(3 * 0 + q.numel() * 2 + k.numel() * 2 + v.numel() * 2),
+                "d2h_bytes_per_step": int(q.numel() * 2)},
+        "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES),
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+/*
+ * attn_rope_tile.h -- C ABI of the B200 (sm_100a) attention core.
+ *
+ * The library computes the attention core of a decoder self-attention block,
+ *     out = softmax(Q K^T / sqrt(hd) + bias, masked) V,
+ * with grouped-query head sharing, interleaved rotary embeddings applied as the Q/K
+ * tiles are loaded, a causal mask with an optional sliding window, an optional ALiBi
+ * bias, a KV-cache decode step, and the projections of the surrounding block.
+ *
+ * Sources of the definitions (page title, then the place on the page):
+ *   [LAB]   "Write attention from scratch" (Inside the Model, lab 2): the worked
+ *           example (rope, softmax, attention), Properties 1 and 2, exercises 2-4.
+ *   [ALIBI] "Building a Multi-Head Self-Attention Block with RoPE and ALiBi from
+ *           Scratch": Step 1 (slopes), Step 3 "Implement ALiBi Bias", Step 4.
+ *   [FLASH] "Building grouped-query attention with RoPE and Flash Attention from
+ *           scratch": Step 3 (tiled online-softmax forward), roadmap (sliding window,
+ *           causal mask with KV cache, bf16 inputs with fp32 statistics).
+ *   [XF5]   "Building a Transformer from Scratch: Attention, Architecture, and Memory":
+ *           Part 1 step 2 (causal mask), Part 3 "KV caching", "FlashAttention" equations.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major, contiguous, caller-owned DEVICE buffers unless a
+ *     parameter says "host". The library never allocates, frees or keeps a pointer
+ *     after a call returns.
+ *   - Layouts: q and out [B, T, H, hd]; k and v [B, T, KV, hd]; decode q/out [B, H, hd];
+ *     caches [B, Lmax, KV, hd]; lse (log-sum-exp of each softmax row, natural log, fp32)
+ *     [B, H, T] for prefill and [B, H] for decode.
+ *   - dtype selects the element type of q, k, v, out, caches, x and weights (all the
+ *     same). Arithmetic is fp32 for either type; bf16 results are rounded to nearest
+ *     even. Statistics (running max and sum) are always fp32.
+ *   - Query head h reads key/value head h / (H / KV) ([LAB] np.repeat; [FLASH]).
+ *   - RoPE: rope_base > 0 turns interleaved pairs (2i, 2i+1) of q and k by the angle
+ *     p * rope_base^(-2i/hd) at position p ([LAB] rope). rope_base <= 0: no rotation.
+ *     Prefill positions are pos0 .. pos0+T-1; pos0 + T must stay below 2^24.
+ *   - Masks: causal keeps key j <= i ([LAB], [XF5]); window > 0 also requires
+ *     i - j < window (a window of W keys including the query's own) ([FLASH] roadmap,
+ *     [LAB] exercise 3). A masked pair has weight exactly zero.
+ *   - ALiBi: alibi_slopes (HOST pointer to H floats, copied at launch) adds
+ *     -slope_h * |i - j| to the scaled score ([ALIBI] Step 3); NULL turns it off.
+ *     attn_alibi_slopes() fills the schedule 2^(-8(h+1)/H).
+ *   - stream is a cudaStream_t (NULL: the legacy default stream). Calls are
+ *     asynchronous; the return value covers argument checks and launch errors. Errors
+ *     found on the device (an out-of-range cache position, a wait that gave up) are
+ *     recorded in a per-device error word read by attn_sync_status().
+ *   - Every call returns ATTN_OK (0) or a negative attn_status; attn_last_error() gives
+ *     a one-line message for the calling thread's last failure. Nothing aborts.
+ *   - Pointers must be 16-byte aligned; hd must be even and at most 256.
+ */
+#ifndef ATTN_ROPE_TILE_H
+#define ATTN_ROPE_TILE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_F32 = 0,   /* IEEE fp32 elements */
+  ATTN_BF16 = 1   /* bfloat16 elements */
+} attn_dtype;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_ARG = -1,          /* a size, flag or pointer is invalid */
+  ATTN_ERR_ALIGN = -2,        /* a pointer is not 16-byte aligned */
+  ATTN_ERR_UNSUPPORTED = -3,  /* a valid request this build does not implement */
+  ATTN_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed */
+  ATTN_ERR_TIMEOUT = -5,      /* a device-side wait gave up (reported by attn_sync_status) */
+  ATTN_ERR_WORKSPACE = -6,    /* workspace missing or smaller than the size query returned */
+  ATTN_ERR_DEVICE_ARG = -7    /* a device-resident argument was out of range (attn_sync_status) */
+} attn_status;
+
+/*
+ * attn_prefill -- causal (or full) attention of T query rows over the same T keys.
+ *
+ * Computes, for every batch b, query head h and row i, the softmax-weighted sum of the
+ * value rows of head g = h / (H/KV) over the allowed keys j ([LAB] attention(); the
+ * tiled online-softmax route of [FLASH] Step 3 reaches the same result):
+ *   s_ij = (R(pos0+i) q_i) . (R(pos0+j) k_j) / sqrt(hd) - slope_h |i - j|
+ *   out_i = sum_j softmax_j(s_ij) v_j,   lse_i = log sum_j exp(s_ij)
+ * q, k, v: inputs (device, read only). out: [B,T,H,hd] (device, written).
+ * lse: [B,H,T] fp32 (device, written) or NULL. B, T >= 1; H % KV == 0.
+ * causal: 0 or 1. window: <= 0 none, else W >= 1 (requires causal).
+ * bf16 with hd in {64, 128} runs the tensor-core (tcgen05/TMEM) kernel; other shapes
+ * and fp32 run the CUDA-core kernel. Returns ATTN_OK or an attn_status.
+ */
+int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse,
+                 int B, int T, int H, int KV, int hd, long long pos0, float rope_base,
+                 int causal, int window, const float* alibi_slopes, int dtype, void* stream);
+
+/*
+ * attn_decode_workspace_size -- bytes of device scratch attn_decode needs for these
+ * sizes (split-KV partial outputs and their softmax statistics). Returns 0 on invalid
+ * sizes.
+ */
+size_t attn_decode_workspace_size(int B, int H, int KV, int hd, int Lmax);
+
+/*
+ * attn_decode -- one decode step per sequence over a KV cache ([XF5] "KV caching";
+ * [LAB] exercise 2: token-by-token decode equals the full causal computation).
+ *
+ * q: [B,H,hd] new-token queries BEFORE rotation; the kernel turns query b at position
+ * qpos[b]. kcache, vcache: [B,Lmax,KV,hd]; slot j holds the key already rotated at
+ * position j (attn_kv_append writes it that way). seqlens: [B] int32 (device): the
+ * query attends to slots 0..seqlens[b]-1; window > 0 also requires qpos - j < window.
+ * qpos: [B] int32 (device). A sequence with seqlens[b] == 0 gets out = 0, lse = -inf.
+ * out: [B,H,hd] (device, written). lse: [B,H] fp32 or NULL.
+ * workspace: device scratch of at least attn_decode_workspace_size(B,H,KV,hd,Lmax)
+ * bytes, owned by the caller; its contents on entry do not matter.
+ * seqlens[b] > Lmax or qpos[b] < 0 is recorded as ATTN_ERR_DEVICE_ARG (read it with
+ * attn_sync_status) and that sequence's output is zeroed.
+ * Two kernels run on stream: split-KV partials (each CTA reads its cache rows once with
+ * 16-byte loads for all H/KV query heads of a key/value head), then a log-sum-exp merge.
+ */
+int attn_decode(const void* q, const void* kcache, const void* vcache, const int* seqlens,
+                const int* qpos, void* out, float* lse, int B, int H, int KV, int hd, int Lmax,
+                float rope_base, int window, const float* alibi_slopes, int dtype,
+                void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * attn_kv_append -- write one new token per sequence into the cache ([XF5] "KV caching";
+ * [FLASH] roadmap: preallocate the cache and write by position).
+ * k_new, v_new: [B,KV,hd] (device). pos: [B] int32 (device) slot = position of the token.
+ * The key is rotated at pos[b] (if rope_base > 0) before it is stored; the value is
+ * stored as is. pos[b] outside [0, Lmax) is recorded as ATTN_ERR_DEVICE_ARG and skipped.
+ */
+int attn_kv_append(const void* k_new, const void* v_new, void* kcache, void* vcache,
+                   const int* pos, int B, int KV, int hd, int Lmax, float rope_base, int dtype,
+                   void* stream);
+
+/*
+ * attn_block_workspace_size -- bytes of device scratch attn_block needs (the q, k, v and
+ * context activations). Returns 0 on invalid sizes.
+ */
+size_t attn_block_workspace_size(int B, int T, int d, int H, int KV, int hd, int dtype);
+
+/*
+ * attn_block -- the attention block of [LAB] attention(): q = x Wq, k = x Wk, v = x Wv
+ * (weights [in, out], applied as x @ W; head h is columns h*hd..h*hd+hd-1), then
+ * attn_prefill on them, then out = ctx Wo. No bias, residual or normalisation.
+ * x: [B,T,d]; Wq: [d, H*hd]; Wk, Wv: [d, KV*hd]; Wo: [H*hd, d]; out: [B,T,d].
+ * workspace: at least attn_block_workspace_size(...) bytes (device, caller-owned).
+ * Intermediate activations are stored in dtype.
+ */
+int attn_block(const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wo,
+               void* out, int B, int T, int d, int H, int KV, int hd, long long pos0,
+               float rope_base, int causal, int window, const float* alibi_slopes, int dtype,
+               void* workspace, size_t ws_bytes, void* stream);
+
+/* attn_alibi_slopes -- host_out[h] = 2^(-8(h+1)/H) for h < H ([ALIBI] Step 1; the slope
+ * schedule with exponent 8/H). host_out is a HOST buffer of H floats. */
+void attn_alibi_slopes(int H, float* host_out);
+
+/* attn_sync_status -- synchronise stream, then read and clear this device's error word.
+ * Returns ATTN_OK, ATTN_ERR_TIMEOUT, ATTN_ERR_DEVICE_ARG or ATTN_ERR_CUDA. */
+int attn_sync_status(void* stream);
+
+/* attn_last_error -- copy the calling thread's last error message (NUL-terminated,
+ * truncated to n bytes) into buf; returns the last status. */
+int attn_last_error(char* buf, size_t n);
+
+/* attn_version -- static version string of the library. */
+const char* attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_ROPE_TILE_H */

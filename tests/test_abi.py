@@ -1,0 +1,125 @@
+"""The C-ABI library builds for sm_100a, loads, and exports every symbol its header declares.
+
+No compute call runs here (there is no GPU): only host-side entry points and argument
+checks that return before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_rope_tile.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from alibi_rope_tile_b200 import build
+    path = build.build()
+    import alibi_rope_tile_b200 as art
+    assert os.path.samefile(path, art.LIB_PATH)
+    return art.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for must in ("attn_prefill", "attn_decode", "attn_block", "attn_kv_append",
+                 "attn_decode_workspace_size", "attn_block_workspace_size", "attn_alibi_slopes",
+                 "attn_sync_status", "attn_last_error", "attn_version"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    import alibi_rope_tile_b200 as art
+    names = declared_functions()
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in the header but not exported"
+    assert sorted(art.SIGNATURES) == names, "binding and header disagree on the entry points"
+
+
+def test_library_is_sm100a_only():
+    from alibi_rope_tile_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_alibi_slopes_host(lib, golden_dir):
+    import alibi_rope_tile_b200 as art
+    with open(os.path.join(golden_dir, "alibi_slopes.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    for H, h, val in rows:
+        assert art.alibi_slopes(int(H))[int(h)] == pytest.approx(float(val), rel=1e-7)
+
+
+def test_version(lib):
+    import alibi_rope_tile_b200 as art
+    assert "sm_100a" in art.attn_version()
+
+
+def test_workspace_sizes(lib):
+    import alibi_rope_tile_b200 as art
+    assert art.attn_decode_workspace_size(64, 32, 8, 128, 8192) > 0
+    assert art.attn_decode_workspace_size(1, 3, 2, 8, 16) == 0          # H % KV != 0
+    n = art.attn_block_workspace_size(1, 6, 32, 4, 2, 8, art.ATTN_F32)
+    assert n >= 4 * (6 * 32 + 6 * 16 + 6 * 16 + 6 * 32)
+    assert art.attn_block_workspace_size(1, 6, 32, 4, 2, 8, 7) == 0      # bad dtype
+
+
+def _call_prefill(lib, **kw):
+    a = dict(q=0x1000, k=0x1000, v=0x1000, out=0x1000, lse=None, B=1, T=8, H=4, KV=2, hd=8,
+             pos0=0, base=10000.0, causal=1, window=0, slopes=None, dtype=1, stream=None)
+    a.update(kw)
+    return lib.attn_prefill(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["T"], a["H"],
+                            a["KV"], a["hd"], a["pos0"], a["base"], a["causal"], a["window"],
+                            a["slopes"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(H=6, KV=4), -1),             # H not a multiple of KV
+    (dict(hd=7), -1),                  # odd head dimension
+    (dict(hd=512), -1),                # beyond the maximum head dimension
+    (dict(q=None), -1),                # NULL pointer
+    (dict(k=0x1008), -2),              # not 16-byte aligned
+    (dict(T=0), -1),                   # empty sequence
+    (dict(causal=0, window=4), -1),    # window without the causal mask
+    (dict(pos0=(1 << 24)), -1),        # positions beyond 2^24
+    (dict(dtype=5), -1),               # unknown dtype
+])
+def test_prefill_argument_errors(lib, kw, code):
+    import alibi_rope_tile_b200 as art
+    assert _call_prefill(lib, **kw) == code
+    buf = ctypes.create_string_buffer(256)
+    assert lib.attn_last_error(buf, 256) == code
+    assert len(buf.value) > 0
+    with pytest.raises(art.AttnError):
+        art._check(code)
+
+
+def test_decode_workspace_error(lib):
+    n = lib.attn_decode_workspace_size(2, 4, 2, 64, 128)
+    st = lib.attn_decode(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, 2, 4, 2, 64, 128,
+                         10000.0, 0, None, 1, 0x1000, n - 1, None)
+    assert st == -6
+    st = lib.attn_decode(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, 2, 4, 2, 48, 128,
+                         10000.0, 0, None, 1, 0x1000, 1 << 30, None)
+    assert st == -3      # hd = 48 is not a decode head size
+
+
+def test_block_workspace_error(lib):
+    st = lib.attn_block(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 1, 6, 32, 4, 2, 8, 0,
+                        10000.0, 1, 0, None, 0, 0x1000, 16, None)
+    assert st == -6
+
+
+def test_binding_requires_cuda_tensors(lib):
+    import torch
+    import alibi_rope_tile_b200 as art
+    q = torch.zeros(1, 4, 2, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        art.attn_prefill(q, q, q, out=q)

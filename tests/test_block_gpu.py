@@ -1,0 +1,63 @@
+"""Block parity on the GPU: projections + attention + output projection vs the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import attention as A
+from tests._gpu_util import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def art():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import alibi_rope_tile_b200 as m
+    m.lib()
+    return m
+
+
+def run_block(art, w, x, pos0, **kw):
+    return art.attn_block(x.cuda(), w["Wq"].cuda(), w["Wk"].cuda(), w["Wv"].cuda(),
+                          w["Wo"].cuda(), pos0=pos0, **kw)
+
+
+@pytest.mark.parametrize("pos0", [0, 100])
+def test_tiny_block_fp32(art, pos0):
+    """The lab's worked example on the GPU, fp32, within 1e-5 of the fp64 oracle."""
+    cfg = workloads.TINY_BLOCK
+    w = {n: torch.from_numpy(a) for n, a in workloads.tiny_block_inputs(cfg.seed).items()}
+    out = run_block(art, w, w["x"][None], pos0, H=cfg.H, KV=cfg.KV, rope_base=cfg.rope_base)
+    ref = A.block(w["x"][None], w["Wq"], w["Wk"], w["Wv"], w["Wo"], H=cfg.H, KV=cfg.KV,
+                  pos0=pos0, rope_base=cfg.rope_base)
+    assert_close(out, ref, torch.float32, f"tiny block pos0={pos0}")
+
+
+def test_tiny_block_lab_properties_on_gpu(art):
+    """Property 1 bit-exact on the GPU; Property 2 within the fp32 bar."""
+    cfg = workloads.TINY_BLOCK
+    w = {n: torch.from_numpy(a) for n, a in workloads.tiny_block_inputs(cfg.seed).items()}
+    kw = dict(H=cfg.H, KV=cfg.KV, rope_base=cfg.rope_base)
+    out = run_block(art, w, w["x"][None], 0, **kw)
+    x2 = w["x"].clone()
+    x2[-1] += 1.0
+    out2 = run_block(art, w, x2[None], 0, **kw)
+    assert torch.equal(out[0, :-1], out2[0, :-1])
+    out3 = run_block(art, w, w["x"][None], 100, **kw)
+    assert (out3 - out).abs().max().item() <= 1e-5
+
+
+@pytest.mark.parametrize("shape", [(2, 256, 512, 8, 2), (1, 300, 256, 4, 4)])
+def test_bf16_block(art, shape):
+    B, T, d, H, KV = shape
+    hd = d // H
+    g = torch.Generator().manual_seed(31)
+    x = workloads.normal((B, T, d), 0, torch.bfloat16, g)
+    W = {n: (torch.randn(*s, generator=g) / np.sqrt(d)).to(torch.bfloat16)
+         for n, s in (("Wq", (d, H * hd)), ("Wk", (d, KV * hd)), ("Wv", (d, KV * hd)),
+                      ("Wo", (H * hd, d)))}
+    out = run_block(art, W, x, 0, H=H, KV=KV, rope_base=10000.0)
+    ref = A.block(x, W["Wq"], W["Wk"], W["Wv"], W["Wo"], H=H, KV=KV, rope_base=10000.0)
+    assert_close(out, ref, torch.bfloat16, f"bf16 block {shape}")
