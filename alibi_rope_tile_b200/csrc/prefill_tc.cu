@@ -1,8 +1,468 @@
-// Tensor-core prefill (tcgen05 + TMEM + TMA): not built yet; every request takes the
-// CUDA-core kernel.
+// Tensor-core flash prefill for sm_100a: TMA-staged tiles, tcgen05 MMAs accumulating in
+// TMEM, warp-specialised online softmax, rotary embedding applied as tiles land.
+//
+// What it computes is the attention core of "Write attention from scratch" (worked
+// example): per query row i, softmax over allowed keys j of
+//   (R(pos0+i) q_i . R(pos0+j) k_j) / sqrt(hd) - slope_h |i - j|
+// weighting the value rows, reached through the key-block recurrences of "Building
+// grouped-query attention with RoPE and Flash Attention from scratch" (Step 3): a running
+// maximum, a running denominator and a rescaled output accumulator.
+//
+// Work unit (one CTA): two "slots" of 128 query rows that read the same key/value head:
+//   * H/KV even: two query heads of one group at the same rows (GQA sharing);
+//   * H/KV odd (MHA included): one head, two consecutive 128-row tiles.
+// Both slots consume every key/value tile the CTA loads, so each tile is fetched and
+// rotated once per 256 query rows. CTAs are numbered longest-first (causal rows near the
+// end see the most keys) so the block scheduler packs them like an LPT schedule.
+//
+// Warp roles (14 warps):
+//   warps 0-3  softmax of slot 0 (thread = query row = TMEM lane)
+//   warps 4-7  softmax of slot 1
+//   warps 8-11 rotary embedding: turns the two Q tiles once, then every K tile in place
+//              in its 128-byte-swizzled shared-memory layout (RoPE on load)
+//   warp 12    TMA producer (Q tiles, then K/V tiles through a ring of NS stages)
+//   warp 13    TMEM allocation and UMMA issue
+// Tensor memory (512 columns): S0 | S1 (128 fp32 columns each) | O0 | O1 (hd each).
+// P (bf16) goes through shared memory, so an S buffer can be refilled as soon as its
+// softmax has read it. Issue order per key tile j: PV0(j), QK0(j+1), PV1(j), QK1(j+1):
+// the tensor core works on one slot while the other slot's softmax runs.
+//
+// Masking: a pair outside the causal/window/length limits gets -inf before the row max,
+// so its weight is exactly 0, and the sums' order depends only on the tile structure;
+// a row's output never depends on the keys it may not see. Tiles outside a slot's key
+// range are skipped entirely.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace attn {
-bool prefill_tc_supported(const PrefillParams&, int) { return false; }
-cudaError_t launch_prefill_tc(const PrefillParams&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace tc {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int NUM_WARPS = 14;
+constexpr int NUM_THREADS = NUM_WARPS * 32;
+constexpr int WARP_ROPE0 = 8;
+constexpr int WARP_TMA = 12;
+constexpr int WARP_MMA = 13;
+constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;  // a wait that lasts 4 s has failed
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+template <int HD>
+struct Cfg {
+  static constexpr int NS = HD == 128 ? 3 : 6;  // key/value ring stages
+  static constexpr int Q_BYTES = BM * HD * 2;
+  static constexpr int P_BYTES = BM * BN * 2;
+  static constexpr int KV_BYTES = BN * HD * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_KV = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
+  static constexpr int NBAR = 3 * NS + 8;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KiB
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, 0, 1);
+};
+
+struct TcArgs {
+  PrefillParams p;
+  int group;       // H / KV
+  int two_heads;   // 1: slots are two heads at the same rows; 0: one head, two row tiles
+  int npairs;      // slot pairs per key/value head
+  int nqb;         // query blocks per (sequence, pair)
+  float scale_log2;
+};
+
+// Turn the interleaved pairs of one 128-byte-swizzled bf16 row in place.
+template <int HD>
+__device__ __forceinline__ void rotate_row(uint8_t* tile, int row, int pos, const RopeFreqs& rope) {
+#pragma unroll 4
+  for (int c = 0; c < HD / 8; ++c) {
+    uint4* ptr = reinterpret_cast<uint4*>(tile + sw128_offset(row, c * 8, BM));
+    uint4 u = *ptr;
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int pc = c * 4 + e;
+      const float t = rope_turns(pos, rope.hi[pc], rope.lo[pc]);
+      float sn, cs;
+      __sincosf(t * 6.283185307179586f, &sn, &cs);
+      float2 f = bf2_to_f2(w[e]);
+      rotate_pair(f.x, f.y, cs, sn);
+      w[e] = f2_to_bf2(f.x, f.y);
+    }
+    *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ TcArgs a) {
+  using C = Cfg<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sP = smem + C::OFF_P;
+  uint8_t* sKV = smem + C::OFF_KV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + C::NS;
+  uint64_t* k_rot = bars + 2 * C::NS;
+  uint64_t* q_full = bars + 3 * C::NS;
+  uint64_t* q_rot = q_full + 1;
+  uint64_t* s_full = q_full + 2;
+  uint64_t* p_full = q_full + 4;
+  uint64_t* o_done = q_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const PrefillParams& p = a.p;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- work unit: longest rows first
+  const int per_qb = p.B * p.KV * a.npairs;
+  const int qb = a.nqb - 1 - (int)(blockIdx.x / per_qb);
+  int rest = blockIdx.x % per_qb;
+  const int pair = rest % a.npairs;
+  rest /= a.npairs;
+  const int g = rest % p.KV;
+  const int b = rest / p.KV;
+  int head[2], qs[2];
+  if (a.two_heads) {
+    head[0] = g * a.group + 2 * pair;
+    head[1] = head[0] + 1;
+    qs[0] = qs[1] = qb * BM;
+  } else {
+    head[0] = head[1] = g * a.group + pair;
+    qs[0] = qb * 2 * BM;
+    qs[1] = qs[0] + BM;
+  }
+  int t0[2], t1[2];
+  bool valid[2];
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    valid[s] = qs[s] < p.T;
+    const int lo = p.window > 0 ? max(0, qs[s] - p.window + 1) : 0;
+    const int hi = p.causal ? min(p.T - 1, qs[s] + BM - 1) : p.T - 1;
+    t0[s] = valid[s] ? lo / BN : 1;
+    t1[s] = valid[s] ? hi / BN : 0;
+  }
+  const int jt0 = valid[1] ? min(t0[0], t0[1]) : t0[0];
+  const int jt1 = valid[1] ? max(t1[0], t1[1]) : t1[0];
+  auto active = [&](int s, int j) { return valid[s] && j >= t0[s] && j <= t1[s]; };
+
+  // ---- set-up: barriers, tensor memory
+  if (tid == 0) {
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(kv_full + i, 1);
+      mbar_init(kv_empty + i, 1);
+      mbar_init(k_rot + i, 128);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_rot, 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full + s, 1);
+      mbar_init(p_full + s, 128);
+      mbar_init(o_done + s, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == WARP_TMA) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch(&tmQ);
+      tma_prefetch(&tmK);
+      tma_prefetch(&tmV);
+      const uint32_t qbytes = (valid[0] ? C::Q_BYTES : 0) + (valid[1] ? C::Q_BYTES : 0);
+      mbar_expect_tx(q_full, qbytes);
+      for (int s = 0; s < 2; ++s)
+        if (valid[s])
+          for (int kb = 0; kb < HD / 64; ++kb)
+            tma_load_4d(sQ + s * C::Q_BYTES + kb * BM * 128, &tmQ, q_full, kb * 64, head[s], qs[s], b);
+      int u = 0;
+      for (int j = jt0; j <= jt1; ++j) {
+        for (int kv = 0; kv < 2; ++kv, ++u) {
+          const int st = u % C::NS, n = u / C::NS;
+          if (!mbar_wait(kv_empty + st, (n & 1) ^ 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+          mbar_expect_tx(kv_full + st, C::KV_BYTES);
+          for (int kb = 0; kb < HD / 64; ++kb)
+            tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, kv ? &tmV : &tmK, kv_full + st,
+                        kb * 64, g, j * BN, b);
+        }
+      }
+    }
+  } else if (warp >= WARP_ROPE0 && warp < WARP_ROPE0 + 4) {
+    // ------------------------------------------------------------ rotary embedding
+    const int r = tid - WARP_ROPE0 * 32;  // row of the tile this thread turns
+    if (!mbar_wait(q_full, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+    if (p.rope.on)
+      for (int s = 0; s < 2; ++s)
+        if (valid[s]) rotate_row<HD>(sQ + s * C::Q_BYTES, r, p.pos0 + qs[s] + r, p.rope);
+    fence_proxy_async();
+    mbar_arrive(q_rot);
+    int u = 0;
+    for (int j = jt0; j <= jt1; ++j) {
+      for (int kv = 0; kv < 2; ++kv, ++u) {
+        const int st = u % C::NS, n = u / C::NS;
+        if (!mbar_wait(kv_full + st, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        if (kv == 0 && p.rope.on) rotate_row<HD>(sKV + st * C::KV_BYTES, r, p.pos0 + j * BN + r, p.rope);
+        fence_proxy_async();
+        mbar_arrive(k_rot + st);
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    // ------------------------------------------------------------ UMMA issue
+    if (lane == 0) {
+      const uint32_t aQ = smem_u32(sQ), aP = smem_u32(sP), aKV = smem_u32(sKV);
+      auto issue_qk = [&](int s, int st) {
+        const uint32_t d = tmem + s * BN;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          umma_ss(d, smem_desc_sw128(aQ + s * C::Q_BYTES + off, 16, 1024),
+                  smem_desc_sw128(aKV + st * C::KV_BYTES + off, 16, 1024), C::IDESC_QK, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int s, int st, bool acc) {
+        const uint32_t d = tmem + 2 * BN + s * HD;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t offp = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          umma_ss(d, smem_desc_sw128(aP + s * C::P_BYTES + offp, 16, 1024),
+                  smem_desc_sw128(aKV + st * C::KV_BYTES + kk * 16 * 128, BN * 128, 1024),
+                  C::IDESC_PV, (kk > 0 || acc) ? 1u : 0u);
+        }
+      };
+      int cnt[2] = {0, 0};
+      if (!mbar_wait(q_rot, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      // K of the first tile
+      if (!mbar_wait(k_rot + 0, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      tc_fence_after();
+      for (int s = 0; s < 2; ++s)
+        if (active(s, jt0)) {
+          issue_qk(s, 0);
+          umma_commit(s_full + s);
+        }
+      umma_commit(kv_empty + 0);
+      for (int j = jt0; j <= jt1; ++j) {
+        const int uV = 2 * (j - jt0) + 1, stV = uV % C::NS;
+        const int uK = uV + 1, stK = uK % C::NS;
+        const bool next = j < jt1;
+        if (!mbar_wait(k_rot + stV, (uV / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        for (int s = 0; s < 2; ++s) {
+          if (active(s, j)) {
+            if (!mbar_wait(p_full + s, cnt[s] & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+            tc_fence_after();
+            issue_pv(s, stV, cnt[s] > 0);
+            umma_commit(o_done + s);
+            ++cnt[s];
+          }
+          if (next && s == 0) {
+            if (!mbar_wait(k_rot + stK, (uK / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+            tc_fence_after();
+          }
+          if (next && active(s, j + 1)) {
+            issue_qk(s, stK);
+            umma_commit(s_full + s);
+          }
+        }
+        umma_commit(kv_empty + stV);
+        if (next) umma_commit(kv_empty + stK);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (warps 0-7)
+    const int s = warp >> 2;
+    const int r = tid & 127;
+    const int i = qs[s] + r;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + s * BN;
+    const uint32_t tO = tmem + lane_off + 2 * BN + s * HD;
+    uint8_t* myP = sP + s * C::P_BYTES;
+    const float slope = p.alibi.on ? p.alibi.slope[head[s]] * LOG2E : 0.f;
+    float m = -INFINITY, l = 0.f;
+    int c = 0;
+    if (valid[s]) {
+      for (int j = t0[s]; j <= t1[s]; ++j, ++c) {
+        if (!mbar_wait(s_full + s, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        tc_fence_after();
+        float x[BN];
+#pragma unroll
+        for (int q4 = 0; q4 < BN / 32; ++q4) {
+          float (&xx)[32] = *reinterpret_cast<float(*)[32]>(&x[q4 * 32]);
+          tmem_ld32(tS + q4 * 32, xx);
+        }
+        tmem_wait_ld();
+        const int key0 = j * BN;
+        // does any row of this slot need per-element masking in this tile?
+        const bool need_mask = (key0 + BN > p.T) ||
+                               (p.causal && key0 + BN - 1 > qs[s]) ||
+                               (p.window > 0 && qs[s] + BM - 1 - key0 >= p.window);
+        float mt = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < BN; ++k) {
+          float v = x[k] * a.scale_log2;
+          if (p.alibi.on) v -= slope * fabsf((float)(i - (key0 + k)));
+          if (need_mask) {
+            const int jk = key0 + k;
+            const bool ok = jk < p.T && (!p.causal || jk <= i) && (p.window <= 0 || i - jk < p.window);
+            v = ok ? v : -INFINITY;
+          }
+          x[k] = v;
+          mt = fmaxf(mt, v);
+        }
+        const float m_new = fmaxf(m, mt);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = ex2(m - m_use);
+        uint32_t pk[BN / 2];
+        float rs = 0.f;
+#pragma unroll
+        for (int k = 0; k < BN / 2; ++k) {
+          const float e0 = ex2(x[2 * k] - m_use), e1 = ex2(x[2 * k + 1] - m_use);
+          rs += e0 + e1;
+          pk[k] = f2_to_bf2(e0, e1);
+        }
+        l = l * alpha + rs;
+        m = m_new;
+        if (c > 0) {
+          // the previous PV must finish before O is rescaled and P is overwritten
+          if (!mbar_wait(o_done + s, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+            for (int q4 = 0; q4 < HD / 32; ++q4) {
+              float o[32];
+              tmem_ld32(tO + q4 * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] *= alpha;
+              tmem_st32(tO + q4 * 32, o);
+            }
+            tmem_wait_st();
+          }
+        }
+#pragma unroll
+        for (int c8 = 0; c8 < BN / 8; ++c8) {
+          uint4* dst = reinterpret_cast<uint4*>(myP + sw128_offset(r, c8 * 8, BM));
+          *dst = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(p_full + s);
+      }
+      if (c > 0) {
+        if (!mbar_wait(o_done + s, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
+                              (((size_t)b * p.T + i) * p.H + head[s]) * HD;
+#pragma unroll
+        for (int q4 = 0; q4 < HD / 32; ++q4) {
+          float o[32];
+          tmem_ld32(tO + q4 * 32, o);
+          tmem_wait_ld();
+          if (i < p.T) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(f2_to_bf2(o[8 * v4] * inv, o[8 * v4 + 1] * inv),
+                                   f2_to_bf2(o[8 * v4 + 2] * inv, o[8 * v4 + 3] * inv),
+                                   f2_to_bf2(o[8 * v4 + 4] * inv, o[8 * v4 + 5] * inv),
+                                   f2_to_bf2(o[8 * v4 + 6] * inv, o[8 * v4 + 7] * inv));
+          }
+        }
+        if (p.lse && i < p.T)
+          p.lse[((size_t)b * p.H + head[s]) * p.T + i] = l > 0.f ? (m + __log2f(l)) * LN2 : -INFINITY;
+      }
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 4-D map over [B][T][heads][hd] bf16 with a box of 128 rows x 64 features of one head.
+bool make_map(CUtensorMap* map, const void* base, int B, int T, int heads, int hd) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)hd * 2, (cuuint64_t)heads * hd * 2,
+                                 (cuuint64_t)T * heads * hd * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int HD>
+cudaError_t launch_hd(const PrefillParams& p, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, p.q, p.B, p.T, p.H, HD) || !make_map(&mk, p.k, p.B, p.T, p.KV, HD) ||
+      !make_map(&mv, p.v, p.B, p.T, p.KV, HD))
+    return cudaErrorInvalidValue;
+  TcArgs a;
+  a.p = p;
+  a.group = p.H / p.KV;
+  a.two_heads = (a.group % 2 == 0) ? 1 : 0;
+  a.npairs = a.two_heads ? a.group / 2 : a.group;
+  const int rows = a.two_heads ? BM : 2 * BM;
+  a.nqb = (p.T + rows - 1) / rows;
+  a.scale_log2 = p.scale * LOG2E;
+  const long long units = (long long)p.B * p.KV * a.npairs * a.nqb;
+  if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg<HD>::SMEM);
+  if (e != cudaSuccess) return e;
+  prefill_tc_kernel<HD><<<(unsigned)units, NUM_THREADS, Cfg<HD>::SMEM, s>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace tc
+
+bool prefill_tc_supported(const PrefillParams& p, int dtype) {
+  return dtype == 1 && (p.hd == 64 || p.hd == 128) && tc::encode_fn() != nullptr;
+}
+
+cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t s) {
+  return p.hd == 128 ? tc::launch_hd<128>(p, s) : tc::launch_hd<64>(p, s);
+}
+
 }  // namespace attn
