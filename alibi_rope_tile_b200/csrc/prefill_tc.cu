@@ -79,10 +79,11 @@ struct TcArgs {
   float scale_log2;
 };
 
-// Turn the interleaved pairs of one 128-byte-swizzled bf16 row in place.
+// Turn the interleaved pairs of one 128-byte-swizzled bf16 row in place (accurate angle
+// for every pair; used once per CTA for the query tiles).
 template <int HD>
 __device__ __forceinline__ void rotate_row(uint8_t* tile, int row, int pos, const RopeFreqs& rope) {
-#pragma unroll 4
+#pragma unroll 2
   for (int c = 0; c < HD / 8; ++c) {
     uint4* ptr = reinterpret_cast<uint4*>(tile + sw128_offset(row, c * 8, BM));
     uint4 u = *ptr;
@@ -90,9 +91,8 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int row, int pos, cons
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int pc = c * 4 + e;
-      const float t = rope_turns(pos, rope.hi[pc], rope.lo[pc]);
       float sn, cs;
-      __sincosf(t * 6.283185307179586f, &sn, &cs);
+      rope_cos_sin(pos, rope.hi[pc], rope.lo[pc], cs, sn);
       float2 f = bf2_to_f2(w[e]);
       rotate_pair(f.x, f.y, cs, sn);
       w[e] = f2_to_bf2(f.x, f.y);
@@ -100,6 +100,57 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int row, int pos, cons
     *ptr = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
+
+// Rotation of a whole key tile by the 128 threads of the rotary warpgroup. Thread t owns
+// one 16-byte chunk (4 pairs) of the row and the rows phase, phase + PH, phase + 2 PH ...
+// Along those rows the angle of a pair grows by the fixed step PH * w, so the cosine and
+// sine follow the angle-addition recurrence (c, s) <- (c C - s S, s C + c S) with (C, S)
+// the step's cosine and sine, computed once per CTA. The start angle of each tile is
+// computed accurately, so rounding can build up over at most NR - 1 steps. Eight threads
+// of a quarter warp cover the 8 chunks of one 128-byte row: shared-memory accesses are
+// free of bank conflicts. Only FMA-pipe arithmetic runs per element.
+template <int HD>
+struct KRot {
+  static constexpr int CH = HD / 8;       // 16-byte chunks per row
+  static constexpr int PH = 128 / CH;     // row step between a thread's rows
+  static constexpr int NR = BN / PH;      // rows per thread
+  int chunk, phase;
+  float stepc[4], steps[4];
+  __device__ __forceinline__ void init(int t, const RopeFreqs& rope) {
+    chunk = t % CH;
+    phase = t / CH;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int pc = chunk * 4 + e;
+      rope_cos_sin(PH, rope.hi[pc], rope.lo[pc], stepc[e], steps[e]);
+    }
+  }
+  __device__ __forceinline__ void rotate(uint8_t* tile, int pos_row0, const RopeFreqs& rope) const {
+    float c[4], s[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int pc = chunk * 4 + e;
+      rope_cos_sin(pos_row0 + phase, rope.hi[pc], rope.lo[pc], c[e], s[e]);
+    }
+#pragma unroll 4
+    for (int k = 0; k < NR; ++k) {
+      const int r = phase + PH * k;
+      uint4* ptr = reinterpret_cast<uint4*>(tile + sw128_offset(r, chunk * 8, BN));
+      uint4 u = *ptr;
+      uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float2 f = bf2_to_f2(w[e]);
+        rotate_pair(f.x, f.y, c[e], s[e]);
+        w[e] = f2_to_bf2(f.x, f.y);
+        const float cn = c[e] * stepc[e] - s[e] * steps[e];
+        s[e] = s[e] * stepc[e] + c[e] * steps[e];
+        c[e] = cn;
+      }
+      *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+};
 
 template <int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -210,7 +261,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= WARP_ROPE0 && warp < WARP_ROPE0 + 4) {
     // ------------------------------------------------------------ rotary embedding
-    const int r = tid - WARP_ROPE0 * 32;  // row of the tile this thread turns
+    const int r = tid - WARP_ROPE0 * 32;  // row of a query tile this thread turns
+    KRot<HD> krot;
+    if (p.rope.on) krot.init(r, p.rope);
     if (!mbar_wait(q_full, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
     if (p.rope.on)
       for (int s = 0; s < 2; ++s)
@@ -222,7 +275,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int kv = 0; kv < 2; ++kv, ++u) {
         const int st = u % C::NS, n = u / C::NS;
         if (!mbar_wait(kv_full + st, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        if (kv == 0 && p.rope.on) rotate_row<HD>(sKV + st * C::KV_BYTES, r, p.pos0 + j * BN + r, p.rope);
+        if (kv == 0 && p.rope.on) krot.rotate(sKV + st * C::KV_BYTES, p.pos0 + j * BN, p.rope);
         fence_proxy_async();
         mbar_arrive(k_rot + st);
       }
@@ -297,50 +350,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tO = tmem + lane_off + 2 * BN + s * HD;
     uint8_t* myP = sP + s * C::P_BYTES;
     const float slope = p.alibi.on ? p.alibi.slope[head[s]] * LOG2E : 0.f;
-    float m = -INFINITY, l = 0.f;
+    const float sc = a.scale_log2;
+    // Row state in the log2 domain: m_ref is the reference the weights of this row are
+    // taken against (-inf until the row has seen an allowed key), l their running sum.
+    // The reference moves only when a tile's maximum exceeds it by more than 8 (a factor
+    // 256), so the accumulator is rescaled rarely; weights stay below 2^8.
+    float m_ref = -INFINITY, l = 0.f;
     int c = 0;
     if (valid[s]) {
       for (int j = t0[s]; j <= t1[s]; ++j, ++c) {
         if (!mbar_wait(s_full + s, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
         tc_fence_after();
-        float x[BN];
-#pragma unroll
-        for (int q4 = 0; q4 < BN / 32; ++q4) {
-          float (&xx)[32] = *reinterpret_cast<float(*)[32]>(&x[q4 * 32]);
-          tmem_ld32(tS + q4 * 32, xx);
-        }
-        tmem_wait_ld();
         const int key0 = j * BN;
         // does any row of this slot need per-element masking in this tile?
-        const bool need_mask = (key0 + BN > p.T) ||
-                               (p.causal && key0 + BN - 1 > qs[s]) ||
+        const bool need_mask = (key0 + BN > p.T) || (p.causal && key0 + BN - 1 > qs[s]) ||
                                (p.window > 0 && qs[s] + BM - 1 - key0 >= p.window);
-        float mt = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < BN; ++k) {
-          float v = x[k] * a.scale_log2;
-          if (p.alibi.on) v -= slope * fabsf((float)(i - (key0 + k)));
+        const bool plain = !need_mask && !p.alibi.on;
+        auto score = [&](float x, int jk) {
+          float v = p.alibi.on ? fmaf(x, sc, -slope * fabsf((float)(i - jk))) : x * sc;
           if (need_mask) {
-            const int jk = key0 + k;
             const bool ok = jk < p.T && (!p.causal || jk <= i) && (p.window <= 0 || i - jk < p.window);
             v = ok ? v : -INFINITY;
           }
-          x[k] = v;
-          mt = fmaxf(mt, v);
-        }
-        const float m_new = fmaxf(m, mt);
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = ex2(m - m_use);
-        uint32_t pk[BN / 2];
-        float rs = 0.f;
+          return v;
+        };
+        // pass 1: the tile's row maximum
+        float mt = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < BN / 2; ++k) {
-          const float e0 = ex2(x[2 * k] - m_use), e1 = ex2(x[2 * k + 1] - m_use);
-          rs += e0 + e1;
-          pk[k] = f2_to_bf2(e0, e1);
+        for (int h2 = 0; h2 < BN / 64; ++h2) {
+          float xa[32], xb[32];
+          tmem_ld32(tS + h2 * 64, xa);
+          tmem_ld32(tS + h2 * 64 + 32, xb);
+          tmem_wait_ld();
+          if (plain) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) mt = fmaxf(mt, fmaxf(xa[k], xb[k]));
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              mt = fmaxf(mt, fmaxf(score(xa[k], key0 + h2 * 64 + k), score(xb[k], key0 + h2 * 64 + 32 + k)));
+          }
         }
-        l = l * alpha + rs;
-        m = m_new;
+        if (plain) mt *= sc;  // a positive scale keeps the order, so max then scale is exact
+        const float m_new = (mt > m_ref + 8.f) ? mt : m_ref;  // also takes mt when m_ref = -inf
+        const float alpha = (m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
+        const float m_exp = (m_new == -INFINITY) ? 0.f : m_new;
+        m_ref = m_new;
         if (c > 0) {
           // the previous PV must finish before O is rescaled and P is overwritten
           if (!mbar_wait(o_done + s, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
@@ -358,11 +413,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_wait_st();
           }
         }
+        // pass 2: weights, their sum, and P (bf16) into shared memory
+        float rs = 0.f;
 #pragma unroll
-        for (int c8 = 0; c8 < BN / 8; ++c8) {
-          uint4* dst = reinterpret_cast<uint4*>(myP + sw128_offset(r, c8 * 8, BM));
-          *dst = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+        for (int h2 = 0; h2 < BN / 64; ++h2) {
+          float xa[32], xb[32];
+          tmem_ld32(tS + h2 * 64, xa);
+          tmem_ld32(tS + h2 * 64 + 32, xb);
+          tmem_wait_ld();
+          uint32_t pk[32];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            float e0, e1, e2, e3;
+            if (plain) {
+              e0 = ex2(fmaf(xa[2 * k], sc, -m_exp));
+              e1 = ex2(fmaf(xa[2 * k + 1], sc, -m_exp));
+              e2 = ex2(fmaf(xb[2 * k], sc, -m_exp));
+              e3 = ex2(fmaf(xb[2 * k + 1], sc, -m_exp));
+            } else {
+              const int jk = key0 + h2 * 64 + 2 * k;
+              e0 = ex2(score(xa[2 * k], jk) - m_exp);
+              e1 = ex2(score(xa[2 * k + 1], jk + 1) - m_exp);
+              e2 = ex2(score(xb[2 * k], jk + 32) - m_exp);
+              e3 = ex2(score(xb[2 * k + 1], jk + 33) - m_exp);
+            }
+            rs += (e0 + e1) + (e2 + e3);
+            pk[k] = f2_to_bf2(e0, e1);
+            pk[16 + k] = f2_to_bf2(e2, e3);
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < 8; ++c8) {
+            uint4* dst = reinterpret_cast<uint4*>(myP + sw128_offset(r, h2 * 64 + c8 * 8, BM));
+            *dst = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+          }
         }
+        l = l * alpha + rs;
         fence_proxy_async();
         tc_fence_before();
         mbar_arrive(p_full + s);
@@ -389,7 +474,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         if (p.lse && i < p.T)
-          p.lse[((size_t)b * p.H + head[s]) * p.T + i] = l > 0.f ? (m + __log2f(l)) * LN2 : -INFINITY;
+          p.lse[((size_t)b * p.H + head[s]) * p.T + i] = l > 0.f ? (m_ref + __log2f(l)) * LN2 : -INFINITY;
       }
     }
   }

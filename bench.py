@@ -196,22 +196,27 @@ def run_ours(args, rank, world):
     stream = torch.cuda.current_stream()
     w, dw = PREFILL, DECODE
 
+    do_p, do_d = args.only in ("all", "prefill"), args.only in ("all", "decode")
     q, k, v = workloads.prefill_inputs(w)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
     dout = torch.empty_like(dq)
-    dq_, dkc, dvc, dsl, dqp = workloads.decode_inputs(dw)
-    dbytes = decode_bytes(dsl, dw)
-    ddq, dkc, dvc, dsl, dqp = dq_.cuda(), dkc.cuda(), dvc.cuda(), dsl.cuda(), dqp.cuda()
-    ddout = torch.empty_like(ddq)
-    ws = torch.empty(art.attn_decode_workspace_size(dw.B, dw.H, dw.KV, dw.hd, dw.Lmax),
-                     dtype=torch.uint8, device="cuda")
+    dbytes = 1
+    if do_d:
+        dq_, dkc, dvc, dsl, dqp = workloads.decode_inputs(dw)
+        dbytes = decode_bytes(dsl, dw)
+        ddq, dkc, dvc, dsl, dqp = dq_.cuda(), dkc.cuda(), dvc.cuda(), dsl.cuda(), dqp.cuda()
+        ddout = torch.empty_like(ddq)
+        ws = torch.empty(art.attn_decode_workspace_size(dw.B, dw.H, dw.KV, dw.hd, dw.Lmax),
+                         dtype=torch.uint8, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
     def prefill():
-        art.attn_prefill(dq, dk, dv, dout, rope_base=w.rope_base, causal=True, window=w.window)
+        if do_p:
+            art.attn_prefill(dq, dk, dv, dout, rope_base=w.rope_base, causal=True, window=w.window)
 
     def decode():
-        art.attn_decode(ddq, dkc, dvc, dsl, dqp, ddout, workspace=ws, rope_base=dw.rope_base)
+        if do_d:
+            art.attn_decode(ddq, dkc, dvc, dsl, dqp, ddout, workspace=ws, rope_base=dw.rope_base)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -243,8 +248,8 @@ def run_ours(args, rank, world):
     art.attn_sync_status()
     p_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
     d_ms = [ev[s][2].elapsed_time(ev[s][3]) for s in range(args.steps)]
-    p_tot = max_over_ranks(sum(p_ms), world)
-    d_tot = max_over_ranks(sum(d_ms), world)
+    p_tot = max(1e-9, max_over_ranks(sum(p_ms), world))
+    d_tot = max(1e-9, max_over_ranks(sum(d_ms), world))
     region_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
 
     # end to end: pinned host inputs -> device -> prefill -> host output, every step
@@ -280,6 +285,10 @@ def run_ours(args, rank, world):
             traffic = json.load(f).get("prefill_tc")
 
     if rank != 0:
+        return
+    if args.only != "all":
+        print(json.dumps({"only": args.only, "prefill_ms": p_tot / args.steps,
+                          "decode_ms": d_tot / args.steps}), flush=True)
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -319,6 +328,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="run one kernel family only (for profiler captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
