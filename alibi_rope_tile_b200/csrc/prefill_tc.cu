@@ -23,9 +23,14 @@
 //   warp 12    TMA producer (Q tiles, then K/V tiles through a ring of NS stages)
 //   warp 13    TMEM allocation and UMMA issue
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each) | O0 | O1 (hd each).
-// P (bf16) goes through shared memory, so an S buffer can be refilled as soon as its
-// softmax has read it. Issue order per key tile j: PV0(j), QK0(j+1), PV1(j), QK1(j+1):
-// the tensor core works on one slot while the other slot's softmax runs.
+// The softmax writes P (bf16, two per 32-bit column) over the first 64 columns of its own
+// S buffer, after reading them, and PV takes P straight from tensor memory (the A operand
+// of the TS-form MMA): P never touches shared memory, whose bandwidth (128 B/clk/SM) the
+// SS-form QK MMAs, the TMA writes and the in-place key rotation already share. The next
+// QK of a slot overwrites that slot's S/P columns; it is issued after the slot's PV, and
+// the tensor core executes one CTA's MMAs in issue order, so P is read before it is
+// overwritten. Issue order per key tile j: PV0(j), QK0(j+1), PV1(j), QK1(j+1): the tensor
+// core works on one slot while the other slot's softmax runs.
 //
 // Masking: a pair outside the causal/window/length limits gets -inf before the row max,
 // so its weight is exactly 0, and the sums' order depends only on the tile structure;
@@ -53,15 +58,28 @@ constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;  // a wait that lasts 4 s has 
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
+#ifdef ATTN_TRACE
+// Diagnostic build only: SM-clock stamps of pipeline events of one CTA, 16 lanes x 2048.
+__device__ long long g_attn_trace[16][2048];
+#define TRACE(lane_id, counter, tag)                                                      \
+  do {                                                                                    \
+    if (blockIdx.x == ATTN_TRACE && (counter) < 2048)                                     \
+      g_attn_trace[lane_id][(counter)++] = (clock64() << 8) | (long long)(tag);           \
+  } while (0)
+#else
+#define TRACE(lane_id, counter, tag) \
+  do {                               \
+    (void)(counter);                 \
+  } while (0)
+#endif
+
 template <int HD>
 struct Cfg {
-  static constexpr int NS = HD == 128 ? 3 : 6;  // key/value ring stages
+  static constexpr int NS = HD == 128 ? 5 : 10;  // key/value ring stages
   static constexpr int Q_BYTES = BM * HD * 2;
-  static constexpr int P_BYTES = BM * BN * 2;
   static constexpr int KV_BYTES = BN * HD * 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
-  static constexpr int OFF_KV = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
   static constexpr int NBAR = 3 * NS + 8;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -79,29 +97,7 @@ struct TcArgs {
   float scale_log2;
 };
 
-// Turn the interleaved pairs of one 128-byte-swizzled bf16 row in place (accurate angle
-// for every pair; used once per CTA for the query tiles).
-template <int HD>
-__device__ __forceinline__ void rotate_row(uint8_t* tile, int row, int pos, const RopeFreqs& rope) {
-#pragma unroll 2
-  for (int c = 0; c < HD / 8; ++c) {
-    uint4* ptr = reinterpret_cast<uint4*>(tile + sw128_offset(row, c * 8, BM));
-    uint4 u = *ptr;
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int pc = c * 4 + e;
-      float sn, cs;
-      rope_cos_sin(pos, rope.hi[pc], rope.lo[pc], cs, sn);
-      float2 f = bf2_to_f2(w[e]);
-      rotate_pair(f.x, f.y, cs, sn);
-      w[e] = f2_to_bf2(f.x, f.y);
-    }
-    *ptr = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
-// Rotation of a whole key tile by the 128 threads of the rotary warpgroup. Thread t owns
+// Rotation of a whole key (or query) tile by the 128 threads of the rotary warpgroup. Thread t owns
 // one 16-byte chunk (4 pairs) of the row and the rows phase, phase + PH, phase + 2 PH ...
 // Along those rows the angle of a pair grows by the fixed step PH * w, so the cosine and
 // sine follow the angle-addition recurrence (c, s) <- (c C - s S, s C + c S) with (C, S)
@@ -132,7 +128,7 @@ struct KRot {
       const int pc = chunk * 4 + e;
       rope_cos_sin(pos_row0 + phase, rope.hi[pc], rope.lo[pc], c[e], s[e]);
     }
-#pragma unroll 4
+#pragma unroll 2
     for (int k = 0; k < NR; ++k) {
       const int r = phase + PH * k;
       uint4* ptr = reinterpret_cast<uint4*>(tile + sw128_offset(r, chunk * 8, BN));
@@ -160,7 +156,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem + C::OFF_Q;
-  uint8_t* sP = smem + C::OFF_P;
   uint8_t* sKV = smem + C::OFF_KV;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars;
@@ -247,11 +242,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (valid[s])
           for (int kb = 0; kb < HD / 64; ++kb)
             tma_load_4d(sQ + s * C::Q_BYTES + kb * BM * 128, &tmQ, q_full, kb * 64, head[s], qs[s], b);
-      int u = 0;
+      int u = 0, tcnt = 0;
       for (int j = jt0; j <= jt1; ++j) {
         for (int kv = 0; kv < 2; ++kv, ++u) {
           const int st = u % C::NS, n = u / C::NS;
           if (!mbar_wait(kv_empty + st, (n & 1) ^ 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+          TRACE(4, tcnt, 30 + kv);
           mbar_expect_tx(kv_full + st, C::KV_BYTES);
           for (int kb = 0; kb < HD / 64; ++kb)
             tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, kv ? &tmV : &tmK, kv_full + st,
@@ -267,43 +263,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (!mbar_wait(q_full, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
     if (p.rope.on)
       for (int s = 0; s < 2; ++s)
-        if (valid[s]) rotate_row<HD>(sQ + s * C::Q_BYTES, r, p.pos0 + qs[s] + r, p.rope);
+        if (valid[s]) krot.rotate(sQ + s * C::Q_BYTES, p.pos0 + qs[s], p.rope);
     fence_proxy_async();
     mbar_arrive(q_rot);
-    int u = 0;
+    int u = 0, tcnt = 0;
     for (int j = jt0; j <= jt1; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++u) {
         const int st = u % C::NS, n = u / C::NS;
         if (!mbar_wait(kv_full + st, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        if (tid == WARP_ROPE0 * 32) TRACE(3, tcnt, 20 + kv);
         if (kv == 0 && p.rope.on) krot.rotate(sKV + st * C::KV_BYTES, p.pos0 + j * BN, p.rope);
         fence_proxy_async();
         mbar_arrive(k_rot + st);
+        if (tid == WARP_ROPE0 * 32) TRACE(3, tcnt, 22);
       }
     }
   } else if (warp == WARP_MMA) {
     // ------------------------------------------------------------ UMMA issue
     if (lane == 0) {
-      const uint32_t aQ = smem_u32(sQ), aP = smem_u32(sP), aKV = smem_u32(sKV);
+      // Descriptors are built once; the start-address field (bits 0-13, in 16-byte
+      // units) is then advanced by plain additions that stay below 2^14.
+      const uint64_t dQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t dV = smem_desc_sw128(smem_u32(sKV), BN * 128, 1024);
       auto issue_qk = [&](int s, int st) {
         const uint32_t d = tmem + s * BN;
+        const uint64_t a0 = dQ + (uint64_t)((s * C::Q_BYTES) >> 4);
+        const uint64_t b0 = dK + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          umma_ss(d, smem_desc_sw128(aQ + s * C::Q_BYTES + off, 16, 1024),
-                  smem_desc_sw128(aKV + st * C::KV_BYTES + off, 16, 1024), C::IDESC_QK, kk > 0);
+          const uint32_t off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
+          umma_ss(d, a0 + off, b0 + off, C::IDESC_QK, kk > 0);
         }
       };
       auto issue_pv = [&](int s, int st, bool acc) {
         const uint32_t d = tmem + 2 * BN + s * HD;
+        const uint32_t aP = tmem + s * BN;  // P: 64 columns of bf16 pairs over S
+        const uint64_t b0 = dV + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t offp = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          umma_ss(d, smem_desc_sw128(aP + s * C::P_BYTES + offp, 16, 1024),
-                  smem_desc_sw128(aKV + st * C::KV_BYTES + kk * 16 * 128, BN * 128, 1024),
-                  C::IDESC_PV, (kk > 0 || acc) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ts(d, aP + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
+                  (kk > 0 || acc) ? 1u : 0u);
       };
       int cnt[2] = {0, 0};
+      int tcnt = 0;
       if (!mbar_wait(q_rot, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
       // K of the first tile
       if (!mbar_wait(k_rot + 0, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
@@ -319,21 +322,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int uK = uV + 1, stK = uK % C::NS;
         const bool next = j < jt1;
         if (!mbar_wait(k_rot + stV, (uV / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        TRACE(0, tcnt, 8);
         for (int s = 0; s < 2; ++s) {
           if (active(s, j)) {
             if (!mbar_wait(p_full + s, cnt[s] & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+            TRACE(0, tcnt, 1 + 4 * s);
             tc_fence_after();
             issue_pv(s, stV, cnt[s] > 0);
             umma_commit(o_done + s);
             ++cnt[s];
+            TRACE(0, tcnt, 2 + 4 * s);
           }
           if (next && s == 0) {
             if (!mbar_wait(k_rot + stK, (uK / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+            TRACE(0, tcnt, 3);
             tc_fence_after();
           }
           if (next && active(s, j + 1)) {
             issue_qk(s, stK);
             umma_commit(s_full + s);
+            TRACE(0, tcnt, 4 + 4 * s);
           }
         }
         umma_commit(kv_empty + stV);
@@ -342,13 +350,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 0-7)
+    // The per-tile loops over 64-column halves are deliberately not unrolled: with ten
+    // warps running four different roles, the instruction cache, not the exponential
+    // unit, bounded the unrolled version.
     const int s = warp >> 2;
     const int r = tid & 127;
     const int i = qs[s] + r;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + s * BN;
     const uint32_t tO = tmem + lane_off + 2 * BN + s * HD;
-    uint8_t* myP = sP + s * C::P_BYTES;
     const float slope = p.alibi.on ? p.alibi.slope[head[s]] * LOG2E : 0.f;
     const float sc = a.scale_log2;
     // Row state in the log2 domain: m_ref is the reference the weights of this row are
@@ -356,10 +366,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // The reference moves only when a tile's maximum exceeds it by more than 8 (a factor
     // 256), so the accumulator is rescaled rarely; weights stay below 2^8.
     float m_ref = -INFINITY, l = 0.f;
-    int c = 0;
+    int c = 0, tcnt = 0;
+    const bool tracer = (tid & 127) == 0;
     if (valid[s]) {
       for (int j = t0[s]; j <= t1[s]; ++j, ++c) {
         if (!mbar_wait(s_full + s, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        if (tracer) TRACE(1 + s, tcnt, 10);
         tc_fence_after();
         const int key0 = j * BN;
         // does any row of this slot need per-element masking in this tile?
@@ -376,7 +388,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         };
         // pass 1: the tile's row maximum
         float mt = -INFINITY;
-#pragma unroll
+#pragma unroll 1
         for (int h2 = 0; h2 < BN / 64; ++h2) {
           float xa[32], xb[32];
           tmem_ld32(tS + h2 * 64, xa);
@@ -396,12 +408,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float alpha = (m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
         const float m_exp = (m_new == -INFINITY) ? 0.f : m_new;
         m_ref = m_new;
+        if (tracer) TRACE(1 + s, tcnt, 11);
         if (c > 0) {
           // the previous PV must finish before O is rescaled and P is overwritten
           if (!mbar_wait(o_done + s, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
           tc_fence_after();
           if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
+#pragma unroll 1
             for (int q4 = 0; q4 < HD / 32; ++q4) {
               float o[32];
               tmem_ld32(tO + q4 * 32, o);
@@ -413,15 +426,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_wait_st();
           }
         }
+        if (tracer) TRACE(1 + s, tcnt, 12);
         // pass 2: weights, their sum, and P (bf16) into shared memory
         float rs = 0.f;
-#pragma unroll
+#pragma unroll 1
         for (int h2 = 0; h2 < BN / 64; ++h2) {
           float xa[32], xb[32];
           tmem_ld32(tS + h2 * 64, xa);
           tmem_ld32(tS + h2 * 64 + 32, xb);
           tmem_wait_ld();
-          uint32_t pk[32];
+          if (tracer) TRACE(1 + s, tcnt, 15 + 2 * h2);
+          uint32_t pk[32];  // column k: keys 2k, 2k+1 of this half (low half = even key)
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             float e0, e1, e2, e3;
@@ -441,16 +456,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             pk[k] = f2_to_bf2(e0, e1);
             pk[16 + k] = f2_to_bf2(e2, e3);
           }
-#pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            uint4* dst = reinterpret_cast<uint4*>(myP + sw128_offset(r, h2 * 64 + c8 * 8, BM));
-            *dst = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
-          }
+          // P of keys h2*64 .. h2*64+63 -> columns h2*32 .. h2*32+31 (already read above)
+          tmem_st32u(tS + h2 * 32, pk);
+          if (tracer) TRACE(1 + s, tcnt, 16 + 2 * h2);
         }
         l = l * alpha + rs;
-        fence_proxy_async();
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full + s);
+        if (tracer) TRACE(1 + s, tcnt, 14);
       }
       if (c > 0) {
         if (!mbar_wait(o_done + s, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
@@ -458,7 +472,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float inv = l > 0.f ? 1.f / l : 0.f;
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
                               (((size_t)b * p.T + i) * p.H + head[s]) * HD;
-#pragma unroll
+#pragma unroll 1
         for (int q4 = 0; q4 < HD / 32; ++q4) {
           float o[32];
           tmem_ld32(tO + q4 * 32, o);
@@ -488,6 +502,21 @@ done:
 }
 
 // ---------------------------------------------------------------- host side
+#ifdef ATTN_TRACE
+}  // namespace
+}  // namespace tc
+}  // namespace attn
+extern "C" int attn_trace_read(long long* host) {
+  return (int)cudaMemcpyFromSymbol(host, attn::tc::g_attn_trace, sizeof(attn::tc::g_attn_trace));
+}
+extern "C" int attn_trace_clear() {
+  static long long zeros[16][2048];
+  return (int)cudaMemcpyToSymbol(attn::tc::g_attn_trace, zeros, sizeof(zeros));
+}
+namespace attn {
+namespace tc {
+namespace {
+#endif
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
