@@ -122,28 +122,48 @@ struct KRot {
     }
   }
   __device__ __forceinline__ void rotate(uint8_t* tile, int pos_row0, const RopeFreqs& rope) const {
-    float c[4], s[4];
+    // pairs (0, 1) and (2, 3) of the chunk are handled two at a time in packed f32x2 form
+    float c[4], sn[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int pc = chunk * 4 + e;
-      rope_cos_sin(pos_row0 + phase, rope.hi[pc], rope.lo[pc], c[e], s[e]);
+      rope_cos_sin(pos_row0 + phase, rope.hi[pc], rope.lo[pc], c[e], sn[e]);
+    }
+    f2x C[2], S[2], N[2], SC[2], SS[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      C[h] = pk2(c[2 * h], c[2 * h + 1]);
+      S[h] = pk2(sn[2 * h], sn[2 * h + 1]);
+      N[h] = neg2(S[h]);
+      SC[h] = pk2(stepc[2 * h], stepc[2 * h + 1]);
+      SS[h] = pk2(steps[2 * h], steps[2 * h + 1]);
     }
 #pragma unroll 2
     for (int k = 0; k < NR; ++k) {
       const int r = phase + PH * k;
       uint4* ptr = reinterpret_cast<uint4*>(tile + sw128_offset(r, chunk * 8, BN));
-      uint4 u = *ptr;
-      uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      const uint4 u = *ptr;
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t o[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float2 f = bf2_to_f2(w[e]);
-        rotate_pair(f.x, f.y, c[e], s[e]);
-        w[e] = f2_to_bf2(f.x, f.y);
-        const float cn = c[e] * stepc[e] - s[e] * steps[e];
-        s[e] = s[e] * stepc[e] + c[e] * steps[e];
-        c[e] = cn;
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t wa = w[2 * h], wb = w[2 * h + 1];
+        const f2x X = pk2(__uint_as_float(wa << 16), __uint_as_float(wb << 16));
+        const f2x Y = pk2(__uint_as_float(wa & 0xffff0000u), __uint_as_float(wb & 0xffff0000u));
+        const f2x Xr = fma2(Y, N[h], mul2(X, C[h]));   // x c - y s
+        const f2x Yr = fma2(X, S[h], mul2(Y, C[h]));   // x s + y c
+        float xa, xb, ya, yb;
+        up2(Xr, xa, xb);
+        up2(Yr, ya, yb);
+        o[2 * h] = f2_to_bf2(xa, ya);
+        o[2 * h + 1] = f2_to_bf2(xb, yb);
+        // advance both angles by the step: (c, s) <- (c C - s S, s C + c S)
+        const f2x Cn = fma2(N[h], SS[h], mul2(C[h], SC[h]));
+        S[h] = fma2(C[h], SS[h], mul2(S[h], SC[h]));
+        C[h] = Cn;
+        N[h] = neg2(S[h]);
       }
-      *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+      *ptr = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
 };
@@ -386,49 +406,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           return v;
         };
-        // pass 1: the tile's row maximum
-        float mt = -INFINITY;
-#pragma unroll 1
-        for (int h2 = 0; h2 < BN / 64; ++h2) {
-          float xa[32], xb[32];
-          tmem_ld32(tS + h2 * 64, xa);
-          tmem_ld32(tS + h2 * 64 + 32, xb);
-          tmem_wait_ld();
-          if (plain) {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) mt = fmaxf(mt, fmaxf(xa[k], xb[k]));
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              mt = fmaxf(mt, fmaxf(score(xa[k], key0 + h2 * 64 + k), score(xb[k], key0 + h2 * 64 + 32 + k)));
-          }
-        }
-        if (plain) mt *= sc;  // a positive scale keeps the order, so max then scale is exact
-        const float m_new = (mt > m_ref + 8.f) ? mt : m_ref;  // also takes mt when m_ref = -inf
-        const float alpha = (m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
-        const float m_exp = (m_new == -INFINITY) ? 0.f : m_new;
-        m_ref = m_new;
+        // Weights are taken against a per-row reference m_exp that starts at the row's
+        // reference m_ref. Each 64-key half is loaded once: its maximum is taken first, and
+        // if it exceeds the reference by more than 8 for some row of the warp, that row's
+        // reference moves up before the weights of the half are formed. When the second
+        // half moves it, the P already written for the first half (and its partial sum)
+        // is rescaled in place; once a row has seen a tile this is rare.
+        float m_exp = m_ref, rs = 0.f;
         if (tracer) TRACE(1 + s, tcnt, 11);
-        if (c > 0) {
-          // the previous PV must finish before O is rescaled and P is overwritten
-          if (!mbar_wait(o_done + s, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-            for (int q4 = 0; q4 < HD / 32; ++q4) {
-              float o[32];
-              tmem_ld32(tO + q4 * 32, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] *= alpha;
-              tmem_st32(tO + q4 * 32, o);
-            }
-            tmem_wait_st();
-          }
-        }
-        if (tracer) TRACE(1 + s, tcnt, 12);
-        // pass 2: weights, their sum, and P (bf16) into shared memory
-        float rs = 0.f;
 #pragma unroll 1
         for (int h2 = 0; h2 < BN / 64; ++h2) {
           float xa[32], xb[32];
@@ -436,30 +421,86 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_ld32(tS + h2 * 64 + 32, xb);
           tmem_wait_ld();
           if (tracer) TRACE(1 + s, tcnt, 15 + 2 * h2);
+          float hx = -INFINITY;
+          if (plain) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) hx = max3(hx, max3(xa[2 * k], xa[2 * k + 1], xb[2 * k]), xb[2 * k + 1]);
+            hx *= sc;  // a positive scale keeps the order: max then scale is exact
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              xa[k] = score(xa[k], key0 + h2 * 64 + k);
+              xb[k] = score(xb[k], key0 + h2 * 64 + 32 + k);
+              hx = max3(hx, xa[k], xb[k]);
+            }
+          }
+          const float m_cand = (hx > m_exp + 8.f) ? hx : m_exp;  // takes hx when m_exp = -inf
+          if (__any_sync(0xffffffffu, m_cand != m_exp)) {
+            if (h2 > 0) {
+              const float f = (m_cand == m_exp) ? 1.f : ex2(m_exp - m_cand);  // 1 where it stays
+              float pp[32];
+              tmem_wait_st();
+              tmem_ld32(tS, pp);
+              tmem_wait_ld();
+              uint32_t pq[32];
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                const float2 v = bf2_to_f2(__float_as_uint(pp[k]));
+                pq[k] = f2_to_bf2(v.x * f, v.y * f);
+              }
+              tmem_st32u(tS, pq);
+              rs *= f;
+            }
+            m_exp = m_cand;
+          }
+          const float mu = (m_exp == -INFINITY) ? 0.f : m_exp;
+          const f2x SC = pk2(sc, sc), NM = pk2(-mu, -mu);
+          float rs0 = 0.f, rs1 = 0.f;
           uint32_t pk[32];  // column k: keys 2k, 2k+1 of this half (low half = even key)
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             float e0, e1, e2, e3;
             if (plain) {
-              e0 = ex2(fmaf(xa[2 * k], sc, -m_exp));
-              e1 = ex2(fmaf(xa[2 * k + 1], sc, -m_exp));
-              e2 = ex2(fmaf(xb[2 * k], sc, -m_exp));
-              e3 = ex2(fmaf(xb[2 * k + 1], sc, -m_exp));
+              float a0, a1, b0, b1;
+              up2(fma2(pk2(xa[2 * k], xa[2 * k + 1]), SC, NM), a0, a1);
+              up2(fma2(pk2(xb[2 * k], xb[2 * k + 1]), SC, NM), b0, b1);
+              e0 = ex2(a0);
+              e1 = ex2(a1);
+              e2 = ex2(b0);
+              e3 = ex2(b1);
             } else {
-              const int jk = key0 + h2 * 64 + 2 * k;
-              e0 = ex2(score(xa[2 * k], jk) - m_exp);
-              e1 = ex2(score(xa[2 * k + 1], jk + 1) - m_exp);
-              e2 = ex2(score(xb[2 * k], jk + 32) - m_exp);
-              e3 = ex2(score(xb[2 * k + 1], jk + 33) - m_exp);
+              e0 = ex2(xa[2 * k] - mu);
+              e1 = ex2(xa[2 * k + 1] - mu);
+              e2 = ex2(xb[2 * k] - mu);
+              e3 = ex2(xb[2 * k + 1] - mu);
             }
-            rs += (e0 + e1) + (e2 + e3);
+            rs0 += e0 + e1;
+            rs1 += e2 + e3;
             pk[k] = f2_to_bf2(e0, e1);
             pk[16 + k] = f2_to_bf2(e2, e3);
           }
+          rs += rs0 + rs1;
           // P of keys h2*64 .. h2*64+63 -> columns h2*32 .. h2*32+31 (already read above)
           tmem_st32u(tS + h2 * 32, pk);
           if (tracer) TRACE(1 + s, tcnt, 16 + 2 * h2);
         }
+        const float m_new = m_exp;
+        const float alpha = (m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
+        m_ref = m_new;
+        // O is rescaled before this tile's PV is issued. The previous PV of this slot has
+        // completed: it was issued before the QK whose completion this tile waited for.
+        if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int q4 = 0; q4 < HD / 32; ++q4) {
+            float o[32];
+            tmem_ld32(tO + q4 * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tO + q4 * 32, o);
+          }
+        }
+        if (tracer) TRACE(1 + s, tcnt, 12);
         l = l * alpha + rs;
         tmem_wait_st();
         tc_fence_before();

@@ -27,14 +27,17 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// One try: true once the phase with the given parity has completed. While it has not,
+// the hardware may suspend the thread for up to ``suspend_ns`` (it resumes as soon as the
+// phase completes), so a waiting role takes no issue slots from the working ones.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
       : "memory");
   return ok != 0;
 }
@@ -44,24 +47,28 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Wait for the phase of ``bar`` with the given parity to complete. The wait is bounded:
-// after ``limit_ns`` (or as soon as another role of the CTA has given up, seen through
-// ``abort``) it records DEV_TIMEOUT in the device status word and returns false.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                       int* status, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait: retries in suspended slices of 1 ms until the phase completes,
+// another role of the CTA gives up (``abort``), or ``limit_ns`` passes; in the last case
+// it records DEV_TIMEOUT in the device status word. Returns false when it gave up.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                            int* status, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 255u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort = 1;
-        flag_error(status, DEV_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait(bar, parity, 1000000u)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort = 1;
+      flag_error(status, DEV_TIMEOUT);
+      return false;
     }
   }
+}
+
+// Bounded wait for the phase of ``bar`` with the given parity.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int* status, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity, 1000000u)) return true;
+  return mbar_wait_slow(bar, parity, abort, status, limit_ns);
 }
 
 __device__ __forceinline__ void fence_barrier_init() {
@@ -230,6 +237,43 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+// Packed pairs of fp32 (Blackwell f32x2 arithmetic: one instruction for two lanes).
+struct f2x {
+  uint64_t v;
+};
+__device__ __forceinline__ f2x pk2(float lo, float hi) {
+  f2x r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void up2(f2x a, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
+}
+__device__ __forceinline__ f2x fma2(f2x a, f2x b, f2x c) {
+  f2x d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+  return d;
+}
+__device__ __forceinline__ f2x mul2(f2x a, f2x b) {
+  f2x d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+  return d;
+}
+__device__ __forceinline__ f2x add2(f2x a, f2x b) {
+  f2x d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+  return d;
+}
+__device__ __forceinline__ f2x neg2(f2x a) {
+  f2x d;
+  d.v = a.v ^ 0x8000000080000000ull;
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 __device__ __forceinline__ float ex2(float x) {
   float y;
