@@ -3,9 +3,10 @@
 // the keys and merged with the log-sum-exp rule of the FlashAttention section's online
 // softmax (m = max m_c, l = sum exp(m_c - m) l_c, O = sum exp(m_c - m) O_c / l).
 //
-// Pass 1, one CTA per (split, key/value head, sequence): the CTA reads its chunk of cache
-// rows once, 16 bytes per lane per load, and serves every query head of the group from
-// those rows. Each warp owns a stream of keys; a key row of hd bf16 is covered by
+// Pass 1 runs on the tensor cores for bf16 with hd 64 or 128 (decode_tc.cu). Otherwise it
+// is the CUDA-core kernel below, one CTA per (split, key/value head, sequence): the CTA
+// reads its chunk of cache rows once, 16 bytes per lane per load, and serves every query
+// head of the group from those rows. Each warp owns a stream of keys; a key row of hd bf16 is covered by
 // hd/8 lanes, so one warp load instruction covers 32*8/hd rows. Per key the group's
 // scores are reduced across the lanes of the row; weights are formed with a running
 // maximum per warp and head, and each lane accumulates the group's outputs for its 8
@@ -267,6 +268,12 @@ template <typename T>
 cudaError_t launch_t(const DecodeParams& p, void* ws, cudaStream_t s) {
   const int chunk = decode_chunk(p.B, p.KV, p.Lmax);
   const int nsplit = (p.Lmax + chunk - 1) / chunk;
+  if (decode_tc_supported(p, sizeof(T) == 2 ? 1 : 0)) {
+    cudaError_t e = launch_decode_tc(p, chunk, nsplit, ws, s);
+    if (e != cudaSuccess) return e;
+    decode_merge_kernel<T><<<dim3(p.H, p.B), 128, 0, s>>>(p, chunk, nsplit, ws);
+    return cudaGetLastError();
+  }
   switch (p.H / p.KV) {
     case 1: return launch_g<T, 1>(p, chunk, nsplit, ws, s);
     case 2: return launch_g<T, 2>(p, chunk, nsplit, ws, s);
@@ -310,12 +317,12 @@ __global__ void kv_append_kernel(const AppendParams p) {
 
 int decode_chunk(int B, int KV, int Lmax) {
   // Enough splits for about four CTAs per SM on 148 SMs when every cache is full, with
-  // chunks a multiple of 64 rows and at least 256 rows.
+  // chunks a multiple of the 128-row key tile and at least 256 rows.
   const long long units = (long long)B * KV;
   long long want = (4LL * 148 + units - 1) / units;  // splits per (sequence, kv head)
   if (want < 1) want = 1;
   long long chunk = ((long long)Lmax + want - 1) / want;
-  chunk = ((chunk + 63) / 64) * 64;
+  chunk = ((chunk + 127) / 128) * 128;
   if (chunk < 256) chunk = 256;
   return (int)chunk;
 }

@@ -1,0 +1,376 @@
+// Split-KV decode on the tensor cores (sm_100a): one new query per sequence attends to
+// its KV cache ("Building a Transformer from Scratch: Attention, Architecture, and
+// Memory", Part 3 "KV caching"); the splits are merged with the log-sum-exp rule of that
+// page's FlashAttention equations by the merge kernel in decode.cu.
+//
+// One CTA = one (split of the cache rows, key/value head, sequence). The H/KV query heads
+// served by the key/value head are the rows of a 128-row MMA tile (rows >= H/KV are zero),
+// so the scores S = Q K^T of a 128-key tile land in tensor memory one head per TMEM lane:
+// the softmax of a head is a row-wise online softmax done by one thread, with no
+// cross-thread reduction. P (bf16) is written back over the S columns and PV is the
+// TS-form MMA. The padded rows cost tensor-core time that decode does not miss: the
+// kernel is bound by streaming K and V from HBM, which TMA does through a two-stage ring
+// (two CTAs per SM keep four 32 KB tiles in flight per SM).
+//
+// Warps: 0 = softmax (lanes 0..H/KV-1 hold one head each) and query set-up, 1 = TMA
+// producer, 2 = TMEM allocation and MMA issue, 3 = query set-up only.
+// The cached keys are already rotated at their slot positions; only q is rotated here,
+// at qpos[b]. Keys at or beyond seqlens[b] and, with a window, keys j with
+// qpos - j >= window get weight exactly 0.
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace attn {
+namespace tcdec {
+namespace {
+
+using namespace attn::tc;
+
+constexpr int BN = 128;               // keys per tile
+constexpr int BM = 128;               // MMA rows (query heads, zero padded)
+constexpr int NS = 2;                 // ring stages (K, V alternate)
+constexpr int THREADS = 128;
+constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
+constexpr float LOG2E = 1.4426950408889634f;
+
+template <int HD>
+struct Cfg {
+  static constexpr int Q_BYTES = BM * HD * 2;
+  static constexpr int KV_BYTES = BN * HD * 2;
+  static constexpr int OFF_KV = Q_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
+  static constexpr int NBAR = 2 * NS + 3;  // kv_full[NS], kv_empty[NS], s_full, p_full, o_done
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, 0, 1);
+};
+
+struct DecArgs {
+  DecodeParams p;
+  int chunk;   // keys per split (multiple of 128)
+  int nsplit;
+  float scale_log2;
+  void* ws;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(THREADS, 2)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ DecArgs a) {
+  using C = Cfg<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + C::OFF_KV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + NS;
+  uint64_t* s_full = bars + 2 * NS;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* o_done = s_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const DecodeParams& p = a.p;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int G = p.H / p.KV;
+
+  int L = p.seqlens[b];
+  const int qp = p.qpos[b];
+  if (L < 0 || L > p.Lmax || qp < 0 || qp >= (1 << 24)) {
+    if (split == 0 && kvh == 0 && tid == 0) flag_error(p.status, DEV_BAD_ARG);
+    L = 0;
+  }
+  int j0 = split * a.chunk;
+  const int j1 = min(L, j0 + a.chunk);         // keys [j0, j1) of this split
+  if (p.window > 0) j0 = max(j0, qp - p.window + 1);
+  const int jt0 = j0 / BN, jt1 = (j1 - 1) / BN;  // tiles (empty when j0 >= j1)
+  const bool empty = j0 >= j1;
+
+  // partial-state layout: O [B][H][nsplit][hd], m [B][H][nsplit], l [B][H][nsplit]
+  float* wsO = static_cast<float*>(a.ws);
+  float* wsM = wsO + (size_t)p.B * p.H * a.nsplit * HD;
+  float* wsL = wsM + (size_t)p.B * p.H * a.nsplit;
+
+  if (empty) {
+    for (int h = tid; h < G; h += THREADS) {
+      const size_t pi = ((size_t)b * p.H + kvh * G + h) * a.nsplit + split;
+      wsM[pi] = -INFINITY;
+      wsL[pi] = 0.f;
+    }
+    return;
+  }
+
+  // ---- query tile: rows 0..G-1 = this group's heads turned at qpos, other rows zero
+  {
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q);
+    const int row = tid;  // one row per thread
+    for (int c = 0; c < HD / 8; ++c) {
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (row < G) {
+        const uint4 u = *reinterpret_cast<const uint4*>(q + ((size_t)b * p.H + kvh * G + row) * HD + c * 8);
+        const uint32_t in[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float2 f = bf2_to_f2(in[e]);
+          if (p.rope.on) {
+            float cs, sn;
+            rope_cos_sin(qp, p.rope.hi[c * 4 + e], p.rope.lo[c * 4 + e], cs, sn);
+            rotate_pair(f.x, f.y, cs, sn);
+          }
+          w[e] = f2_to_bf2(f.x, f.y);
+        }
+      }
+      *reinterpret_cast<uint4*>(sQ + sw128_offset(row, c * 8, BM)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_proxy_async();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(kv_full + i, 1);
+      mbar_init(kv_empty + i, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 32);
+    mbar_init(o_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;  // S: columns 0..127 (P over 0..63), O: 128..128+HD-1
+
+  if (warp == 1) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch(&tmK);
+      tma_prefetch(&tmV);
+      int u = 0;
+      for (int j = jt0; j <= jt1; ++j)
+        for (int kv = 0; kv < 2; ++kv, ++u) {
+          const int st = u % NS, n = u / NS;
+          if (!mbar_wait(kv_empty + st, (n & 1) ^ 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+          mbar_expect_tx(kv_full + st, C::KV_BYTES);
+          for (int kb = 0; kb < HD / 64; ++kb)
+            tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, kv ? &tmV : &tmK, kv_full + st,
+                        kb * 64, kvh, j * BN, b);
+        }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint64_t dQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t dV = smem_desc_sw128(smem_u32(sKV), BN * 128, 1024);
+      int u = 0, c = 0;
+      for (int j = jt0; j <= jt1; ++j, ++c) {
+        const int stK = u % NS, stV = (u + 1) % NS;
+        if (!mbar_wait(kv_full + stK, (u / NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        tc_fence_after();
+        const uint64_t bk = dK + (uint64_t)((stK * C::KV_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4;
+          umma_ss(tmem, dQ + off, bk + off, C::IDESC_QK, kk > 0);
+        }
+        umma_commit(s_full);
+        umma_commit(kv_empty + stK);
+        ++u;
+        if (!mbar_wait(kv_full + stV, (u / NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        if (!mbar_wait(p_full, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        tc_fence_after();
+        const uint64_t bv = dV + (uint64_t)((stV * C::KV_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ts(tmem + 128, tmem + kk * 8, bv + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
+                  (kk > 0 || c > 0) ? 1u : 0u);
+        umma_commit(o_done);
+        umma_commit(kv_empty + stV);
+        ++u;
+      }
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ softmax (lane = head)
+    const int h = kvh * G + lane;
+    const float slope = (p.alibi.on && lane < G) ? p.alibi.slope[h] * LOG2E : 0.f;
+    const float sc = a.scale_log2;
+    float m_ref = -INFINITY, l = 0.f;
+    int c = 0;
+    for (int j = jt0; j <= jt1; ++j, ++c) {
+      if (!mbar_wait(s_full, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      tc_fence_after();
+      const int key0 = j * BN;
+      const bool need_mask = key0 < j0 || key0 + BN > j1;
+      float m_exp = m_ref, rs = 0.f;
+#pragma unroll 1
+      for (int h2 = 0; h2 < BN / 64; ++h2) {
+        float xa[32], xb[32];
+        tmem_ld32(tmem + h2 * 64, xa);
+        tmem_ld32(tmem + h2 * 64 + 32, xb);
+        tmem_wait_ld();
+        float hx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const int ja = key0 + h2 * 64 + k, jb = ja + 32;
+          float va = p.alibi.on ? fmaf(xa[k], sc, -slope * fabsf((float)(qp - ja))) : xa[k] * sc;
+          float vb = p.alibi.on ? fmaf(xb[k], sc, -slope * fabsf((float)(qp - jb))) : xb[k] * sc;
+          if (need_mask) {
+            va = (ja >= j0 && ja < j1) ? va : -INFINITY;
+            vb = (jb >= j0 && jb < j1) ? vb : -INFINITY;
+          }
+          xa[k] = va;
+          xb[k] = vb;
+          hx = max3(hx, va, vb);
+        }
+        // same lazy reference as the prefill: move it only by more than 8 (log2 units)
+        const float m_cand = (hx > m_exp + 8.f) ? hx : m_exp;
+        if (__any_sync(0xffffffffu, m_cand != m_exp)) {
+          if (h2 > 0) {
+            const float f = (m_cand == m_exp) ? 1.f : ex2(m_exp - m_cand);
+            float pp[32];
+            tmem_wait_st();
+            tmem_ld32(tmem, pp);
+            tmem_wait_ld();
+            uint32_t pq[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const float2 v = bf2_to_f2(__float_as_uint(pp[k]));
+              pq[k] = f2_to_bf2(v.x * f, v.y * f);
+            }
+            tmem_st32u(tmem, pq);
+            rs *= f;
+          }
+          m_exp = m_cand;
+        }
+        const float mu = (m_exp == -INFINITY) ? 0.f : m_exp;
+        uint32_t pk[32];
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float e0 = ex2(xa[2 * k] - mu), e1 = ex2(xa[2 * k + 1] - mu);
+          const float e2 = ex2(xb[2 * k] - mu), e3 = ex2(xb[2 * k + 1] - mu);
+          rs0 += e0 + e1;
+          rs1 += e2 + e3;
+          pk[k] = f2_to_bf2(e0, e1);
+          pk[16 + k] = f2_to_bf2(e2, e3);
+        }
+        rs += rs0 + rs1;
+        tmem_st32u(tmem + h2 * 32, pk);
+      }
+      const float alpha = (m_exp == m_ref) ? 1.f : ex2(m_ref - m_exp);
+      m_ref = m_exp;
+      // rescale O (its previous PV finished before this tile's QK, which this tile waited for)
+      if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int q4 = 0; q4 < HD / 32; ++q4) {
+          float o[32];
+          tmem_ld32(tmem + 128 + q4 * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tmem_st32(tmem + 128 + q4 * 32, o);
+        }
+      }
+      l = l * alpha + rs;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // write this split's partial state
+    if (!mbar_wait(o_done, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+    tc_fence_after();
+    const size_t pi = ((size_t)b * p.H + h) * a.nsplit + split;
+#pragma unroll 1
+    for (int q4 = 0; q4 < HD / 32; ++q4) {
+      float o[32];
+      tmem_ld32(tmem + 128 + q4 * 32, o);
+      tmem_wait_ld();
+      if (lane < G) {
+        float4* dst = reinterpret_cast<float4*>(wsO + pi * HD + q4 * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_float4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
+      }
+    }
+    if (lane < G) {
+      // the merge kernel works in natural-log units
+      wsM[pi] = m_ref == -INFINITY ? -INFINITY : m_ref * 0.6931471805599453f;
+      wsL[pi] = l;
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 4-D map over the cache [B][Lmax][KV][hd] with a box of 128 slots x 64 features of one head.
+bool make_cache_map(CUtensorMap* map, const void* base, int B, int Lmax, int KV, int hd) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)KV, (cuuint64_t)Lmax, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)hd * 2, (cuuint64_t)KV * hd * 2, (cuuint64_t)Lmax * KV * hd * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int HD>
+cudaError_t launch_hd(const DecodeParams& p, int chunk, int nsplit, void* ws, cudaStream_t s) {
+  CUtensorMap mk, mv;
+  if (!make_cache_map(&mk, p.kcache, p.B, p.Lmax, p.KV, HD) || !make_cache_map(&mv, p.vcache, p.B, p.Lmax, p.KV, HD))
+    return cudaErrorInvalidValue;
+  DecArgs a;
+  a.p = p;
+  a.chunk = chunk;
+  a.nsplit = nsplit;
+  a.scale_log2 = p.scale * LOG2E;
+  a.ws = ws;
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg<HD>::SMEM);
+  if (e != cudaSuccess) return e;
+  decode_tc_kernel<HD><<<dim3(nsplit, p.KV, p.B), THREADS, Cfg<HD>::SMEM, s>>>(mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace tcdec
+
+bool decode_tc_supported(const DecodeParams& p, int dtype) {
+  const int G = p.H / p.KV;
+  return dtype == 1 && (p.hd == 64 || p.hd == 128) && G >= 1 && G <= 32 && tcdec::encode_fn() != nullptr;
+}
+
+cudaError_t launch_decode_tc(const DecodeParams& p, int chunk, int nsplit, void* ws, cudaStream_t s) {
+  return p.hd == 128 ? tcdec::launch_hd<128>(p, chunk, nsplit, ws, s)
+                     : tcdec::launch_hd<64>(p, chunk, nsplit, ws, s);
+}
+
+}  // namespace attn

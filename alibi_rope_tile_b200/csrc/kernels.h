@@ -52,6 +52,10 @@ struct DecodeParams {
 int decode_chunk(int B, int KV, int Lmax);
 size_t decode_workspace_bytes(int B, int H, int KV, int hd, int Lmax);
 cudaError_t launch_decode(const DecodeParams& p, int dtype, void* workspace, cudaStream_t s);
+// Tensor-core split pass (bf16, hd in {64, 128}, H/KV <= 32); writes the same partials as
+// the CUDA-core split pass, which the log-sum-exp merge then combines.
+bool decode_tc_supported(const DecodeParams& p, int dtype);
+cudaError_t launch_decode_tc(const DecodeParams& p, int chunk, int nsplit, void* ws, cudaStream_t s);
 
 struct AppendParams {
   const void* k_new;

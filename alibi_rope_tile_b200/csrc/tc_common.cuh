@@ -50,7 +50,7 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Slow path of mbar_wait: retries in suspended slices of 1 ms until the phase completes,
 // another role of the CTA gives up (``abort``), or ``limit_ns`` passes; in the last case
 // it records DEV_TIMEOUT in the device status word. Returns false when it gave up.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
                                             int* status, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
