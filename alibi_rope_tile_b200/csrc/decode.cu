@@ -316,14 +316,11 @@ __global__ void kv_append_kernel(const AppendParams p) {
 }  // namespace
 
 int decode_chunk(int B, int KV, int Lmax) {
-  // Enough splits for about four CTAs per SM on 148 SMs when every cache is full, with
-  // chunks a multiple of the 128-row key tile and at least 256 rows.
+  // Keys per split: 2048 (a multiple of the 128-key tile) unless that leaves fewer than
+  // about two CTAs per SM on 148 SMs when every cache is full; then smaller, down to 256.
   const long long units = (long long)B * KV;
-  long long want = (4LL * 148 + units - 1) / units;  // splits per (sequence, kv head)
-  if (want < 1) want = 1;
-  long long chunk = ((long long)Lmax + want - 1) / want;
-  chunk = ((chunk + 127) / 128) * 128;
-  if (chunk < 256) chunk = 256;
+  long long chunk = 2048;
+  while (chunk > 256 && units * (((long long)Lmax + chunk - 1) / chunk) < 2LL * 148) chunk /= 2;
   return (int)chunk;
 }
 

@@ -3,7 +3,8 @@
 // Memory", Part 3 "KV caching"); the splits are merged with the log-sum-exp rule of that
 // page's FlashAttention equations by the merge kernel in decode.cu.
 //
-// One CTA = one (split of the cache rows, key/value head, sequence). The H/KV query heads
+// One CTA = one (split of the cache rows, key/value head, sequence); splits are 2048 keys
+// (fewer CTAs amortise the set-up; see decode_chunk). The H/KV query heads
 // served by the key/value head are the rows of a 128-row MMA tile (rows >= H/KV are zero),
 // so the scores S = Q K^T of a 128-key tile land in tensor memory one head per TMEM lane:
 // the softmax of a head is a row-wise online softmax done by one thread, with no
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(THREADS, 2)
 
   const DecodeParams& p = a.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int kvh = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
   const int G = p.H / p.KV;
 
   int L = p.seqlens[b];
@@ -105,11 +106,12 @@ __global__ void __launch_bounds__(THREADS, 2)
     return;
   }
 
-  // ---- query tile: rows 0..G-1 = this group's heads turned at qpos, other rows zero
+  // ---- query tile: rows 0..G-1 = this group's heads turned at qpos, other rows zero.
+  // Work items are (row, 16-byte chunk) pairs spread over all threads.
   {
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q);
-    const int row = tid;  // one row per thread
-    for (int c = 0; c < HD / 8; ++c) {
+    for (int it = tid; it < BM * (HD / 8); it += THREADS) {
+      const int row = it / (HD / 8), c = it % (HD / 8);
       uint32_t w[4] = {0u, 0u, 0u, 0u};
       if (row < G) {
         const uint4 u = *reinterpret_cast<const uint4*>(q + ((size_t)b * p.H + kvh * G + row) * HD + c * 8);
@@ -356,7 +358,9 @@ cudaError_t launch_hd(const DecodeParams& p, int chunk, int nsplit, void* ws, cu
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg<HD>::SMEM);
   if (e != cudaSuccess) return e;
-  decode_tc_kernel<HD><<<dim3(nsplit, p.KV, p.B), THREADS, Cfg<HD>::SMEM, s>>>(mk, mv, a);
+  // split is the slowest grid dimension: the full leading splits of every sequence are
+  // scheduled before the (shorter, often empty) trailing ones
+  decode_tc_kernel<HD><<<dim3(p.KV, p.B, nsplit), THREADS, Cfg<HD>::SMEM, s>>>(mk, mv, a);
   return cudaGetLastError();
 }
 
