@@ -32,6 +32,8 @@ SIGNATURES = {
     "attn_decode_workspace_size": (_S, [_I, _I, _I, _I, _I]),
     "attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _FP, _I, _P, _S,
                          _P]),
+    "attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _FP, _I,
+                                 _P]),
     "attn_kv_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "attn_block_workspace_size": (_S, [_I, _I, _I, _I, _I, _I, _I]),
     "attn_block": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _L, _F, _I, _I, _FP, _I,
@@ -157,6 +159,23 @@ def attn_decode(q, kcache, vcache, seqlens, qpos, out=None, lse=None, workspace=
                            float(rope_base), int(window), _slopes(alibi_slopes, H), _dtype(q),
                            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                            _stream(stream))
+    _check(st)
+    return out
+
+
+def attn_decode_noalloc(q, kcache, vcache, seqlens, qpos, out, lse=None, *,
+                        rope_base: float = 0.0, window: int = 0, alibi_slopes=None, stream=None):
+    """attn_decode for callers that cannot allocate device memory: the split partials use
+    the library's fixed scratch array, so no workspace is passed; ``out`` must be given."""
+    B, H, hd = q.shape
+    _, Lmax, KV, _ = kcache.shape
+    dt = q.dtype
+    st = lib().attn_decode_noalloc(_dev(q, "q"), _dev(kcache, "kcache", dt),
+                                   _dev(vcache, "vcache", dt), _dev(seqlens, "seqlens", torch.int32),
+                                   _dev(qpos, "qpos", torch.int32), _dev(out, "out", dt),
+                                   _dev(lse, "lse", torch.float32), B, H, KV, hd, Lmax,
+                                   float(rope_base), int(window), _slopes(alibi_slopes, H),
+                                   _dtype(q), _stream(stream))
     _check(st)
     return out
 

@@ -37,6 +37,10 @@ int cuda_fail(cudaError_t e, const char* where) {
 
 }  // namespace
 
+namespace attn {
+int record_error(int code, const char* message) { return fail(code, "%s", message); }
+}  // namespace attn
+
 // Per-device status word written by kernels that find a bad device-resident argument or
 // give up on a bounded wait. Host code reaches it through cudaGetSymbolAddress.
 __device__ int g_attn_device_status;

@@ -77,4 +77,8 @@ bool gemm_tc_supported(int M, int N, int K, int dtype);
 cudaError_t launch_gemm_tc(const void* A, const void* W, void* C, int M, int N, int K,
                            cudaStream_t s);
 
+// Records a failure for attn_last_error() and returns ``code`` (used by entry points
+// defined outside api.cu).
+int record_error(int code, const char* message);
+
 }  // namespace attn

@@ -120,6 +120,33 @@ int attn_decode(const void* q, const void* kcache, const void* vcache, const int
                 void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * attn_decode_noalloc -- attn_decode for callers that cannot allocate device memory.
+ *
+ * There is no counterpart to this entry point on the pages; it exists for callers that
+ * must not call cudaMalloc (or any allocating library routine) and cannot hand over a
+ * workspace: code running under an allocator or memory budget that it does not own (a
+ * plugin inside another framework's memory pool), or a latency-critical step where an
+ * allocation, which may synchronise the device, is not allowed.
+ *
+ * Arguments and results are those of attn_decode without workspace/ws_bytes. The split
+ * partials live in a fixed scratch array of ATTN_DECODE_NOALLOC_MAX_SCRATCH bytes that is
+ * part of the library's device image: every GPU that loads the library holds it until the
+ * process exits. Sizes whose attn_decode_workspace_size() exceeds that maximum are
+ * rejected with ATTN_ERR_UNSUPPORTED and a message naming the limit; nothing is launched.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * once per device, with that device current); make that first call before any stream
+ * capture. Every call on a device shares the one array and leaves its contents behind:
+ * nothing in it needs to start at zero, but two calls that overlap on the GPU (different
+ * streams without ordering between them) race on it and may return wrong results.
+ * The entry point allocates nothing.
+ */
+#define ATTN_DECODE_NOALLOC_MAX_SCRATCH ((size_t)8 << 20)
+int attn_decode_noalloc(const void* q, const void* kcache, const void* vcache, const int* seqlens,
+                        const int* qpos, void* out, float* lse, int B, int H, int KV, int hd,
+                        int Lmax, float rope_base, int window, const float* alibi_slopes,
+                        int dtype, void* stream);
+
+/*
  * attn_kv_append -- write one new token per sequence into the cache ([XF5] "KV caching";
  * [FLASH] roadmap: preallocate the cache and write by position).
  * k_new, v_new: [B,KV,hd] (device). pos: [B] int32 (device) slot = position of the token.
