@@ -4,9 +4,10 @@ One step = one pass of the whole hot path over one batch of synthetic input:
   * prefill of the GQA workload (B=2, T=4096, H=32, KV=8, hd=128, causal, RoPE base 5e5):
     RoPE on load, QK^T, mask, online softmax, PV, epilogue;
   * one decode step of the KV-cache workload (batch 64, H=32, KV=8, hd=128, cache lengths
-    uniform in [1024, 8192]): split-KV partials and the log-sum-exp merge.
+    uniform in [1024, 8192]) and of its MQA variant (KV=1): split-KV partials and the
+    log-sum-exp merge.
 ``value`` is the prefill TFLOP/s (causal FLOPs counted: 4*B*H*hd*allowed pairs); the decode
-GB/s rides along under ``decode``. Kernels are timed with CUDA events on the stream they
+GB/s (cache rows read + q + out, per launch pair) ride along under ``decode``. Kernels are timed with CUDA events on the stream they
 are launched on; L2 is flushed (a 256 MiB memset, outside the timed events) before every
 step. ``e2e`` times the same call with the step's inputs copied from pinned host memory and
 its output copied back, all inside the timed region.
@@ -39,10 +40,11 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 METRIC = "causal GQA prefill TFLOP/s and decode HBM GB/s on 1 B200, % of roofline"
 PREFILL = workloads.GQA
 DECODE = workloads.DECODE_GQA
+DECODE_MQA = workloads.DECODE_MQA
 # Algorithmic bytes and launches, stated once (see the design notes):
 #   decode bytes = cache rows read (K and V) + q + out; prefill FLOPs = PREFILL.flops.
 PREFILL_LAUNCHES = 1
-DECODE_LAUNCHES = 2
+DECODE_LAUNCHES = 2       # split pass + merge, per decode workload
 
 
 def peaks():
@@ -53,6 +55,30 @@ def peaks():
         p["source"] = "measured"
         return p
     return dict(PEAKS_FALLBACK)
+
+
+def csrc_sha256() -> str:
+    """Hash of the CUDA sources: DRAM counters taken with other sources are not reported."""
+    import hashlib
+    d = os.path.join(ROOT, "alibi_rope_tile_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic() -> dict:
+    """Per-launch DRAM bytes (read + write) from profiles/traffic.json, or {} when the file
+    was written for different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return {}
+    with open(path) as f:
+        t = json.load(f)
+    if t.get("csrc_sha256") != csrc_sha256():
+        return {}
+    return t.get("per_launch_dram_bytes", {})
 
 
 def decode_bytes(seqlens, w) -> int:
@@ -143,24 +169,26 @@ def cpu_cores() -> int:
 
 
 def oracle_sample_tflops(budget_s: float = 12.0):
-    """The fp64 oracle on a bounded sample of the prefill workload (rows of the first
-    sequence, the four query heads of key/value head 0), as TFLOP/s of causal FLOPs."""
+    """The fp64 oracle on a bounded sample of the prefill workload, as TFLOP/s of causal
+    FLOPs: sequence 0, one key/value group (4 query heads) at a time, all 4096 rows, until
+    the time budget is spent (about 1 s per group on 16 cores)."""
     from oracle import attention as A
     w = PREFILL
     q, k, v = workloads.prefill_inputs(w)
-    q, k, v = q[:1, :, :4], k[:1, :, :1], v[:1, :, :1]
-    rows_all = torch.arange(w.T).numpy()
+    group = w.H // w.KV
+    pairs = w.T * (w.T + 1) // 2
     flops = done = 0
     t0 = time.perf_counter()
-    chunk = 512
-    while time.perf_counter() - t0 < budget_s and done < w.T:
-        rows = rows_all[w.T - done - chunk: w.T - done] if done + chunk <= w.T else rows_all[:w.T - done]
-        A.attention(q, k, v, rope_base=w.rope_base, causal=True, rows=rows)
-        flops += 4 * 4 * w.hd * int((rows + 1).sum())
-        done += len(rows)
+    for g in range(w.KV):
+        if time.perf_counter() - t0 >= budget_s:
+            break
+        A.attention(q[:1, :, g * group:(g + 1) * group], k[:1, :, g:g + 1], v[:1, :, g:g + 1],
+                    rope_base=w.rope_base, causal=True)
+        flops += 4 * group * w.hd * pairs
+        done += 1
     dt = time.perf_counter() - t0
-    sample = (f"GQA prefill, batch 0, query heads 0-3 (key/value head 0), last {done} of "
-              f"{w.T} rows, full key range, fp64 numpy/OpenBLAS")
+    sample = (f"GQA prefill, sequence 0, {done} of {w.KV} key/value groups ({done * group} of "
+              f"{w.H} query heads), all {w.T} rows, fp64 numpy/OpenBLAS")
     return flops / dt / 1e12, dt, sample
 
 
@@ -194,38 +222,43 @@ def run_ours(args, rank, world):
     art.lib()
     dev = torch.cuda.current_device()
     stream = torch.cuda.current_stream()
-    w, dw = PREFILL, DECODE
-
+    w = PREFILL
     do_p, do_d = args.only in ("all", "prefill"), args.only in ("all", "decode")
+
     q, k, v = workloads.prefill_inputs(w)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
     dout = torch.empty_like(dq)
-    dbytes = 1
+    decs = []
     if do_d:
-        dq_, dkc, dvc, dsl, dqp = workloads.decode_inputs(dw)
-        dbytes = decode_bytes(dsl, dw)
-        ddq, dkc, dvc, dsl, dqp = dq_.cuda(), dkc.cuda(), dvc.cuda(), dsl.cuda(), dqp.cuda()
-        ddout = torch.empty_like(ddq)
-        ws = torch.empty(art.attn_decode_workspace_size(dw.B, dw.H, dw.KV, dw.hd, dw.Lmax),
-                         dtype=torch.uint8, device="cuda")
+        for dw in (DECODE, DECODE_MQA):
+            hq, hkc, hvc, hsl, hqp = workloads.decode_inputs(dw)
+            decs.append(dict(
+                w=dw, bytes=decode_bytes(hsl, dw), hq=hq,
+                q=hq.cuda(), kc=hkc.cuda(), vc=hvc.cuda(), sl=hsl.cuda(), qp=hqp.cuda(),
+                out=torch.empty(hq.shape, dtype=hq.dtype, device="cuda"),
+                ws=torch.empty(art.attn_decode_workspace_size(dw.B, dw.H, dw.KV, dw.hd, dw.Lmax),
+                               dtype=torch.uint8, device="cuda")))
+            del hkc, hvc
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
     def prefill():
         if do_p:
             art.attn_prefill(dq, dk, dv, dout, rope_base=w.rope_base, causal=True, window=w.window)
 
-    def decode():
-        if do_d:
-            art.attn_decode(ddq, dkc, dvc, dsl, dqp, ddout, workspace=ws, rope_base=dw.rope_base)
+    def decode(d):
+        art.attn_decode(d["q"], d["kc"], d["vc"], d["sl"], d["qp"], d["out"], workspace=d["ws"],
+                        rope_base=d["w"].rope_base)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
         prefill()
-        decode()
+        for d in decs:
+            decode(d)
     torch.cuda.synchronize()
     art.attn_sync_status()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    nev = 2 + 2 * len(decs)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     clocks = Clocks(dev)
@@ -233,88 +266,105 @@ def run_ours(args, rank, world):
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_begin.record(stream)
-    for s in range(args.steps):
+    for s_ in range(args.steps):
         flush.zero_()
-        ev[s][0].record(stream)
+        ev[s_][0].record(stream)
         prefill()
-        ev[s][1].record(stream)
-        ev[s][2].record(stream)
-        decode()
-        ev[s][3].record(stream)
+        ev[s_][1].record(stream)
+        for n, d in enumerate(decs):
+            flush.zero_()
+            ev[s_][2 + 2 * n].record(stream)
+            decode(d)
+            ev[s_][3 + 2 * n].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
     art.attn_sync_status()
-    p_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
-    d_ms = [ev[s][2].elapsed_time(ev[s][3]) for s in range(args.steps)]
-    p_tot = max(1e-9, max_over_ranks(sum(p_ms), world))
-    d_tot = max(1e-9, max_over_ranks(sum(d_ms), world))
+    p_tot = max(1e-9, max_over_ranks(sum(ev[s_][0].elapsed_time(ev[s_][1]) for s_ in range(args.steps)), world))
+    d_tot = [max(1e-9, max_over_ranks(sum(ev[s_][2 + 2 * n].elapsed_time(ev[s_][3 + 2 * n])
+                                          for s_ in range(args.steps)), world))
+             for n in range(len(decs))]
     region_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
 
-    # end to end: pinned host inputs -> device -> prefill -> host output, every step
+    # end to end through the public API: the step's inputs go host (pinned) -> device, the
+    # kernels run, the results come back device -> host; all inside the timed region
     hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
     hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hdec = [(d["hq"].pin_memory(), torch.empty(d["hq"].shape, dtype=d["hq"].dtype).pin_memory())
+            for d in decs]
+
+    def e2e_step():
+        if do_p:
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            prefill()
+            hout.copy_(dout, non_blocking=True)
+        for d, (hdq, hdo) in zip(decs, hdec):
+            d["q"].copy_(hdq, non_blocking=True)
+            decode(d)
+            hdo.copy_(d["out"], non_blocking=True)
+
     for _ in range(2):
-        dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
-        prefill()
-        hout.copy_(dout, non_blocking=True)
+        e2e_step()
     torch.cuda.synchronize()
     barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
-        prefill()
-        hout.copy_(dout, non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-
-    pk = peaks()
-    flops_step = w.flops
-    tflops = world * flops_step * args.steps / (p_tot * 1e-3) / 1e12
-    per_launch_ms = p_tot / args.steps
-    achieved = flops_step / (per_launch_ms * 1e-3) / 1e12
-    d_gbs = world * dbytes * args.steps / (d_tot * 1e-3) / 1e9
-    d_per = d_tot / args.steps
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof):
-        with open(prof) as f:
-            traffic = json.load(f).get("prefill_tc")
 
     if rank != 0:
         return
     if args.only != "all":
         print(json.dumps({"only": args.only, "prefill_ms": p_tot / args.steps,
-                          "decode_ms": d_tot / args.steps}), flush=True)
+                          "decode_ms": [t / args.steps for t in d_tot]}), flush=True)
         return
+    pk = peaks()
+    flops_step = w.flops
+    per_launch_ms = p_tot / args.steps
+    achieved = flops_step / (per_launch_ms * 1e-3) / 1e12
+    traffic = measured_traffic()
+    decode_out = {}
+    for n, d in enumerate(decs):
+        ms = d_tot[n] / args.steps
+        gbs = d["bytes"] / (ms * 1e-3) / 1e9
+        decode_out[d["w"].name] = {
+            "value": world * gbs, "unit": "GB/s", "ms": ms, "bytes": d["bytes"],
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": traffic.get(d["w"].name),
+                         "peak_source": f"{pk.get('source')} copy"}}
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v)) + sum(
+        d["hq"].numel() * d["hq"].element_size() for d in decs)
+    d2h = q.numel() * q.element_size() + sum(d["hq"].numel() * d["hq"].element_size() for d in decs)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         val, dt, sample = oracle_sample_tflops()
         cpu = {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                "sample": sample, "seconds": round(dt, 2)}
     line = {
-        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": (p_tot + d_tot) / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": world * flops_step * args.steps / (p_tot * 1e-3) / 1e12,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": (p_tot + sum(d_tot)) / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "decode_workload": dw.name, "parallelism": f"replicas{world}",
-                   "l2": "flushed: 256 MiB memset before every step, outside the kernel events",
+        "config": {"workload": w.name, "decode_workloads": [d["w"].name for d in decs],
+                   "parallelism": f"replicas{world}",
+                   "l2": "flushed: 256 MiB memset before every kernel family, outside the events",
                    "timed_region_ms": region_ms},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
+                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                     "traffic": traffic.get(w.name), "kernel": "prefill_tc_kernel<128>",
                      "peak_source": f"{pk.get('source')} burst bf16 dense"},
-        "decode": {"value": d_gbs, "unit": "GB/s", "ms": d_per, "bytes": dbytes,
-                   "roofline": {"bound": "hbm", "achieved": dbytes / (d_per * 1e-3) / 1e9,
-                                "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                "frac": dbytes / (d_per * 1e-3) / 1e9 / pk["hbm_gbs"],
-                                "traffic": None, "peak_source": f"{pk.get('source')} copy"}},
-        "e2e": {"value": world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": int(3 * 0 + q.numel() * 2 + k.numel() * 2 + v.numel() * 2),
-                "d2h_bytes_per_step": int(q.numel() * 2)},
-        "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES),
+        "decode": decode_out,
+        "e2e": {"value": world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12,
+                "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": e2e_ms / args.steps,
+                "note": "prefill FLOPs over the whole step incl. copies and both decodes"},
+        "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES * len(decs)),
         "clocks": clk,
         "cpu_baseline": cpu,
     }
