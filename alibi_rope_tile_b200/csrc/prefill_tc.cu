@@ -306,6 +306,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t dQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
       const uint64_t dV = smem_desc_sw128(smem_u32(sKV), BN * 128, 1024);
+      int tcnt = 0;
       auto issue_qk = [&](int s, int st) {
         const uint32_t d = tmem + s * BN;
         const uint64_t a0 = dQ + (uint64_t)((s * C::Q_BYTES) >> 4);
@@ -321,12 +322,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t aP = tmem + s * BN;  // P: 64 columns of bf16 pairs over S
         const uint64_t b0 = dV + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
+        for (int kk = 0; kk < BN / 16; ++kk) {
           umma_ts(d, aP + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
                   (kk > 0 || acc) ? 1u : 0u);
+          if (kk == 0 || kk == 3) TRACE(0, tcnt, 40 + kk);
+        }
       };
       int cnt[2] = {0, 0};
-      int tcnt = 0;
       if (!mbar_wait(q_rot, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
       // K of the first tile
       if (!mbar_wait(k_rot + 0, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
