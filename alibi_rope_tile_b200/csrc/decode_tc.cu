@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           w[e] = f2_to_bf2(f.x, f.y);
         }
       }
-      *reinterpret_cast<uint4*>(sQ + sw128_offset(row, c * 8, BM)) = make_uint4(w[0], w[1], w[2], w[3]);
+      sts128(smem_u32(sQ) + sw128_offset(row, c * 8, BM), make_uint4(w[0], w[1], w[2], w[3]));
     }
     fence_proxy_async();
   }

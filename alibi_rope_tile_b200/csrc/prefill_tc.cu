@@ -138,11 +138,12 @@ struct KRot {
       SC[h] = pk2(stepc[2 * h], stepc[2 * h + 1]);
       SS[h] = pk2(steps[2 * h], steps[2 * h + 1]);
     }
-#pragma unroll 2
+    const uint32_t base = smem_u32(tile);
+#pragma unroll 4
     for (int k = 0; k < NR; ++k) {
       const int r = phase + PH * k;
-      uint4* ptr = reinterpret_cast<uint4*>(tile + sw128_offset(r, chunk * 8, BN));
-      const uint4 u = *ptr;
+      const uint32_t addr = base + sw128_offset(r, chunk * 8, BN);
+      const uint4 u = lds128(addr);
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
       uint32_t o[4];
 #pragma unroll
@@ -163,7 +164,7 @@ struct KRot {
         C[h] = Cn;
         N[h] = neg2(S[h]);
       }
-      *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+      sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
     }
   }
 };
