@@ -236,8 +236,9 @@ BlockLayout block_layout(int B, int T, int H, int KV, int hd, int dtype) {
   L.total = L.ctx + round256(nq);
   return L;
 }
-cudaError_t gemm(const void* A, const void* W, void* C, int M, int N, int K, int dtype, cudaStream_t s) {
-  if (gemm_tc_supported(M, N, K, dtype)) return launch_gemm_tc(A, W, C, M, N, K, s);
+cudaError_t gemm(const void* A, const void* W, void* C, int M, int N, int K, int dtype, int* status,
+               cudaStream_t s) {
+  if (gemm_tc_supported(M, N, K, dtype)) return launch_gemm_tc(A, W, C, M, N, K, status, s);
   return launch_gemm_simt(A, W, C, M, N, K, dtype, s);
 }
 }  // namespace
@@ -269,14 +270,17 @@ int attn_block(const void* x, const void* Wq, const void* Wk, const void* Wv, co
   void *q = ws + L.q, *k = ws + L.k, *v = ws + L.v, *ctx = ws + L.ctx;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int M = B * T;
+  int err = 0;
+  int* status = device_status(&err);
+  if (!status) return err;
   cudaError_t e;
-  if ((e = gemm(x, Wq, q, M, H * hd, d, dtype, s)) != cudaSuccess) return cuda_fail(e, "block Wq GEMM");
-  if ((e = gemm(x, Wk, k, M, KV * hd, d, dtype, s)) != cudaSuccess) return cuda_fail(e, "block Wk GEMM");
-  if ((e = gemm(x, Wv, v, M, KV * hd, d, dtype, s)) != cudaSuccess) return cuda_fail(e, "block Wv GEMM");
+  if ((e = gemm(x, Wq, q, M, H * hd, d, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wq GEMM");
+  if ((e = gemm(x, Wk, k, M, KV * hd, d, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wk GEMM");
+  if ((e = gemm(x, Wv, v, M, KV * hd, d, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wv GEMM");
   st = attn_prefill(q, k, v, ctx, nullptr, B, T, H, KV, hd, pos0, rope_base, causal, window,
                     alibi_slopes, dtype, stream);
   if (st) return st;
-  if ((e = gemm(ctx, Wo, out, M, d, H * hd, dtype, s)) != cudaSuccess) return cuda_fail(e, "block Wo GEMM");
+  if ((e = gemm(ctx, Wo, out, M, d, H * hd, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wo GEMM");
   return ok();
 }
 

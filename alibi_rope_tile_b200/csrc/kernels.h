@@ -74,7 +74,7 @@ cudaError_t launch_gemm_simt(const void* A, const void* W, void* C, int M, int N
                              cudaStream_t s);
 // Tensor-core (tcgen05) version for bf16 when M, N, K fit its tiles.
 bool gemm_tc_supported(int M, int N, int K, int dtype);
-cudaError_t launch_gemm_tc(const void* A, const void* W, void* C, int M, int N, int K,
+cudaError_t launch_gemm_tc(const void* A, const void* W, void* C, int M, int N, int K, int* status,
                            cudaStream_t s);
 
 // Records a failure for attn_last_error() and returns ``code`` (used by entry points

@@ -49,7 +49,8 @@ def test_tiny_block_lab_properties_on_gpu(art):
     assert (out3 - out).abs().max().item() <= 1e-5
 
 
-@pytest.mark.parametrize("shape", [(2, 256, 512, 8, 2), (1, 300, 256, 4, 4)])
+@pytest.mark.parametrize("shape", [(2, 256, 512, 8, 2), (1, 300, 256, 4, 4), (1, 1024, 2048, 16, 4),
+                                   (1, 200, 1040, 8, 8)])
 def test_bf16_block(art, shape):
     B, T, d, H, KV = shape
     hd = d // H
