@@ -20,6 +20,8 @@
 // qpos - j >= window get weight exactly 0.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
+
 #include "kernels.h"
 #include "tc_common.cuh"
 
@@ -34,6 +36,7 @@ constexpr int BM = 128;               // MMA rows (query heads, zero padded)
 constexpr int NS = 2;                 // ring stages (K, V alternate)
 constexpr int THREADS = 128;
 constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
+constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;  // own copies/MMAs finish in microseconds
 constexpr float LOG2E = 1.4426950408889634f;
 
 template <int HD>
@@ -42,7 +45,7 @@ struct Cfg {
   static constexpr int KV_BYTES = BN * HD * 2;
   static constexpr int OFF_KV = Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
-  static constexpr int NBAR = 2 * NS + 3;  // kv_full[NS], kv_empty[NS], s_full, p_full, o_done
+  static constexpr int NBAR = 2 * NS + 5;  // kv_full[NS], kv_empty[NS], s_full, p_full, o_done, never, drain
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
@@ -55,6 +58,8 @@ struct DecArgs {
   int nsplit;
   float scale_log2;
   void* ws;
+  unsigned long long wait_ns;  // bound of every wait (4 s unless a test lowers it)
+  int test_stall;              // test hook: the MMA warp waits on a barrier nothing signals
 };
 
 template <int HD>
@@ -72,6 +77,8 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint64_t* s_full = bars + 2 * NS;
   uint64_t* p_full = s_full + 1;
   uint64_t* o_done = s_full + 2;
+  uint64_t* never = s_full + 3;  // not signalled by anything (test hook)
+  uint64_t* drain = s_full + 4;  // the MMA thread's final commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -139,6 +146,8 @@ __global__ void __launch_bounds__(THREADS, 2)
     mbar_init(s_full, 1);
     mbar_init(p_full, 32);
     mbar_init(o_done, 1);
+    mbar_init(never, 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -156,16 +165,20 @@ __global__ void __launch_bounds__(THREADS, 2)
     if (lane == 0) {
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
+      const int total = 2 * (jt1 - jt0 + 1);  // K and V of every tile
       int u = 0;
-      for (int j = jt0; j <= jt1; ++j)
-        for (int kv = 0; kv < 2; ++kv, ++u) {
-          const int st = u % NS, n = u / NS;
-          if (!mbar_wait(kv_empty + st, (n & 1) ^ 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-          mbar_expect_tx(kv_full + st, C::KV_BYTES);
-          for (int kb = 0; kb < HD / 64; ++kb)
-            tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, kv ? &tmV : &tmK, kv_full + st,
-                        kb * 64, kvh, j * BN, b);
-        }
+      for (; u < total; ++u) {
+        const int st = u % NS, n = u / NS, j = jt0 + u / 2;
+        if (!mbar_wait(kv_empty + st, (n & 1) ^ 1, abort_flag, p.status, a.wait_ns)) break;
+        mbar_expect_tx(kv_full + st, C::KV_BYTES);
+        for (int kb = 0; kb < HD / 64; ++kb)
+          tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, (u & 1) ? &tmV : &tmK, kv_full + st,
+                      kb * 64, kvh, j * BN, b);
+      }
+      // The loads of the last NS uses land before the CTA exits (immediate when the MMA
+      // warp consumed them; after an abort they may still be in flight).
+      for (int w = (u > NS ? u - NS : 0); w < u; ++w)
+        mbar_wait_drain(kv_full + w % NS, (w / NS) & 1, DRAIN_LIMIT_NS);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ MMA issue
@@ -174,9 +187,10 @@ __global__ void __launch_bounds__(THREADS, 2)
       const uint64_t dK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
       const uint64_t dV = smem_desc_sw128(smem_u32(sKV), BN * 128, 1024);
       int u = 0, c = 0;
+      if (a.test_stall && !mbar_wait(never, 0, abort_flag, p.status, a.wait_ns)) goto mma_drain;
       for (int j = jt0; j <= jt1; ++j, ++c) {
         const int stK = u % NS, stV = (u + 1) % NS;
-        if (!mbar_wait(kv_full + stK, (u / NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        if (!mbar_wait(kv_full + stK, (u / NS) & 1, abort_flag, p.status, a.wait_ns)) goto mma_drain;
         tc_fence_after();
         const uint64_t bk = dK + (uint64_t)((stK * C::KV_BYTES) >> 4);
 #pragma unroll
@@ -187,8 +201,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         umma_commit(s_full);
         umma_commit(kv_empty + stK);
         ++u;
-        if (!mbar_wait(kv_full + stV, (u / NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        if (!mbar_wait(p_full, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        if (!mbar_wait(kv_full + stV, (u / NS) & 1, abort_flag, p.status, a.wait_ns)) goto mma_drain;
+        if (!mbar_wait(p_full, c & 1, abort_flag, p.status, a.wait_ns)) goto mma_drain;
         tc_fence_after();
         const uint64_t bv = dV + (uint64_t)((stV * C::KV_BYTES) >> 4);
 #pragma unroll
@@ -199,6 +213,10 @@ __global__ void __launch_bounds__(THREADS, 2)
         umma_commit(kv_empty + stV);
         ++u;
       }
+    mma_drain:
+      // every MMA issued above completes before tensor memory is released
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0, DRAIN_LIMIT_NS);
     }
   } else if (warp == 0) {
     // ------------------------------------------------------------ softmax (lane = head)
@@ -208,7 +226,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     float m_ref = -INFINITY, l = 0.f;
     int c = 0;
     for (int j = jt0; j <= jt1; ++j, ++c) {
-      if (!mbar_wait(s_full, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      if (!mbar_wait(s_full, c & 1, abort_flag, p.status, a.wait_ns)) goto done;
       tc_fence_after();
       const int key0 = j * BN;
       const bool need_mask = key0 < j0 || key0 + BN > j1;
@@ -288,7 +306,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       mbar_arrive(p_full);
     }
     // write this split's partial state
-    if (!mbar_wait(o_done, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+    if (!mbar_wait(o_done, (c - 1) & 1, abort_flag, p.status, a.wait_ns)) goto done;
     tc_fence_after();
     const size_t pi = ((size_t)b * p.H + h) * a.nsplit + split;
 #pragma unroll 1
@@ -355,6 +373,19 @@ cudaError_t launch_hd(const DecodeParams& p, int chunk, int nsplit, void* ws, cu
   a.nsplit = nsplit;
   a.scale_log2 = p.scale * LOG2E;
   a.ws = ws;
+  // Test hook (failure detection without a GPU fault): with ATTN_TEST_DECODE_STALL_NS set
+  // to a positive number of nanoseconds, every wait of this kernel is bounded by it and
+  // the MMA warp first waits on a barrier that nothing signals, so each CTA gives up,
+  // records ATTN_ERR_TIMEOUT in the device status word, drains its own copies and exits.
+  a.wait_ns = WAIT_LIMIT_NS;
+  a.test_stall = 0;
+  if (const char* e = std::getenv("ATTN_TEST_DECODE_STALL_NS")) {
+    const long long ns = std::atoll(e);
+    if (ns > 0) {
+      a.wait_ns = (unsigned long long)ns;
+      a.test_stall = 1;
+    }
+  }
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg<HD>::SMEM);
   if (e != cudaSuccess) return e;

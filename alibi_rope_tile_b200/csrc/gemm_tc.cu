@@ -26,9 +26,10 @@ constexpr int A_BYTES = BM * BK * 2;       // 16 KB
 constexpr int B_BYTES = BK * BN * 2;       // 32 KB
 constexpr int STAGE = A_BYTES + B_BYTES;
 constexpr int OFF_BAR = NS * STAGE;
-constexpr int SMEM = OFF_BAR + (2 * NS + 1) * 8 + 16 + 1024;
+constexpr int SMEM = OFF_BAR + (2 * NS + 2) * 8 + 16 + 1024;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 1);
 constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
+constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;
 
 struct GemmArgs {
   __nv_bfloat16* C;
@@ -44,8 +45,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* empty = full + NS;
   uint64_t* acc_full = full + 2 * NS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(acc_full + 1) + 1;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1) + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
@@ -57,6 +59,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(empty + i, 1);
     }
     mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -73,7 +76,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       tma_prefetch(&tmA);
       tma_prefetch(&tmW);
-      for (int kb = 0; kb < nk; ++kb) {
+      int kb = 0;
+      for (; kb < nk; ++kb) {
         const int st = kb % NS, n = kb / NS;
         if (!mbar_wait(empty + st, (n & 1) ^ 1, abort_flag, g.status, WAIT_LIMIT_NS)) break;
         uint8_t* sa = smem + st * STAGE;
@@ -84,6 +88,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int nb = 0; nb < nbv; ++nb)
           tma_load_2d(sa + A_BYTES + nb * (BK * 128), &tmW, full + st, n0 + nb * 64, kb * BK);
       }
+      // the copies issued last land before the CTA exits
+      for (int w = (kb > NS ? kb - NS : 0); w < kb; ++w) mbar_wait_drain(full + w % NS, (w / NS) & 1, DRAIN_LIMIT_NS);
     }
   } else if (warp == 5) {
     if (lane == 0) {
@@ -101,6 +107,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma_commit(empty + st);
       }
       umma_commit(acc_full);
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0, DRAIN_LIMIT_NS);  // every MMA completes before TMEM is freed
     }
   } else {
     // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = rows m0 + 32*w .. of C

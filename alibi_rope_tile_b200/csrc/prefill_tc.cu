@@ -55,6 +55,7 @@ constexpr int WARP_ROPE0 = 8;
 constexpr int WARP_TMA = 12;
 constexpr int WARP_MMA = 13;
 constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;  // a wait that lasts 4 s has failed
+constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;  // own copies/MMAs finish in microseconds
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -81,7 +82,7 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
-  static constexpr int NBAR = 3 * NS + 8;
+  static constexpr int NBAR = 3 * NS + 9;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KiB
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
@@ -187,6 +188,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* s_full = q_full + 2;
   uint64_t* p_full = q_full + 4;
   uint64_t* o_done = q_full + 6;
+  uint64_t* drain = q_full + 8;  // the MMA thread's final commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -239,6 +241,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(p_full + s, 128);
       mbar_init(o_done + s, 1);
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -263,18 +266,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (valid[s])
           for (int kb = 0; kb < HD / 64; ++kb)
             tma_load_4d(sQ + s * C::Q_BYTES + kb * BM * 128, &tmQ, q_full, kb * 64, head[s], qs[s], b);
-      int u = 0, tcnt = 0;
-      for (int j = jt0; j <= jt1; ++j) {
-        for (int kv = 0; kv < 2; ++kv, ++u) {
-          const int st = u % C::NS, n = u / C::NS;
-          if (!mbar_wait(kv_empty + st, (n & 1) ^ 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-          TRACE(4, tcnt, 30 + kv);
-          mbar_expect_tx(kv_full + st, C::KV_BYTES);
-          for (int kb = 0; kb < HD / 64; ++kb)
-            tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, kv ? &tmV : &tmK, kv_full + st,
-                        kb * 64, g, j * BN, b);
-        }
+      int tcnt = 0;
+      const int total = 2 * (jt1 - jt0 + 1);  // K and V of every tile
+      int u = 0;
+      for (; u < total; ++u) {
+        const int st = u % C::NS, n = u / C::NS, j = jt0 + u / 2, kv = u & 1;
+        if (!mbar_wait(kv_empty + st, (n & 1) ^ 1, abort_flag, p.status, WAIT_LIMIT_NS)) break;
+        TRACE(4, tcnt, 30 + kv);
+        mbar_expect_tx(kv_full + st, C::KV_BYTES);
+        for (int kb = 0; kb < HD / 64; ++kb)
+          tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, kv ? &tmV : &tmK, kv_full + st,
+                      kb * 64, g, j * BN, b);
       }
+      // The copies issued last land before the CTA exits (immediate when they were
+      // consumed; after an abort they may still be in flight).
+      mbar_wait_drain(q_full, 0, DRAIN_LIMIT_NS);
+      for (int w = (u > C::NS ? u - C::NS : 0); w < u; ++w)
+        mbar_wait_drain(kv_full + w % C::NS, (w / C::NS) & 1, DRAIN_LIMIT_NS);
     }
   } else if (warp >= WARP_ROPE0 && warp < WARP_ROPE0 + 4) {
     // ------------------------------------------------------------ rotary embedding
@@ -330,9 +338,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       };
       int cnt[2] = {0, 0};
-      if (!mbar_wait(q_rot, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      if (!mbar_wait(q_rot, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
       // K of the first tile
-      if (!mbar_wait(k_rot + 0, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      if (!mbar_wait(k_rot + 0, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
       tc_fence_after();
       for (int s = 0; s < 2; ++s)
         if (active(s, jt0)) {
@@ -344,11 +352,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int uV = 2 * (j - jt0) + 1, stV = uV % C::NS;
         const int uK = uV + 1, stK = uK % C::NS;
         const bool next = j < jt1;
-        if (!mbar_wait(k_rot + stV, (uV / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        if (!mbar_wait(k_rot + stV, (uV / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
         TRACE(0, tcnt, 8);
         for (int s = 0; s < 2; ++s) {
           if (active(s, j)) {
-            if (!mbar_wait(p_full + s, cnt[s] & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+            if (!mbar_wait(p_full + s, cnt[s] & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
             TRACE(0, tcnt, 1 + 4 * s);
             tc_fence_after();
             issue_pv(s, stV, cnt[s] > 0);
@@ -357,7 +365,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             TRACE(0, tcnt, 2 + 4 * s);
           }
           if (next && s == 0) {
-            if (!mbar_wait(k_rot + stK, (uK / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+            if (!mbar_wait(k_rot + stK, (uK / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
             TRACE(0, tcnt, 3);
             tc_fence_after();
           }
@@ -370,6 +378,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         umma_commit(kv_empty + stV);
         if (next) umma_commit(kv_empty + stK);
       }
+    mma_drain:
+      // every MMA issued above completes before tensor memory is released
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0, DRAIN_LIMIT_NS);
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 0-7)

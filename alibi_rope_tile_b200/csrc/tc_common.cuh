@@ -80,6 +80,15 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
   }
 }
 
+// Wait for a phase regardless of the abort flag, at most ``limit_ns``: used after an abort
+// to let the copies and MMAs a role has issued finish before the CTA releases its memory.
+static __device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity, 1000000u))
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  return true;
+}
+
 // Bounded wait for the phase of ``bar`` with the given parity.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* status, uint64_t limit_ns) {
