@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           const float mu = (m_exp == -INFINITY) ? 0.f : m_exp;
           const f2x SC = pk2(sc, sc), NM = pk2(-mu, -mu);
-          float rs0 = 0.f, rs1 = 0.f;
+          f2x RS = pk2(0.f, 0.f);  // row-sum partials, two lanes of packed adds
           uint32_t pk[32];  // column k: keys 2k, 2k+1 of this half (low half = even key)
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
@@ -489,12 +489,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               e2 = ex2(xb[2 * k] - mu);
               e3 = ex2(xb[2 * k + 1] - mu);
             }
-            rs0 += e0 + e1;
-            rs1 += e2 + e3;
+            RS = add2(RS, add2(pk2(e0, e1), pk2(e2, e3)));
             pk[k] = f2_to_bf2(e0, e1);
             pk[16 + k] = f2_to_bf2(e2, e3);
           }
-          rs += rs0 + rs1;
+          {
+            float r0, r1;
+            up2(RS, r0, r1);
+            rs += r0 + r1;
+          }
           // P of keys h2*64 .. h2*64+63 -> columns h2*32 .. h2*32+31 (already read above)
           tmem_st32u(tS + h2 * 32, pk);
           if (tracer) TRACE(1 + s, tcnt, 16 + 2 * h2);
