@@ -15,16 +15,18 @@
 // rotated once per 256 query rows. CTAs are numbered longest-first (causal rows near the
 // end see the most keys) so the block scheduler packs them like an LPT schedule.
 //
-// Warp roles (14 warps):
-//   warps 0-3  softmax of slot 0 (thread = query row = TMEM lane)
-//   warps 4-7  softmax of slot 1
-//   warps 8-11 rotary embedding: turns the two Q tiles once, then every K tile in place
-//              in its 128-byte-swizzled shared-memory layout (RoPE on load)
-//   warp 12    TMA producer (Q tiles, then K/V tiles through a ring of NS stages)
-//   warp 13    TMEM allocation and UMMA issue
+// Warp roles (22 warps):
+//   warps 0-7   softmax of slot 0 (thread = query row = TMEM lane; warps 0-3 own keys
+//               0..63 of every tile, warps 4-7 keys 64..127)
+//   warps 8-15  softmax of slot 1 (same split)
+//   warps 16-19 rotary embedding: turns the two Q tiles once, then every K tile in place
+//               in its 128-byte-swizzled shared-memory layout (RoPE on load)
+//   warp 20     TMA producer (Q tiles, then K/V tiles through a ring of NS stages)
+//   warp 21     TMEM allocation and UMMA issue
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each) | O0 | O1 (hd each).
-// The softmax writes P (bf16, two per 32-bit column) over the first 64 columns of its own
-// S buffer, after reading them, and PV takes P straight from tensor memory (the A operand
+// Each softmax half writes its P (bf16, two per 32-bit column) over the first 32 columns
+// of its own 64 S columns, after reading them (keys 0..63 -> columns 0..31, keys 64..127 ->
+// columns 64..95), and PV takes P straight from tensor memory (the A operand
 // of the TS-form MMA): P never touches shared memory, whose bandwidth (128 B/clk/SM) the
 // SS-form QK MMAs, the TMA writes and the in-place key rotation already share. The next
 // QK of a slot overwrites that slot's S/P columns; it is issued after the slot's PV, and
@@ -49,11 +51,11 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int NUM_WARPS = 14;
+constexpr int NUM_WARPS = 22;
 constexpr int NUM_THREADS = NUM_WARPS * 32;
-constexpr int WARP_ROPE0 = 8;
-constexpr int WARP_TMA = 12;
-constexpr int WARP_MMA = 13;
+constexpr int WARP_ROPE0 = 16;
+constexpr int WARP_TMA = 20;
+constexpr int WARP_MMA = 21;
 constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;  // a wait that lasts 4 s has failed
 constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;  // own copies/MMAs finish in microseconds
 constexpr float LOG2E = 1.4426950408889634f;
@@ -76,15 +78,18 @@ __device__ long long g_attn_trace[16][2048];
 
 template <int HD>
 struct Cfg {
-  static constexpr int NS = HD == 128 ? 5 : 10;  // key/value ring stages
+  static constexpr int NS = HD == 128 ? 4 : 10;  // key/value ring stages
   static constexpr int Q_BYTES = BM * HD * 2;
   static constexpr int KV_BYTES = BN * HD * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
-  static constexpr int NBAR = 3 * NS + 9;
+  static constexpr int NBAR = 3 * NS + 15;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KiB
+  // row-max exchange [slot][tile parity][half][128] and row-sum exchange [slot][half][128]
+  static constexpr int OFF_RED = (OFF_MISC + 16 + 15) / 16 * 16;
+  static constexpr int RED_FLOATS = 2 * 2 * 2 * 128 + 2 * 2 * 128;
+  static constexpr int SMEM = OFF_RED + RED_FLOATS * 4 + 1024;  // + slack to align the base
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, 0, 1);
 };
@@ -189,6 +194,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* p_full = q_full + 4;
   uint64_t* o_done = q_full + 6;
   uint64_t* drain = q_full + 8;  // the MMA thread's final commit
+  uint64_t* red_bar = q_full + 9;   // [slot][tile parity]: both halves' row maxima written
+  uint64_t* lsum_bar = q_full + 13;  // [slot]: both halves' row sums written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -238,7 +245,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(q_rot, 128);
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(p_full + s, 128);
+      mbar_init(p_full + s, 256);
+      mbar_init(red_bar + 2 * s, 256);
+      mbar_init(red_bar + 2 * s + 1, 256);
+      mbar_init(lsum_bar + s, 256);
       mbar_init(o_done + s, 1);
     }
     mbar_init(drain, 1);
@@ -332,7 +342,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint64_t b0 = dV + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          umma_ts(d, aP + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
+          umma_ts(d, aP + kk * 8 + (kk >= 4 ? 32 : 0), b0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
                   (kk > 0 || acc) ? 1u : 0u);
           if (kk == 0 || kk == 3) TRACE(0, tcnt, 40 + kk);
         }
@@ -384,33 +394,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait_drain(drain, 0, DRAIN_LIMIT_NS);
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 0-7)
-    // The per-tile loops over 64-column halves are deliberately not unrolled: with ten
-    // warps running four different roles, the instruction cache, not the exponential
-    // unit, bounded the unrolled version.
-    const int s = warp >> 2;
-    const int r = tid & 127;
+    // ------------------------------------------------------------ softmax (warps 0-15)
+    // Two warpgroups per slot: warpgroup hc owns keys hc*64 .. hc*64+63 of every tile of
+    // the slot's 128 rows (thread = row = TMEM lane). Per tile each thread takes its half's
+    // maximum (first pass over TMEM), the halves exchange maxima through shared memory
+    // (an mbarrier per slot and tile parity), both derive the same row reference, then each
+    // forms the weights of its 64 keys in two 32-column chunks and writes their P (bf16)
+    // over the first 32 columns of its own S half; O is rescaled (rarely) half by half.
+    // The loops over chunks are deliberately not unrolled: the instruction cache, not the
+    // exponential unit, bounded the unrolled versions.
+    const int s = warp >> 3;
+    const int hc = (warp >> 2) & 1;
+    const int r = (warp & 3) * 32 + lane;
     const int i = qs[s] + r;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_off + s * BN;
-    const uint32_t tO = tmem + lane_off + 2 * BN + s * HD;
+    const uint32_t tSh = tmem + lane_off + s * BN + hc * 64;          // my S half; my P over its first 32
+    const uint32_t tOh = tmem + lane_off + 2 * BN + s * HD + hc * (HD / 2);  // my half of O
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+    float* lsum = red + 2 * 2 * 2 * 128;
     const float slope = p.alibi.on ? p.alibi.slope[head[s]] * LOG2E : 0.f;
     const float sc = a.scale_log2;
     // Row state in the log2 domain: m_ref is the reference the weights of this row are
-    // taken against (-inf until the row has seen an allowed key), l their running sum.
-    // The reference moves only when a tile's maximum exceeds it by more than 8 (a factor
-    // 256), so the accumulator is rescaled rarely; weights stay below 2^8.
+    // taken against (-inf until the row has seen an allowed key), l the running sum of this
+    // half's weights. The reference moves only when a tile's maximum exceeds it by more
+    // than 8 (a factor 256), so O is rescaled rarely; weights stay below 2^8.
     float m_ref = -INFINITY, l = 0.f;
     int c = 0, tcnt = 0;
-    const bool tracer = (tid & 127) == 0;
+    const bool tracer = (warp == 8 * s) && lane == 0;
     if (valid[s]) {
       for (int j = t0[s]; j <= t1[s]; ++j, ++c) {
         if (!mbar_wait(s_full + s, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
         if (tracer) TRACE(1 + s, tcnt, 10);
         tc_fence_after();
-        const int key0 = j * BN;
-        // does any row of this slot need per-element masking in this tile?
-        const bool need_mask = (key0 + BN > p.T) || (p.causal && key0 + BN - 1 > qs[s]) ||
+        const int key0 = j * BN + hc * 64;  // first key of my half
+        // does any row of this slot need per-element masking in my half of this tile?
+        const bool need_mask = (key0 + 64 > p.T) || (p.causal && key0 + 63 > qs[s]) ||
                                (p.window > 0 && qs[s] + BM - 1 - key0 >= p.window);
         const bool plain = !need_mask && !p.alibi.on;
         auto score = [&](float x, int jk) {
@@ -421,101 +439,84 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           return v;
         };
-        // Weights are taken against a per-row reference m_exp that starts at the row's
-        // reference m_ref. Each 64-key half is loaded once: its maximum is taken first, and
-        // if it exceeds the reference by more than 8 for some row of the warp, that row's
-        // reference moves up before the weights of the half are formed. When the second
-        // half moves it, the P already written for the first half (and its partial sum)
-        // is rescaled in place; once a row has seen a tile this is rare.
-        float m_exp = m_ref, rs = 0.f;
-        if (tracer) TRACE(1 + s, tcnt, 11);
+        // pass 1: my half's maximum
+        float hx = -INFINITY;
 #pragma unroll 1
-        for (int h2 = 0; h2 < BN / 64; ++h2) {
-          float xa[32], xb[32];
-          tmem_ld32(tS + h2 * 64, xa);
-          tmem_ld32(tS + h2 * 64 + 32, xb);
+        for (int q2 = 0; q2 < 2; ++q2) {
+          float x[32];
+          tmem_ld32(tSh + q2 * 32, x);
           tmem_wait_ld();
-          if (tracer) TRACE(1 + s, tcnt, 15 + 2 * h2);
-          float hx = -INFINITY;
           if (plain) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) hx = max3(hx, max3(xa[2 * k], xa[2 * k + 1], xb[2 * k]), xb[2 * k + 1]);
-            hx *= sc;  // a positive scale keeps the order: max then scale is exact
+            for (int k = 0; k < 16; ++k) hx = max3(hx, x[2 * k], x[2 * k + 1]);
           } else {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              xa[k] = score(xa[k], key0 + h2 * 64 + k);
-              xb[k] = score(xb[k], key0 + h2 * 64 + 32 + k);
-              hx = max3(hx, xa[k], xb[k]);
-            }
+            for (int k = 0; k < 16; ++k)
+              hx = max3(hx, score(x[2 * k], key0 + q2 * 32 + 2 * k), score(x[2 * k + 1], key0 + q2 * 32 + 2 * k + 1));
           }
-          const float m_cand = (hx > m_exp + 8.f) ? hx : m_exp;  // takes hx when m_exp = -inf
-          if (__any_sync(0xffffffffu, m_cand != m_exp)) {
-            if (h2 > 0) {
-              const float f = (m_cand == m_exp) ? 1.f : ex2(m_exp - m_cand);  // 1 where it stays
-              float pp[32];
-              tmem_wait_st();
-              tmem_ld32(tS, pp);
-              tmem_wait_ld();
-              uint32_t pq[32];
+        }
+        if (plain) hx *= sc;  // a positive scale keeps the order: max then scale is exact
+        float* rb = red + ((s * 2 + (c & 1)) * 2) * 128;
+        rb[hc * 128 + r] = hx;
+        mbar_arrive(red_bar + 2 * s + (c & 1));
+        if (!mbar_wait(red_bar + 2 * s + (c & 1), (c >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        const float mt = fmaxf(hx, rb[(1 - hc) * 128 + r]);
+        const float m_new = (mt > m_ref + 8.f) ? mt : m_ref;  // takes mt when m_ref = -inf
+        const float alpha = (m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
+        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+        m_ref = m_new;
+        if (tracer) TRACE(1 + s, tcnt, 11);
+        // pass 2: weights of my 64 keys; chunk q2 reads S columns q2*32.. of my half and
+        // writes its P to columns q2*16.. of my half (already read by chunk 0)
+        f2x RS = pk2(0.f, 0.f);
+        const f2x SC = pk2(sc, sc), NM = pk2(-mu, -mu);
+#pragma unroll 1
+        for (int q2 = 0; q2 < 2; ++q2) {
+          float x[32];
+          tmem_ld32(tSh + q2 * 32, x);
+          tmem_wait_ld();
+          uint32_t pk[16];  // column k: keys 2k, 2k+1 of this chunk (low half = even key)
 #pragma unroll
-              for (int k = 0; k < 32; ++k) {
-                const float2 v = bf2_to_f2(__float_as_uint(pp[k]));
-                pq[k] = f2_to_bf2(v.x * f, v.y * f);
-              }
-              tmem_st32u(tS, pq);
-              rs *= f;
-            }
-            m_exp = m_cand;
-          }
-          const float mu = (m_exp == -INFINITY) ? 0.f : m_exp;
-          const f2x SC = pk2(sc, sc), NM = pk2(-mu, -mu);
-          f2x RS = pk2(0.f, 0.f);  // row-sum partials, two lanes of packed adds
-          uint32_t pk[32];  // column k: keys 2k, 2k+1 of this half (low half = even key)
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
+          for (int k = 0; k < 8; ++k) {
             float e0, e1, e2, e3;
             if (plain) {
               float a0, a1, b0, b1;
-              up2(fma2(pk2(xa[2 * k], xa[2 * k + 1]), SC, NM), a0, a1);
-              up2(fma2(pk2(xb[2 * k], xb[2 * k + 1]), SC, NM), b0, b1);
+              up2(fma2(pk2(x[4 * k], x[4 * k + 1]), SC, NM), a0, a1);
+              up2(fma2(pk2(x[4 * k + 2], x[4 * k + 3]), SC, NM), b0, b1);
               e0 = ex2(a0);
               e1 = ex2(a1);
               e2 = ex2(b0);
               e3 = ex2(b1);
             } else {
-              e0 = ex2(xa[2 * k] - mu);
-              e1 = ex2(xa[2 * k + 1] - mu);
-              e2 = ex2(xb[2 * k] - mu);
-              e3 = ex2(xb[2 * k + 1] - mu);
+              const int jk = key0 + q2 * 32 + 4 * k;
+              e0 = ex2(score(x[4 * k], jk) - mu);
+              e1 = ex2(score(x[4 * k + 1], jk + 1) - mu);
+              e2 = ex2(score(x[4 * k + 2], jk + 2) - mu);
+              e3 = ex2(score(x[4 * k + 3], jk + 3) - mu);
             }
             RS = add2(RS, add2(pk2(e0, e1), pk2(e2, e3)));
-            pk[k] = f2_to_bf2(e0, e1);
-            pk[16 + k] = f2_to_bf2(e2, e3);
+            pk[2 * k] = f2_to_bf2(e0, e1);
+            pk[2 * k + 1] = f2_to_bf2(e2, e3);
           }
-          {
-            float r0, r1;
-            up2(RS, r0, r1);
-            rs += r0 + r1;
-          }
-          // P of keys h2*64 .. h2*64+63 -> columns h2*32 .. h2*32+31 (already read above)
-          tmem_st32u(tS + h2 * 32, pk);
-          if (tracer) TRACE(1 + s, tcnt, 16 + 2 * h2);
+          tmem_st16u(tSh + q2 * 16, pk);
         }
-        const float m_new = m_exp;
-        const float alpha = (m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
-        m_ref = m_new;
+        float rs;
+        {
+          float r0, r1;
+          up2(RS, r0, r1);
+          rs = r0 + r1;
+        }
         // O is rescaled before this tile's PV is issued. The previous PV of this slot has
         // completed: it was issued before the QK whose completion this tile waited for.
         if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-          for (int q4 = 0; q4 < HD / 32; ++q4) {
+          for (int q4 = 0; q4 < HD / 64; ++q4) {
             float o[32];
-            tmem_ld32(tO + q4 * 32, o);
+            tmem_ld32(tOh + q4 * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tO + q4 * 32, o);
+            tmem_st32(tOh + q4 * 32, o);
           }
         }
         if (tracer) TRACE(1 + s, tcnt, 12);
@@ -526,15 +527,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (tracer) TRACE(1 + s, tcnt, 14);
       }
       if (c > 0) {
+        // the row's total sum: both halves' partial sums, exchanged through shared memory
+        lsum[(s * 2 + hc) * 128 + r] = l;
+        mbar_arrive(lsum_bar + s);
+        if (!mbar_wait(lsum_bar + s, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        const float lt = l + lsum[(s * 2 + 1 - hc) * 128 + r];
         if (!mbar_wait(o_done + s, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
         tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
-                              (((size_t)b * p.T + i) * p.H + head[s]) * HD;
+                              (((size_t)b * p.T + i) * p.H + head[s]) * HD + hc * (HD / 2);
 #pragma unroll 1
-        for (int q4 = 0; q4 < HD / 32; ++q4) {
+        for (int q4 = 0; q4 < HD / 64; ++q4) {
           float o[32];
-          tmem_ld32(tO + q4 * 32, o);
+          tmem_ld32(tOh + q4 * 32, o);
           tmem_wait_ld();
           if (i < p.T) {
             uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
@@ -546,8 +552,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                    f2_to_bf2(o[8 * v4 + 6] * inv, o[8 * v4 + 7] * inv));
           }
         }
-        if (p.lse && i < p.T)
-          p.lse[((size_t)b * p.H + head[s]) * p.T + i] = l > 0.f ? (m_ref + __log2f(l)) * LN2 : -INFINITY;
+        if (p.lse && i < p.T && hc == 0)
+          p.lse[((size_t)b * p.H + head[s]) * p.T + i] = lt > 0.f ? (m_ref + __log2f(lt)) * LN2 : -INFINITY;
       }
     }
   }
