@@ -16,23 +16,23 @@
 // end see the most keys) so the block scheduler packs them like an LPT schedule.
 //
 // Warp roles (22 warps):
-//   warps 0-7   softmax of slot 0 (thread = query row = TMEM lane; warps 0-3 own keys
-//               0..63 of every tile, warps 4-7 keys 64..127)
-//   warps 8-15  softmax of slot 1 (same split)
+//   warps 0-15  softmax, one slot at a time (slot 0, then slot 1, for every key tile):
+//               warp w owns 32 query rows (TMEM lanes 32*(w%4)..) and 32 keys of the tile
+//               (keys 32*(w/4)..)
 //   warps 16-19 rotary embedding: turns the two Q tiles once, then every K tile in place
 //               in its 128-byte-swizzled shared-memory layout (RoPE on load)
 //   warp 20     TMA producer (Q tiles, then K/V tiles through a ring of NS stages)
 //   warp 21     TMEM allocation and UMMA issue
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each) | O0 | O1 (hd each).
-// Each softmax half writes its P (bf16, two per 32-bit column) over the first 32 columns
-// of its own 64 S columns, after reading them (keys 0..63 -> columns 0..31, keys 64..127 ->
-// columns 64..95), and PV takes P straight from tensor memory (the A operand
-// of the TS-form MMA): P never touches shared memory, whose bandwidth (128 B/clk/SM) the
-// SS-form QK MMAs, the TMA writes and the in-place key rotation already share. The next
+// P (bf16, two per 32-bit column) goes over the first 64 columns of the slot's S region
+// once every softmax warp has read its S columns (keys 2c, 2c+1 -> column c), and PV takes
+// P straight from tensor memory (the A operand of the TS-form MMA): P never touches shared
+// memory, which the SS-form QK MMAs, the TMA writes and the in-place key rotation already
+// share (an M=128, N=128 SS MMA reads 8 KB of operands from shared memory). The next
 // QK of a slot overwrites that slot's S/P columns; it is issued after the slot's PV, and
 // the tensor core executes one CTA's MMAs in issue order, so P is read before it is
 // overwritten. Issue order per key tile j: PV0(j), QK0(j+1), PV1(j), QK1(j+1): the tensor
-// core works on one slot while the other slot's softmax runs.
+// core works on one slot while the softmax warps work on the other.
 //
 // Masking: a pair outside the causal/window/length limits gets -inf before the row max,
 // so its weight is exactly 0, and the sums' order depends only on the tile structure;
@@ -86,9 +86,9 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
   static constexpr int NBAR = 3 * NS + 15;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // row-max exchange [slot][tile parity][half][128] and row-sum exchange [slot][half][128]
+  // row-max exchange [parity][key quarter][128] and row-sum exchange [slot][key quarter][128]
   static constexpr int OFF_RED = (OFF_MISC + 16 + 15) / 16 * 16;
-  static constexpr int RED_FLOATS = 2 * 2 * 2 * 128 + 2 * 2 * 128;
+  static constexpr int RED_FLOATS = 2 * 4 * 128 + 2 * 4 * 128;
   static constexpr int SMEM = OFF_RED + RED_FLOATS * 4 + 1024;  // + slack to align the base
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, 0, 1);
@@ -194,8 +194,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* p_full = q_full + 4;
   uint64_t* o_done = q_full + 6;
   uint64_t* drain = q_full + 8;  // the MMA thread's final commit
-  uint64_t* red_bar = q_full + 9;   // [slot][tile parity]: both halves' row maxima written
-  uint64_t* lsum_bar = q_full + 13;  // [slot]: both halves' row sums written
+  uint64_t* red_bar = q_full + 9;    // [parity of the slot-tile count]: all warps' row maxima written
+  uint64_t* lsum_bar = q_full + 13;  // [slot]: all warps' row sums written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -245,10 +245,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(q_rot, 128);
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(p_full + s, 256);
-      mbar_init(red_bar + 2 * s, 256);
-      mbar_init(red_bar + 2 * s + 1, 256);
-      mbar_init(lsum_bar + s, 256);
+      mbar_init(p_full + s, 16);  // one arrival per softmax warp
+      mbar_init(red_bar + s, 16);
+      mbar_init(lsum_bar + s, 16);
       mbar_init(o_done + s, 1);
     }
     mbar_init(drain, 1);
@@ -338,11 +337,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       auto issue_pv = [&](int s, int st, bool acc) {
         const uint32_t d = tmem + 2 * BN + s * HD;
-        const uint32_t aP = tmem + s * BN;  // P: 64 columns of bf16 pairs over S
+        const uint32_t aP = tmem + s * BN;  // P: 64 columns of bf16 pairs over the first half of S
         const uint64_t b0 = dV + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          umma_ts(d, aP + kk * 8 + (kk >= 4 ? 32 : 0), b0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
+          umma_ts(d, aP + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
                   (kk > 0 || acc) ? 1u : 0u);
           if (kk == 0 || kk == 3) TRACE(0, tcnt, 40 + kk);
         }
@@ -395,111 +394,110 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 0-15)
-    // Two warpgroups per slot: warpgroup hc owns keys hc*64 .. hc*64+63 of every tile of
-    // the slot's 128 rows (thread = row = TMEM lane). Per tile each thread takes its half's
-    // maximum (first pass over TMEM), the halves exchange maxima through shared memory
-    // (an mbarrier per slot and tile parity), both derive the same row reference, then each
-    // forms the weights of its 64 keys in two 32-column chunks and writes their P (bf16)
-    // over the first 32 columns of its own S half; O is rescaled (rarely) half by half.
-    // The loops over chunks are deliberately not unrolled: the instruction cache, not the
-    // exponential unit, bounded the unrolled versions.
-    const int s = warp >> 3;
-    const int hc = (warp >> 2) & 1;
+    // All sixteen warps work on one slot at a time, slot 0 then slot 1 for every key tile, so
+    // the tensor core runs one slot's PV and next QK while the other slot's weights are
+    // formed. Warp w owns TMEM lanes 32*(w%4).. (32 query rows) and keys kq*32 .. kq*32+31 of
+    // the tile, kq = w/4: one 32-column TMEM load per thread per slot and tile. The four
+    // warps of a row exchange their maxima through shared memory (an mbarrier per parity of
+    // the slot-tile count), all derive the same row reference, and each writes the P (bf16)
+    // of its 32 keys to TMEM columns kq*16 .. kq*16+15 of the slot's S region; every S column
+    // was read before the exchange, so P may overwrite any of them. O is rescaled (rarely)
+    // by column quarter.
+    const int kq = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
-    const int i = qs[s] + r;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tSh = tmem + lane_off + s * BN + hc * 64;          // my S half; my P over its first 32
-    const uint32_t tOh = tmem + lane_off + 2 * BN + s * HD + hc * (HD / 2);  // my half of O
-    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
-    float* lsum = red + 2 * 2 * 2 * 128;
-    const float slope = p.alibi.on ? p.alibi.slope[head[s]] * LOG2E : 0.f;
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [parity][kq][128] row maxima
+    float* lsum = red + 2 * 4 * 128;                            // [slot][kq][128] row sums
     const float sc = a.scale_log2;
-    // Row state in the log2 domain: m_ref is the reference the weights of this row are
-    // taken against (-inf until the row has seen an allowed key), l the running sum of this
-    // half's weights. The reference moves only when a tile's maximum exceeds it by more
-    // than 8 (a factor 256), so O is rescaled rarely; weights stay below 2^8.
-    float m_ref = -INFINITY, l = 0.f;
-    int c = 0, tcnt = 0;
-    const bool tracer = (warp == 8 * s) && lane == 0;
-    if (valid[s]) {
-      for (int j = t0[s]; j <= t1[s]; ++j, ++c) {
+    // Row state per slot in the log2 domain: m_ref is the reference the weights are taken
+    // against (-inf until the row has seen an allowed key), l the running sum of this warp's
+    // share of the weights. The reference moves only when a tile's maximum exceeds it by
+    // more than 8 (a factor 256), so O is rescaled rarely; weights stay below 2^8.
+    float m_ref0 = -INFINITY, m_ref1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    int cs0 = 0, cs1 = 0, t = 0, tcnt = 0;
+    const bool tracer = warp == 0 && lane == 0;
+#pragma unroll 1
+    for (int j = jt0; j <= jt1; ++j) {
+#pragma unroll 1
+      for (int s = 0; s < 2; ++s) {
+        if (!active(s, j)) continue;
+        // this slot's row state (scalars selected by slot: no indexed local arrays)
+        const int c = s ? cs1 : cs0;
+        float m_ref = s ? m_ref1 : m_ref0;
         if (!mbar_wait(s_full + s, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
         if (tracer) TRACE(1 + s, tcnt, 10);
         tc_fence_after();
-        const int key0 = j * BN + hc * 64;  // first key of my half
-        // does any row of this slot need per-element masking in my half of this tile?
-        const bool need_mask = (key0 + 64 > p.T) || (p.causal && key0 + 63 > qs[s]) ||
-                               (p.window > 0 && qs[s] + BM - 1 - key0 >= p.window);
+        const int q0s = qs[s];  // first query row of the slot
+        const int hs = head[s];
+        const int i = q0s + r;
+        const uint32_t tS = tmem + lane_off + s * BN;
+        const int key0 = j * BN + kq * 32;  // first of my 32 keys
+        const float slope = p.alibi.on ? p.alibi.slope[hs] * LOG2E : 0.f;
+        // does any row of this slot need per-element masking in my keys of this tile?
+        const bool need_mask = (key0 + 32 > p.T) || (p.causal && key0 + 31 > q0s) ||
+                               (p.window > 0 && q0s + BM - 1 - key0 >= p.window);
         const bool plain = !need_mask && !p.alibi.on;
-        auto score = [&](float x, int jk) {
-          float v = p.alibi.on ? fmaf(x, sc, -slope * fabsf((float)(i - jk))) : x * sc;
-          if (need_mask) {
-            const bool ok = jk < p.T && (!p.causal || jk <= i) && (p.window <= 0 || i - jk < p.window);
-            v = ok ? v : -INFINITY;
-          }
-          return v;
-        };
-        // pass 1: my half's maximum
+        float x[32];
+        tmem_ld32(tS + kq * 32, x);
+        tmem_wait_ld();
         float hx = -INFINITY;
-#pragma unroll 1
-        for (int q2 = 0; q2 < 2; ++q2) {
-          float x[32];
-          tmem_ld32(tSh + q2 * 32, x);
-          tmem_wait_ld();
-          if (plain) {
+        if (plain) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) hx = max3(hx, x[2 * k], x[2 * k + 1]);
-          } else {
+          for (int k = 0; k < 16; ++k) hx = max3(hx, x[2 * k], x[2 * k + 1]);
+          hx *= sc;  // a positive scale keeps the order: max then scale is exact
+        } else {
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-              hx = max3(hx, score(x[2 * k], key0 + q2 * 32 + 2 * k), score(x[2 * k + 1], key0 + q2 * 32 + 2 * k + 1));
+          for (int k = 0; k < 32; ++k) {
+            const int jk = key0 + k;
+            float v = p.alibi.on ? fmaf(x[k], sc, -slope * fabsf((float)(i - jk))) : x[k] * sc;
+            if (need_mask) {
+              const bool ok = jk < p.T && (!p.causal || jk <= i) && (p.window <= 0 || i - jk < p.window);
+              v = ok ? v : -INFINITY;
+            }
+            x[k] = v;
           }
+#pragma unroll
+          for (int k = 0; k < 16; ++k) hx = max3(hx, x[2 * k], x[2 * k + 1]);
         }
-        if (plain) hx *= sc;  // a positive scale keeps the order: max then scale is exact
-        float* rb = red + ((s * 2 + (c & 1)) * 2) * 128;
-        rb[hc * 128 + r] = hx;
-        mbar_arrive(red_bar + 2 * s + (c & 1));
-        if (!mbar_wait(red_bar + 2 * s + (c & 1), (c >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        const float mt = fmaxf(hx, rb[(1 - hc) * 128 + r]);
+        float* rb = red + (t & 1) * 512;
+        rb[kq * 128 + r] = hx;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(red_bar + (t & 1));
+        if (!mbar_wait(red_bar + (t & 1), (t >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        const float mt = fmaxf(fmaxf(rb[r], rb[128 + r]), fmaxf(rb[256 + r], rb[384 + r]));
         const float m_new = (mt > m_ref + 8.f) ? mt : m_ref;  // takes mt when m_ref = -inf
         const float alpha = (m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
         m_ref = m_new;
         if (tracer) TRACE(1 + s, tcnt, 11);
-        // pass 2: weights of my 64 keys; chunk q2 reads S columns q2*32.. of my half and
-        // writes its P to columns q2*16.. of my half (already read by chunk 0)
         f2x RS = pk2(0.f, 0.f);
-        const f2x SC = pk2(sc, sc), NM = pk2(-mu, -mu);
-#pragma unroll 1
-        for (int q2 = 0; q2 < 2; ++q2) {
-          float x[32];
-          tmem_ld32(tSh + q2 * 32, x);
-          tmem_wait_ld();
-          uint32_t pk[16];  // column k: keys 2k, 2k+1 of this chunk (low half = even key)
+        uint32_t pk[16];  // column k: keys 2k, 2k+1 of my 32 (low half = even key)
+        if (plain) {
+          const f2x SC = pk2(sc, sc), NM = pk2(-mu, -mu);
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            float e0, e1, e2, e3;
-            if (plain) {
-              float a0, a1, b0, b1;
-              up2(fma2(pk2(x[4 * k], x[4 * k + 1]), SC, NM), a0, a1);
-              up2(fma2(pk2(x[4 * k + 2], x[4 * k + 3]), SC, NM), b0, b1);
-              e0 = ex2(a0);
-              e1 = ex2(a1);
-              e2 = ex2(b0);
-              e3 = ex2(b1);
-            } else {
-              const int jk = key0 + q2 * 32 + 4 * k;
-              e0 = ex2(score(x[4 * k], jk) - mu);
-              e1 = ex2(score(x[4 * k + 1], jk + 1) - mu);
-              e2 = ex2(score(x[4 * k + 2], jk + 2) - mu);
-              e3 = ex2(score(x[4 * k + 3], jk + 3) - mu);
-            }
+            float a0, a1, b0, b1;
+            up2(fma2(pk2(x[4 * k], x[4 * k + 1]), SC, NM), a0, a1);
+            up2(fma2(pk2(x[4 * k + 2], x[4 * k + 3]), SC, NM), b0, b1);
+            const float e0 = ex2(a0), e1 = ex2(a1), e2 = ex2(b0), e3 = ex2(b1);
             RS = add2(RS, add2(pk2(e0, e1), pk2(e2, e3)));
             pk[2 * k] = f2_to_bf2(e0, e1);
             pk[2 * k + 1] = f2_to_bf2(e2, e3);
           }
-          tmem_st16u(tSh + q2 * 16, pk);
+        } else {
+          const f2x NM = pk2(-mu, -mu);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            float a0, a1, b0, b1;
+            up2(add2(pk2(x[4 * k], x[4 * k + 1]), NM), a0, a1);
+            up2(add2(pk2(x[4 * k + 2], x[4 * k + 3]), NM), b0, b1);
+            const float e0 = ex2(a0), e1 = ex2(a1), e2 = ex2(b0), e3 = ex2(b1);
+            RS = add2(RS, add2(pk2(e0, e1), pk2(e2, e3)));
+            pk[2 * k] = f2_to_bf2(e0, e1);
+            pk[2 * k + 1] = f2_to_bf2(e2, e3);
+          }
         }
+        tmem_st16u(tS + kq * 16, pk);
         float rs;
         {
           float r0, r1;
@@ -508,53 +506,66 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         // O is rescaled before this tile's PV is issued. The previous PV of this slot has
         // completed: it was issued before the QK whose completion this tile waited for.
-        if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-          for (int q4 = 0; q4 < HD / 64; ++q4) {
-            float o[32];
-            tmem_ld32(tOh + q4 * 32, o);
-            tmem_wait_ld();
+        if (c > 0 && kq * 32 < HD && __any_sync(0xffffffffu, alpha != 1.f)) {
+          const uint32_t tO = tmem + lane_off + 2 * BN + s * HD + kq * 32;
+          float o[32];
+          tmem_ld32(tO, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tOh + q4 * 32, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tmem_st32(tO, o);
         }
-        if (tracer) TRACE(1 + s, tcnt, 12);
-        l = l * alpha + rs;
+        if (s) {
+          l1 = l1 * alpha + rs;
+          m_ref1 = m_ref;
+          cs1 = c + 1;
+        } else {
+          l0 = l0 * alpha + rs;
+          m_ref0 = m_ref;
+          cs0 = c + 1;
+        }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full + s);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + s);
         if (tracer) TRACE(1 + s, tcnt, 14);
+        ++t;
       }
-      if (c > 0) {
-        // the row's total sum: both halves' partial sums, exchanged through shared memory
-        lsum[(s * 2 + hc) * 128 + r] = l;
-        mbar_arrive(lsum_bar + s);
-        if (!mbar_wait(lsum_bar + s, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        const float lt = l + lsum[(s * 2 + 1 - hc) * 128 + r];
-        if (!mbar_wait(o_done + s, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        tc_fence_after();
-        const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
-                              (((size_t)b * p.T + i) * p.H + head[s]) * HD + hc * (HD / 2);
+    }
 #pragma unroll 1
-        for (int q4 = 0; q4 < HD / 64; ++q4) {
-          float o[32];
-          tmem_ld32(tOh + q4 * 32, o);
-          tmem_wait_ld();
-          if (i < p.T) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
+    for (int s = 0; s < 2; ++s) {
+      const int c = s ? cs1 : cs0;
+      if (c == 0) continue;
+      const float m_ref = s ? m_ref1 : m_ref0;
+      // the row's total sum: the four warps' partial sums, exchanged through shared memory
+      lsum[(s * 4 + kq) * 128 + r] = s ? l1 : l0;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(lsum_bar + s);
+      if (!mbar_wait(lsum_bar + s, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      const float* ls = lsum + s * 4 * 128 + r;
+      const float lt = (ls[0] + ls[128]) + (ls[256] + ls[384]);
+      if (!mbar_wait(o_done + s, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      tc_fence_after();
+      const int hs = head[s];
+      const int i = qs[s] + r;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      if (kq * 32 < HD) {
+        float o[32];
+        tmem_ld32(tmem + lane_off + 2 * BN + s * HD + kq * 32, o);
+        tmem_wait_ld();
+        if (i < p.T) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                (((size_t)b * p.T + i) * p.H + hs) * HD + kq * 32);
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              dst[v4] = make_uint4(f2_to_bf2(o[8 * v4] * inv, o[8 * v4 + 1] * inv),
-                                   f2_to_bf2(o[8 * v4 + 2] * inv, o[8 * v4 + 3] * inv),
-                                   f2_to_bf2(o[8 * v4 + 4] * inv, o[8 * v4 + 5] * inv),
-                                   f2_to_bf2(o[8 * v4 + 6] * inv, o[8 * v4 + 7] * inv));
-          }
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[v4] = make_uint4(f2_to_bf2(o[8 * v4] * inv, o[8 * v4 + 1] * inv),
+                                 f2_to_bf2(o[8 * v4 + 2] * inv, o[8 * v4 + 3] * inv),
+                                 f2_to_bf2(o[8 * v4 + 4] * inv, o[8 * v4 + 5] * inv),
+                                 f2_to_bf2(o[8 * v4 + 6] * inv, o[8 * v4 + 7] * inv));
         }
-        if (p.lse && i < p.T && hc == 0)
-          p.lse[((size_t)b * p.H + head[s]) * p.T + i] = lt > 0.f ? (m_ref + __log2f(lt)) * LN2 : -INFINITY;
       }
+      if (p.lse && i < p.T && kq == 0)
+        p.lse[((size_t)b * p.H + hs) * p.T + i] = lt > 0.f ? (m_ref + __log2f(lt)) * LN2 : -INFINITY;
     }
   }
 done:

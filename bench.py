@@ -5,9 +5,12 @@ One step = one pass of the whole hot path over one batch of synthetic input:
     RoPE on load, QK^T, mask, online softmax, PV, epilogue;
   * one decode step of the KV-cache workload (batch 64, H=32, KV=8, hd=128, cache lengths
     uniform in [1024, 8192]) and of its MQA variant (KV=1): split-KV partials and the
-    log-sum-exp merge.
+    log-sum-exp merge;
+  * one pass of the bf16 block around the same attention shape (x [2,4096,4096], weights
+    resident): the x@Wq, x@Wk, x@Wv projections, the attention core, then ctx@Wo.
 ``value`` is the prefill TFLOP/s (causal FLOPs counted: 4*B*H*hd*allowed pairs); the decode
-GB/s (cache rows read + q + out, per launch pair) ride along under ``decode``. Kernels are timed with CUDA events on the stream they
+GB/s (cache rows read + q + out, per launch pair) ride along under ``decode``, the block's
+TFLOP/s (projection FLOPs 2*M*N*K plus the attention's) under ``block``. Kernels are timed with CUDA events on the stream they
 are launched on; L2 is flushed (a 256 MiB memset, outside the timed events) before every
 step. ``e2e`` times the same call with the step's inputs copied from pinned host memory and
 its output copied back, all inside the timed region.
@@ -41,10 +44,12 @@ METRIC = "causal GQA prefill TFLOP/s and decode HBM GB/s on 1 B200, % of rooflin
 PREFILL = workloads.GQA
 DECODE = workloads.DECODE_GQA
 DECODE_MQA = workloads.DECODE_MQA
+BLOCK = workloads.GQA_BLOCK
 # Algorithmic bytes and launches, stated once (see the design notes):
 #   decode bytes = cache rows read (K and V) + q + out; prefill FLOPs = PREFILL.flops.
 PREFILL_LAUNCHES = 1
 DECODE_LAUNCHES = 2       # split pass + merge, per decode workload
+BLOCK_LAUNCHES = 5        # three projection GEMMs, the prefill, the output GEMM
 
 
 def peaks():
@@ -230,6 +235,7 @@ def run_ours(args, rank, world):
     stream = torch.cuda.current_stream()
     w = PREFILL
     do_p, do_d = args.only in ("all", "prefill"), args.only in ("all", "decode")
+    do_b = args.only in ("all", "block")
 
     q, k, v = workloads.prefill_inputs(w)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
@@ -245,6 +251,16 @@ def run_ours(args, rank, world):
                 ws=torch.empty(art.attn_decode_workspace_size(dw.B, dw.H, dw.KV, dw.hd, dw.Lmax),
                                dtype=torch.uint8, device="cuda")))
             del hkc, hvc
+    blk = None
+    if do_b:
+        bw = BLOCK
+        hx, hW = workloads.block_inputs(bw)
+        blk = dict(w=bw, hx=hx, x=hx.cuda(), W={n: t.cuda() for n, t in hW.items()},
+                   out=torch.empty(hx.shape, dtype=hx.dtype, device="cuda"),
+                   ws=torch.empty(art.attn_block_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV, bw.hd,
+                                                                 torch.bfloat16),
+                                  dtype=torch.uint8, device="cuda"))
+        del hW
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
     def prefill():
@@ -255,15 +271,23 @@ def run_ours(args, rank, world):
         art.attn_decode(d["q"], d["kc"], d["vc"], d["sl"], d["qp"], d["out"], workspace=d["ws"],
                         rope_base=d["w"].rope_base)
 
+    def block():
+        if blk is not None:
+            bw, W = blk["w"], blk["W"]
+            art.attn_block(blk["x"], W["Wq"], W["Wk"], W["Wv"], W["Wo"], blk["out"],
+                           workspace=blk["ws"], H=bw.H, KV=bw.KV, rope_base=bw.rope_base,
+                           causal=bw.causal, window=bw.window)
+
     for _ in range(max(3, args.warmup)):
         flush.zero_()
         prefill()
         for d in decs:
             decode(d)
+        block()
     torch.cuda.synchronize()
     art.attn_sync_status()
 
-    nev = 2 + 2 * len(decs)
+    nev = 2 + 2 * len(decs) + 2
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
@@ -282,6 +306,10 @@ def run_ours(args, rank, world):
             ev[s_][2 + 2 * n].record(stream)
             decode(d)
             ev[s_][3 + 2 * n].record(stream)
+        flush.zero_()
+        ev[s_][nev - 2].record(stream)
+        block()
+        ev[s_][nev - 1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -291,6 +319,8 @@ def run_ours(args, rank, world):
     d_tot = [max(1e-9, max_over_ranks(sum(ev[s_][2 + 2 * n].elapsed_time(ev[s_][3 + 2 * n])
                                           for s_ in range(args.steps)), world))
              for n in range(len(decs))]
+    b_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 2].elapsed_time(ev[s_][nev - 1])
+                                         for s_ in range(args.steps)), world))
     region_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
 
     # end to end through the public API: the step's inputs go host (pinned) -> device, the
@@ -299,6 +329,9 @@ def run_ours(args, rank, world):
     hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     hdec = [(d["hq"].pin_memory(), torch.empty(d["hq"].shape, dtype=d["hq"].dtype).pin_memory())
             for d in decs]
+    if blk is not None:
+        hbx = blk["hx"].pin_memory()
+        hbo = torch.empty(blk["hx"].shape, dtype=blk["hx"].dtype).pin_memory()
 
     def e2e_step():
         if do_p:
@@ -311,6 +344,10 @@ def run_ours(args, rank, world):
             d["q"].copy_(hdq, non_blocking=True)
             decode(d)
             hdo.copy_(d["out"], non_blocking=True)
+        if blk is not None:
+            blk["x"].copy_(hbx, non_blocking=True)
+            block()
+            hbo.copy_(blk["out"], non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -328,7 +365,8 @@ def run_ours(args, rank, world):
         return
     if args.only != "all":
         print(json.dumps({"only": args.only, "prefill_ms": p_tot / args.steps,
-                          "decode_ms": [t / args.steps for t in d_tot]}), flush=True)
+                          "decode_ms": [t / args.steps for t in d_tot],
+                          "block_ms": b_tot / args.steps}), flush=True)
         return
     pk = peaks()
     flops_step = w.flops
@@ -345,9 +383,26 @@ def run_ours(args, rank, world):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": traffic.get(d["w"].name),
                          "peak_source": f"{pk.get('source')} copy"}}
+    bw = blk["w"]
+    b_ms = b_tot / args.steps
+    b_tflops = bw.flops / (b_ms * 1e-3) / 1e12
+    # the block's attention has the prefill's shape and flags, so its time is the prefill's
+    proj_ms = max(1e-9, b_ms - per_launch_ms)
+    proj_tflops = bw.projection_flops / (proj_ms * 1e-3) / 1e12
+    block_out = {
+        "workload": bw.name, "value": aggregate_rate(bw.flops * args.steps, world, b_tot) / 1e12,
+        "unit": "TFLOP/s", "ms": b_ms, "flops": bw.flops, "projection_flops": bw.projection_flops,
+        "roofline": {"bound": "tensor", "achieved": b_tflops, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": b_tflops / pk["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{pk.get('source')} burst bf16 dense"},
+        "projections_derived": {"tflops": proj_tflops, "ms": proj_ms,
+                                "frac": proj_tflops / pk["bf16_tflops"],
+                                "how": "block time minus the prefill time of the same shape"}}
+    xb = blk["hx"].numel() * blk["hx"].element_size()
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v)) + sum(
-        d["hq"].numel() * d["hq"].element_size() for d in decs)
-    d2h = q.numel() * q.element_size() + sum(d["hq"].numel() * d["hq"].element_size() for d in decs)
+        d["hq"].numel() * d["hq"].element_size() for d in decs) + xb
+    d2h = q.numel() * q.element_size() + sum(
+        d["hq"].numel() * d["hq"].element_size() for d in decs) + xb
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         val, dt, sample = oracle_sample_tflops()
@@ -356,9 +411,10 @@ def run_ours(args, rank, world):
     line = {
         "metric": METRIC, "value": aggregate_rate(flops_step * args.steps, world, p_tot) / 1e12,
         "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": (p_tot + sum(d_tot)) / args.steps, "higher_is_better": True,
+        "ms_per_step": (p_tot + sum(d_tot) + b_tot) / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "decode_workloads": [d["w"].name for d in decs],
+                   "block_workload": bw.name,
                    "parallelism": f"replicas{world}",
                    "l2": "flushed: 256 MiB memset before every kernel family, outside the events",
                    "timed_region_ms": region_ms},
@@ -367,11 +423,13 @@ def run_ours(args, rank, world):
                      "traffic": traffic.get(w.name), "kernel": "prefill_tc_kernel<128>",
                      "peak_source": f"{pk.get('source')} burst bf16 dense"},
         "decode": decode_out,
+        "block": block_out,
         "e2e": {"value": aggregate_rate(flops_step * args.steps, world, e2e_ms) / 1e12,
                 "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": e2e_ms / args.steps,
-                "note": "prefill FLOPs over the whole step incl. copies and both decodes"},
-        "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES * len(decs)),
+                "note": "prefill FLOPs over the whole step incl. copies, both decodes and the "
+                        "block (block weights resident; x in, out back)"},
+        "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES * len(decs) + BLOCK_LAUNCHES),
         "clocks": clk,
         "cpu_baseline": cpu,
     }
@@ -385,7 +443,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "block"], default="all",
                     help="run one kernel family only (for profiler captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:

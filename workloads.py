@@ -89,6 +89,23 @@ class Block:
     pos0: int = 0
     seed: int = 0
 
+    @property
+    def attention(self) -> Prefill:
+        """The attention core this block runs between its projections."""
+        return Prefill(self.name + "_attention", B=self.B, T=self.T, H=self.H, KV=self.KV,
+                       hd=self.hd, causal=self.causal, window=self.window,
+                       rope_base=self.rope_base, alibi=self.alibi, pos0=self.pos0, seed=self.seed)
+
+    @property
+    def projection_flops(self) -> int:
+        """2*M*N*K of x@Wq, x@Wk, x@Wv and ctx@Wo, with M = B*T rows."""
+        M = self.B * self.T
+        return 2 * M * self.d * (self.H + 2 * self.KV) * self.hd + 2 * M * self.H * self.hd * self.d
+
+    @property
+    def flops(self) -> int:
+        return self.projection_flops + self.attention.flops
+
 
 # The workloads of this library, named by what they are.
 TINY_BLOCK = Block("tiny_block_fp32_T6_d32_H4_KV2_hd8", B=1, T=6, d=32, H=4, KV=2, hd=8,
@@ -105,6 +122,9 @@ DECODE_GQA = Decode("decode_bf16_B64_H32_KV8_hd128_L1024-8192", B=64, H=32, KV=8
                     Lmax=8192, len_lo=1024, len_hi=8192, seed=4)
 DECODE_MQA = Decode("decode_bf16_B64_H32_KV1_hd128_L1024-8192", B=64, H=32, KV=1, hd=128,
                     Lmax=8192, len_lo=1024, len_hi=8192, seed=5)
+# A Llama-style bf16 block whose attention is the GQA prefill's shape (d_model 4096).
+GQA_BLOCK = Block("gqa_block_bf16_B2_T4096_d4096_H32_KV8_hd128", B=2, T=4096, d=4096, H=32, KV=8,
+                  hd=128, rope_base=500000.0, causal=True, seed=6)
 
 PREFILLS = {w.name: w for w in (MHA_ROPE, MHA_ALIBI, GQA, LONG_WINDOW)}
 DECODES = {w.name: w for w in (DECODE_GQA, DECODE_MQA)}
@@ -140,6 +160,19 @@ def prefill_inputs(w: Prefill, dtype=torch.bfloat16):
     k = normal((w.B, w.T, w.KV, w.hd), w.seed, dtype, gen)
     v = normal((w.B, w.T, w.KV, w.hd), w.seed, dtype, gen)
     return q, k, v
+
+
+def block_inputs(w: Block, dtype=torch.bfloat16):
+    """x [B,T,d] ~ N(0,1); Wq [d,H*hd], Wk/Wv [d,KV*hd], Wo [H*hd,d] ~ N(0,1)/sqrt(d), drawn in
+    the order x, Wq, Wk, Wv, Wo from one generator (the lab's order and scaling)."""
+    gen = torch.Generator().manual_seed(w.seed)
+    x = normal((w.B, w.T, w.d), w.seed, dtype, gen)
+    scale = 1.0 / float(np.sqrt(w.d))
+    Ws = {}
+    for n, shape in (("Wq", (w.d, w.H * w.hd)), ("Wk", (w.d, w.KV * w.hd)),
+                     ("Wv", (w.d, w.KV * w.hd)), ("Wo", (w.H * w.hd, w.d))):
+        Ws[n] = (torch.randn(*shape, generator=gen, dtype=torch.float32) * scale).to(dtype)
+    return x, Ws
 
 
 def decode_lengths(w: Decode) -> torch.Tensor:
