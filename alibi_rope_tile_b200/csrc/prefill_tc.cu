@@ -107,10 +107,12 @@ struct TcArgs {
 // one 16-byte chunk (4 pairs) of the row and the rows phase, phase + PH, phase + 2 PH ...
 // Along those rows the angle of a pair grows by the fixed step PH * w, so the cosine and
 // sine follow the angle-addition recurrence (c, s) <- (c C - s S, s C + c S) with (C, S)
-// the step's cosine and sine, computed once per CTA. The start angle of each tile is
-// computed accurately, so rounding can build up over at most NR - 1 steps. Eight threads
-// of a quarter warp cover the 8 chunks of one 128-byte row: shared-memory accesses are
-// free of bank conflicts. Only FMA-pipe arithmetic runs per element.
+// the step's cosine and sine, computed once per CTA. A query tile's start angle is computed
+// accurately; consecutive key tiles take theirs from the previous one by the same recurrence
+// with the step BN * w (rotate_next), so fp32 rounding builds up over the tiles of one CTA
+// (a few hundred steps at most, far below bf16 resolution). Eight threads of a quarter warp
+// cover the 8 chunks of one 128-byte row: shared-memory accesses are free of bank
+// conflicts. Only FMA-pipe arithmetic runs per element.
 template <int HD>
 struct KRot {
   static constexpr int CH = HD / 8;       // 16-byte chunks per row
@@ -118,6 +120,8 @@ struct KRot {
   static constexpr int NR = BN / PH;      // rows per thread
   int chunk, phase;
   float stepc[4], steps[4];
+  f2x TC[2], TS[2];  // cosine and sine of the key-tile step BN * w (pairs 0-1, 2-3 of the chunk)
+  f2x KC[2], KS[2];  // start angle of the next key tile
   __device__ __forceinline__ void init(int t, const RopeFreqs& rope) {
     chunk = t % CH;
     phase = t / CH;
@@ -127,19 +131,52 @@ struct KRot {
       rope_cos_sin(PH, rope.hi[pc], rope.lo[pc], stepc[e], steps[e]);
     }
   }
+  // The key tiles that follow start at position pos_row0 (first tile), pos_row0 + BN, ...
+  __device__ __forceinline__ void start_keys(int pos_row0, const RopeFreqs& rope) {
+    float c[4], sn[4], tc[4], ts[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int pc = chunk * 4 + e;
+      rope_cos_sin(pos_row0 + phase, rope.hi[pc], rope.lo[pc], c[e], sn[e]);
+      rope_cos_sin(BN, rope.hi[pc], rope.lo[pc], tc[e], ts[e]);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      KC[h] = pk2(c[2 * h], c[2 * h + 1]);
+      KS[h] = pk2(sn[2 * h], sn[2 * h + 1]);
+      TC[h] = pk2(tc[2 * h], tc[2 * h + 1]);
+      TS[h] = pk2(ts[2 * h], ts[2 * h + 1]);
+    }
+  }
+  // Rotate the next key tile, then advance the start angle by BN rows.
+  __device__ __forceinline__ void rotate_next(uint8_t* tile) {
+    rotate_from(tile, KC, KS);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const f2x Cn = fma2(neg2(KS[h]), TS[h], mul2(KC[h], TC[h]));
+      KS[h] = fma2(KC[h], TS[h], mul2(KS[h], TC[h]));
+      KC[h] = Cn;
+    }
+  }
+  // Rotate a tile whose first row sits at position pos_row0 (start angle computed accurately).
   __device__ __forceinline__ void rotate(uint8_t* tile, int pos_row0, const RopeFreqs& rope) const {
-    // pairs (0, 1) and (2, 3) of the chunk are handled two at a time in packed f32x2 form
     float c[4], sn[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int pc = chunk * 4 + e;
       rope_cos_sin(pos_row0 + phase, rope.hi[pc], rope.lo[pc], c[e], sn[e]);
     }
+    const f2x C0[2] = {pk2(c[0], c[1]), pk2(c[2], c[3])};
+    const f2x S0[2] = {pk2(sn[0], sn[1]), pk2(sn[2], sn[3])};
+    rotate_from(tile, C0, S0);
+  }
+  __device__ __forceinline__ void rotate_from(uint8_t* tile, const f2x (&C0)[2], const f2x (&S0)[2]) const {
+    // pairs (0, 1) and (2, 3) of the chunk are handled two at a time in packed f32x2 form
     f2x C[2], S[2], N[2], SC[2], SS[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      C[h] = pk2(c[2 * h], c[2 * h + 1]);
-      S[h] = pk2(sn[2 * h], sn[2 * h + 1]);
+      C[h] = C0[h];
+      S[h] = S0[h];
       N[h] = neg2(S[h]);
       SC[h] = pk2(stepc[2 * h], stepc[2 * h + 1]);
       SS[h] = pk2(steps[2 * h], steps[2 * h + 1]);
@@ -304,13 +341,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (valid[s]) krot.rotate(sQ + s * C::Q_BYTES, p.pos0 + qs[s], p.rope);
     fence_proxy_async();
     mbar_arrive(q_rot);
+    // hd = 128: key-tile start angles by recurrence; hd = 64 (half the rotation work per
+    // tile, and registers are tighter) computes each accurately
+    if constexpr (HD == 128)
+      if (p.rope.on) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
     int u = 0, tcnt = 0;
     for (int j = jt0; j <= jt1; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++u) {
         const int st = u % C::NS, n = u / C::NS;
         if (!mbar_wait(kv_full + st, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
         if (tid == WARP_ROPE0 * 32) TRACE(3, tcnt, 20 + kv);
-        if (kv == 0 && p.rope.on) krot.rotate(sKV + st * C::KV_BYTES, p.pos0 + j * BN, p.rope);
+        if (kv == 0 && p.rope.on) {
+          if constexpr (HD == 128)
+            krot.rotate_next(sKV + st * C::KV_BYTES);
+          else
+            krot.rotate(sKV + st * C::KV_BYTES, p.pos0 + j * BN, p.rope);
+        }
         fence_proxy_async();
         mbar_arrive(k_rot + st);
         if (tid == WARP_ROPE0 * 32) TRACE(3, tcnt, 22);
