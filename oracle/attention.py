@@ -171,6 +171,65 @@ def decode(q, kcache, vcache, seqlens, qpos, *, rope_base: float = 0.0, window: 
     return out, lse
 
 
+def kv_write(k_new, v_new, kcache, vcache, pos0, *, rope_base: float = 0.0):
+    """Write a chunk of keys and values into the cache ([XF5] "KV caching"), in fp64.
+
+    k_new, v_new [B,Tn,KV,hd]; row t of sequence b goes to slot pos0[b] + t, its key turned
+    at that position (slots are positions). Returns the updated caches (fp64 copies).
+    """
+    kc, vc = _f64(kcache).copy(), _f64(vcache).copy()
+    k_new, v_new = _f64(k_new), _f64(v_new)
+    B, Tn = k_new.shape[:2]
+    for b in range(B):
+        p = int(pos0[b]) + np.arange(Tn)
+        kb = k_new[b].transpose(1, 0, 2)                       # [KV,Tn,hd]
+        if rope_base > 0:
+            kb = rope(kb, p, rope_base)
+        kc[b, p] = kb.transpose(1, 0, 2)
+        vc[b, p] = v_new[b]
+    return kc, vc
+
+
+def chunk(q, kcache, vcache, seqlens, qpos0, *, rope_base: float = 0.0, causal: bool = True,
+          window: int = 0, slopes=None):
+    """A chunk of queries against a cache: prefill that continues a sequence ([XF5] "KV
+    caching"; [LAB] exercise 2 with several new tokens at once).
+
+    q [B,Tq,H,hd] before rotation; row i of sequence b sits at position qpos0[b] + i and is
+    turned there. kcache, vcache [B,Lmax,KV,hd] hold keys already rotated at their slot;
+    slots 0..seqlens[b]-1 are candidates, and (query position P, slot j) is allowed under the
+    same causal / window rule as a prefill: j <= P, P - j < W. ALiBi adds -slope_h |P - j|.
+    Returns out [B,Tq,H,hd] and lse [B,H,Tq]; a row with no allowed slot gets zeros, -inf.
+    """
+    q = _f64(q)
+    B, Tq, H, hd = q.shape
+    KV = kcache.shape[2]
+    group = H // KV
+    out = np.zeros((B, Tq, H, hd))
+    lse = np.full((B, H, Tq), -np.inf)
+    for b in range(B):
+        L = int(seqlens[b])
+        P = int(qpos0[b]) + np.arange(Tq)                    # query positions
+        qb = q[b].transpose(1, 0, 2)                         # [H,Tq,hd]
+        if rope_base > 0:
+            qb = rope(qb, P, rope_base)
+        if L == 0:
+            continue
+        kb = _f64(kcache[b, :L]).transpose(1, 0, 2)          # [KV,L,hd]
+        vb = _f64(vcache[b, :L]).transpose(1, 0, 2)
+        i = P.reshape(-1, 1)
+        j = np.arange(L).reshape(1, -1)
+        ok = _allowed(i, j, causal, window)
+        for h in range(H):
+            g = h // group
+            s = qb[h] @ kb[g].T / np.sqrt(hd)
+            if slopes is not None:
+                s = s - float(slopes[h]) * np.abs(i - j)
+            w, lse[b, h] = _masked_softmax_rows(s, ok)
+            out[b, :, h] = w @ vb[g]
+    return out, lse
+
+
 def block(x, Wq, Wk, Wv, Wo, *, H: int, KV: int, pos0: int = 0, rope_base: float = 0.0,
           causal: bool = True, window: int = 0, slopes=None):
     """Projections, attention and output projection of [LAB] attention(): x [B,T,d] -> [B,T,d].

@@ -138,3 +138,26 @@ def decode(q, kcache, vcache, seqlens, qpos, *, rope_base=0.0, window=0, slopes=
         out.append(ob)
         lse.append(lb)
     return out, lse
+
+
+def chunk(q, kcache, vcache, seqlens, qpos0, *, rope_base=0.0, causal=True, window=0, slopes=None):
+    """q [B][Tq][H][hd] (not rotated), row i at position qpos0[b] + i; caches with rotated keys."""
+    q, kc, vc = _rows(q), _rows(kcache), _rows(vcache)
+    B, Tq, H, KV = len(q), len(q[0]), len(q[0][0]), len(kc[0][0])
+    out = [[[None] * H for _ in range(Tq)] for _ in range(B)]
+    lse = [[[None] * Tq for _ in range(H)] for _ in range(B)]
+    for b in range(B):
+        L = int(seqlens[b])
+        for h in range(H):
+            g = h // (H // KV)
+            keys = [kc[b][j][g] for j in range(L)]
+            vals = [vc[b][j][g] for j in range(L)]
+            slope = None if slopes is None else float(slopes[h])
+            for i in range(Tq):
+                p = int(qpos0[b]) + i
+                qv = rotate_vec(q[b][i][h], p, rope_base) if rope_base > 0 else q[b][i][h]
+                o, s = attend_one(qv, keys, vals, p, list(range(L)), causal=causal, window=window,
+                                  slope=slope)
+                out[b][i][h] = o
+                lse[b][h][i] = s
+    return out, lse

@@ -39,6 +39,12 @@ MUTANTS = {
     "decode_qpos_shift": ("qb = rope(qb[:, None, :], [p], rope_base)[:, 0, :]",
                           "qb = rope(qb[:, None, :], [p - 1], rope_base)[:, 0, :]"),
     "decode_window": ("ok = (p - j) < window if window > 0", "ok = (p - j) <= window if window > 0"),
+    "chunk_position_shift": ("P = int(qpos0[b]) + np.arange(Tq)                    # query positions",
+                             "P = int(qpos0[b]) + np.arange(Tq) + 1"),
+    "chunk_keys_beyond_length": ("kb = _f64(kcache[b, :L]).transpose(1, 0, 2)          # [KV,L,hd]",
+                                 "kb = _f64(kcache[b, :L + 1]).transpose(1, 0, 2)"),
+    "kv_write_rotation_position": ("kb = rope(kb, p, rope_base)\n        kc[b, p]",
+                                   "kb = rope(kb, p + 1, rope_base)\n        kc[b, p]"),
     "block_wq_transposed": ("q = (x @ Wq).reshape(B, T, H, hd)", "q = (x @ Wq.T).reshape(B, T, H, hd)"),
     "block_head_split": ("q = (x @ Wq).reshape(B, T, H, hd)",
                          "q = (x @ Wq).reshape(B, T, hd, H).swapaxes(2, 3)"),
@@ -52,7 +58,9 @@ PIN_TESTS = [
     ("test_zero_query_prefix_mean", False), ("test_weights_sum_to_one", False),
     ("test_scale_is_inverse_sqrt_hd", False), ("test_gqa_equals_mha_with_repeated_heads", False),
     ("test_lab_properties", True), ("test_decode_token_by_token_equals_full", False),
-    ("test_decode_brute_force_and_empty_cache", False),
+    ("test_decode_brute_force_and_empty_cache", False), ("test_chunked_prefill_equals_full", False),
+    ("test_chunk_brute_force_and_cache_route", False),
+    ("test_chunk_of_one_row_is_a_decode_step_and_empty_cache", False),
 ]
 
 

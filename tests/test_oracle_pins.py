@@ -278,6 +278,51 @@ def test_decode_brute_force_and_empty_cache():
         assert np.all(out[1] == 0.0) and np.all(np.isneginf(lse[1]))
 
 
+def test_chunked_prefill_equals_full():
+    """A sequence prefilled in chunks over a cache (each chunk's keys written at their own
+    positions, then its queries attending the cache) equals the one-pass prefill."""
+    B, T, H, KV, hd, base, Lmax = 2, 23, 4, 2, 8, 10000.0, 32
+    q, k, v = _rand((B, T, H, hd), 80), _rand((B, T, KV, hd), 81), _rand((B, T, KV, hd), 82)
+    bounds = [0, 7, 8, 23]  # chunks of 7, 1 and 15 rows
+    for window, slopes in [(0, None), (5, None), (0, A.alibi_slopes(H))]:
+        full, full_lse = A.attention(q, k, v, rope_base=base, window=window, slopes=slopes)
+        kc = np.zeros((B, Lmax, KV, hd)); vc = np.zeros((B, Lmax, KV, hd))
+        for c0, c1 in zip(bounds[:-1], bounds[1:]):
+            kc, vc = A.kv_write(k[:, c0:c1], v[:, c0:c1], kc, vc, [c0] * B, rope_base=base)
+            o, l = A.chunk(q[:, c0:c1], kc, vc, [c1] * B, [c0] * B, rope_base=base, window=window,
+                           slopes=slopes)
+            np.testing.assert_allclose(o, full[:, c0:c1], rtol=0, atol=1e-13)
+            np.testing.assert_allclose(l, full_lse[:, :, c0:c1], rtol=0, atol=1e-13)
+
+
+def test_chunk_brute_force_and_cache_route():
+    """chunk() against scalar loops over a cache whose keys the loops rotate themselves."""
+    B, Tq, H, KV, hd, Lmax, base = 2, 5, 4, 1, 6, 12, 10000.0
+    q = _rand((B, Tq, H, hd), 90)
+    kraw, vc = _rand((B, Lmax, KV, hd), 91), _rand((B, Lmax, KV, hd), 92)
+    kc = [[[brute.rotate_vec(list(kraw[b, j, g]), j, base) for g in range(KV)] for j in range(Lmax)]
+          for b in range(B)]
+    seqlens, qpos0 = [9, 12], [4, 7]
+    for causal, window, slopes in [(True, 0, None), (True, 3, A.alibi_slopes(H)), (False, 0, None)]:
+        out, lse = A.chunk(q, np.array(kc), vc, seqlens, qpos0, rope_base=base, causal=causal,
+                           window=window, slopes=slopes)
+        bo, bl = brute.chunk(q, kc, vc, seqlens, qpos0, rope_base=base, causal=causal, window=window,
+                             slopes=slopes)
+        np.testing.assert_allclose(out, np.array(bo), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, np.array(bl), rtol=0, atol=1e-12)
+
+
+def test_chunk_of_one_row_is_a_decode_step_and_empty_cache():
+    B, H, KV, hd, Lmax, base = 3, 4, 2, 8, 10, 10000.0
+    q, kc, vc = _rand((B, 1, H, hd), 95), _rand((B, Lmax, KV, hd), 96), _rand((B, Lmax, KV, hd), 97)
+    seqlens = [6, 0, 10]
+    o, l = A.chunk(q, kc, vc, seqlens, [5, 0, 9], rope_base=base)
+    do, dl = A.decode(q[:, 0], kc, vc, seqlens, [5, 0, 9], rope_base=base)
+    np.testing.assert_allclose(o[:, 0], do, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l[:, :, 0], dl, rtol=0, atol=1e-13)
+    assert np.all(o[1] == 0.0) and np.all(np.isneginf(l[1]))
+
+
 # ----------------------------------------------------------------------------- workloads
 def test_workload_pair_counts():
     """FLOP counts used by the bench: causal pairs T(T+1)/2, windowed pairs sum min(i+1, W)."""
