@@ -35,6 +35,9 @@ SIGNATURES = {
     "attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _FP, _I,
                                  _P]),
     "attn_kv_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_prefill_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _FP,
+                                _I, _P]),
+    "attn_kv_write": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
     "attn_block_workspace_size": (_S, [_I, _I, _I, _I, _I, _I, _I]),
     "attn_block": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _L, _F, _I, _I, _FP, _I,
                         _P, _S, _P]),
@@ -178,6 +181,36 @@ def attn_decode_noalloc(q, kcache, vcache, seqlens, qpos, out, lse=None, *,
                                    _dtype(q), _stream(stream))
     _check(st)
     return out
+
+
+def attn_prefill_chunk(q, kcache, vcache, seqlens, qpos0, out=None, lse=None, *,
+                       rope_base: float = 0.0, causal: bool = True, window: int = 0,
+                       alibi_slopes=None, stream=None):
+    """q [B,Tq,H,hd] (not rotated; row i at position qpos0[b]+i) over caches [B,Lmax,KV,hd]
+    (keys rotated), slots < seqlens[b] -> out [B,Tq,H,hd] (and lse [B,H,Tq])."""
+    B, Tq, H, hd = q.shape
+    _, Lmax, KV, _ = kcache.shape
+    dt = q.dtype
+    if out is None:
+        out = torch.empty_like(q)
+    st = lib().attn_prefill_chunk(_dev(q, "q"), _dev(kcache, "kcache", dt), _dev(vcache, "vcache", dt),
+                                  _dev(seqlens, "seqlens", torch.int32), _dev(qpos0, "qpos0", torch.int32),
+                                  _dev(out, "out", dt), _dev(lse, "lse", torch.float32), B, Tq, H, KV, hd,
+                                  Lmax, float(rope_base), int(bool(causal)), int(window),
+                                  _slopes(alibi_slopes, H), _dtype(q), _stream(stream))
+    _check(st)
+    return out
+
+
+def attn_kv_write(k_new, v_new, kcache, vcache, pos0, *, rope_base: float = 0.0, stream=None):
+    """Write k_new, v_new [B,Tn,KV,hd] into cache slots pos0[b] .. pos0[b]+Tn-1 (keys rotated)."""
+    B, Tn, KV, hd = k_new.shape
+    Lmax = kcache.shape[1]
+    dt = k_new.dtype
+    st = lib().attn_kv_write(_dev(k_new, "k_new"), _dev(v_new, "v_new", dt), _dev(kcache, "kcache", dt),
+                             _dev(vcache, "vcache", dt), _dev(pos0, "pos0", torch.int32), B, Tn, KV, hd,
+                             Lmax, float(rope_base), _dtype(k_new), _stream(stream))
+    _check(st)
 
 
 def attn_kv_append(k_new, v_new, kcache, vcache, pos, *, rope_base: float = 0.0, stream=None):

@@ -152,6 +152,44 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
   return ok();
 }
 
+int attn_prefill_chunk(const void* q, const void* kcache, const void* vcache, const int* seqlens,
+                       const int* qpos0, void* out, float* lse, int B, int Tq, int H, int KV, int hd,
+                       int Lmax, float rope_base, int causal, int window, const float* alibi_slopes,
+                       int dtype, void* stream) {
+  int st = check_common(H, KV, hd, dtype, rope_base);
+  if (st) return st;
+  if (!q || !kcache || !vcache || !seqlens || !qpos0 || !out)
+    return fail(ATTN_ERR_ARG, "q, kcache, vcache, seqlens, qpos0 and out must not be NULL");
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out) || (lse && !aligned16(lse)))
+    return fail(ATTN_ERR_ALIGN, "q, kcache, vcache, out and lse must be 16-byte aligned");
+  if (B < 1 || Tq < 1 || Lmax < 1 || Lmax >= (1 << 24) || Tq >= (1 << 24))
+    return fail(ATTN_ERR_ARG, "B, Tq >= 1 and 1 <= Lmax < 2^24");
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
+  if (window < 0) window = 0;
+  if (window > 0 && !causal) return fail(ATTN_ERR_ARG, "a window requires the causal mask");
+  if ((long long)B * Tq * H * hd >= (1LL << 40) || (long long)B * Lmax * KV * hd >= (1LL << 40))
+    return fail(ATTN_ERR_ARG, "tensor too large");
+
+  PrefillParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.k = kcache; p.v = vcache; p.out = out; p.lse = lse;
+  p.B = B; p.T = Tq; p.H = H; p.KV = KV; p.hd = hd;
+  p.pos0 = 0; p.causal = causal; p.window = window;
+  p.seqlens = seqlens; p.qpos0 = qpos0; p.Lk = Lmax;
+  p.scale = (float)(1.0 / std::sqrt((double)hd));
+  p.rope = make_rope(hd, rope_base);
+  if ((st = make_alibi(H, alibi_slopes, &p.alibi))) return st;
+  if (!prefill_tc_supported(p, dtype))
+    return fail(ATTN_ERR_UNSUPPORTED, "attn_prefill_chunk runs bf16 with hd 64 or 128 (got dtype %d, hd %d)",
+                dtype, hd);
+  int err = 0;
+  p.status = device_status(&err);
+  if (!p.status) return err;
+  cudaError_t e = launch_prefill_tc(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_prefill_chunk launch");
+  return ok();
+}
+
 size_t attn_decode_workspace_size(int B, int H, int KV, int hd, int Lmax) {
   if (B < 1 || H < 1 || KV < 1 || H % KV || hd < 2 || hd > ATTN_MAX_HD || Lmax < 1) return 0;
   return decode_workspace_bytes(B, H, KV, hd, Lmax);
@@ -210,13 +248,36 @@ int attn_kv_append(const void* k_new, const void* v_new, void* kcache, void* vca
   AppendParams p;
   std::memset(&p, 0, sizeof(p));
   p.k_new = k_new; p.v_new = v_new; p.kcache = kcache; p.vcache = vcache; p.pos = pos;
-  p.B = B; p.KV = KV; p.hd = hd; p.Lmax = Lmax;
+  p.B = B; p.Tn = 1; p.KV = KV; p.hd = hd; p.Lmax = Lmax;
   p.rope = make_rope(hd, rope_base);
   int err = 0;
   p.status = device_status(&err);
   if (!p.status) return err;
   cudaError_t e = launch_kv_append(p, dtype, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attn_kv_append launch");
+  return ok();
+}
+
+int attn_kv_write(const void* k_new, const void* v_new, void* kcache, void* vcache, const int* pos0,
+                  int B, int Tn, int KV, int hd, int Lmax, float rope_base, int dtype, void* stream) {
+  int st = check_common(KV, KV, hd, dtype, rope_base);
+  if (st) return st;
+  if (!k_new || !v_new || !kcache || !vcache || !pos0)
+    return fail(ATTN_ERR_ARG, "k_new, v_new, kcache, vcache and pos0 must not be NULL");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kcache) || !aligned16(vcache))
+    return fail(ATTN_ERR_ALIGN, "k_new, v_new and the caches must be 16-byte aligned");
+  if (B < 1 || B > 0x7fffffff || Tn < 1 || Tn > 65535 || Lmax < 1 || Lmax >= (1 << 24))
+    return fail(ATTN_ERR_ARG, "B >= 1, 1 <= Tn <= 65535 and 1 <= Lmax < 2^24");
+  AppendParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.k_new = k_new; p.v_new = v_new; p.kcache = kcache; p.vcache = vcache; p.pos = pos0;
+  p.B = B; p.Tn = Tn; p.KV = KV; p.hd = hd; p.Lmax = Lmax;
+  p.rope = make_rope(hd, rope_base);
+  int err = 0;
+  p.status = device_status(&err);
+  if (!p.status) return err;
+  cudaError_t e = launch_kv_append(p, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_kv_write launch");
   return ok();
 }
 

@@ -285,17 +285,18 @@ cudaError_t launch_t(const DecodeParams& p, void* ws, cudaStream_t s) {
   }
 }
 
+// Row t of sequence b (block (b, t)) goes to slot pos[b] + t, its key turned at that position.
 template <typename T>
 __global__ void kv_append_kernel(const AppendParams p) {
-  const int b = blockIdx.x;
-  const int pos = p.pos[b];
-  if (pos < 0 || pos >= p.Lmax) {
+  const int b = blockIdx.x, t = blockIdx.y;
+  const int pos = p.pos[b] + t;
+  if (p.pos[b] < 0 || pos < 0 || pos >= p.Lmax) {
     if (threadIdx.x == 0) flag_error(p.status, DEV_BAD_ARG);
     return;
   }
   const int half = p.hd / 2;
-  const T* kn = static_cast<const T*>(p.k_new) + (size_t)b * p.KV * p.hd;
-  const T* vn = static_cast<const T*>(p.v_new) + (size_t)b * p.KV * p.hd;
+  const T* kn = static_cast<const T*>(p.k_new) + ((size_t)b * p.Tn + t) * p.KV * p.hd;
+  const T* vn = static_cast<const T*>(p.v_new) + ((size_t)b * p.Tn + t) * p.KV * p.hd;
   T* kc = static_cast<T*>(p.kcache) + ((size_t)b * p.Lmax + pos) * p.KV * p.hd;
   T* vc = static_cast<T*>(p.vcache) + ((size_t)b * p.Lmax + pos) * p.KV * p.hd;
   for (int idx = threadIdx.x; idx < p.KV * half; idx += blockDim.x) {
@@ -335,10 +336,11 @@ cudaError_t launch_decode(const DecodeParams& p, int dtype, void* ws, cudaStream
 }
 
 cudaError_t launch_kv_append(const AppendParams& p, int dtype, cudaStream_t s) {
+  const dim3 grid(p.B, p.Tn);
   if (dtype == 0)
-    kv_append_kernel<float><<<p.B, 128, 0, s>>>(p);
+    kv_append_kernel<float><<<grid, 128, 0, s>>>(p);
   else
-    kv_append_kernel<__nv_bfloat16><<<p.B, 128, 0, s>>>(p);
+    kv_append_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(p);
   return cudaGetLastError();
 }
 

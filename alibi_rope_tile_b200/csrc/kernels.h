@@ -23,6 +23,12 @@ struct PrefillParams {
   int* status;      // device error word
   RopeFreqs rope;
   Alibi alibi;
+  // Chunk mode (seqlens != nullptr): k and v are caches [B,Lk,KV,hd] whose keys are already
+  // rotated; query row i of sequence b sits at position qpos0[b] + i (T = query rows) and
+  // attends slots j < seqlens[b] under the same causal / window rule. Otherwise nullptr.
+  const int* seqlens;
+  const int* qpos0;
+  int Lk;
 };
 
 // CUDA-core flash prefill: fp32 or bf16 elements, any even hd <= 256.
@@ -62,8 +68,8 @@ struct AppendParams {
   const void* v_new;
   void* kcache;
   void* vcache;
-  const int* pos;
-  int B, KV, hd, Lmax;
+  const int* pos;   // [B]: slot of row 0 of sequence b
+  int B, Tn, KV, hd, Lmax;  // Tn rows per sequence
   int* status;
   RopeFreqs rope;
 };

@@ -212,7 +212,8 @@ struct KRot {
   }
 };
 
-template <int HD>
+// CHUNK: the queries continue sequences held in a cache (PrefillParams::seqlens != nullptr).
+template <int HD, bool CHUNK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ TcArgs a) {
@@ -257,19 +258,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     qs[0] = qb * 2 * BM;
     qs[1] = qs[0] + BM;
   }
+  // Keys are indexed by position in k/v (a prefill: key j = row j) or by cache slot (chunk
+  // mode); qoff is the key index of query row 0 and Tk the number of keys there are.
+  int qoff = 0, Tk = p.T, qrope0 = p.pos0;
+  if constexpr (CHUNK) {
+    qoff = p.qpos0[b];
+    Tk = p.seqlens[b];
+    qrope0 = qoff;
+    if (qoff < 0 || qoff > (1 << 24) - p.T || Tk < 0 || Tk > p.Lk) {
+      if (tid == 0) flag_error(p.status, DEV_BAD_ARG);
+      qoff = 0;
+      Tk = 0;  // nothing is attended: zero rows
+    }
+  }
   int t0[2], t1[2];
-  bool valid[2];
+  bool valid[2], has[2];
 #pragma unroll
   for (int s = 0; s < 2; ++s) {
     valid[s] = qs[s] < p.T;
-    const int lo = p.window > 0 ? max(0, qs[s] - p.window + 1) : 0;
-    const int hi = p.causal ? min(p.T - 1, qs[s] + BM - 1) : p.T - 1;
-    t0[s] = valid[s] ? lo / BN : 1;
-    t1[s] = valid[s] ? hi / BN : 0;
+    const int lo = p.window > 0 ? max(0, qoff + qs[s] - p.window + 1) : 0;
+    const int hi = p.causal ? min(Tk - 1, qoff + qs[s] + BM - 1) : Tk - 1;
+    has[s] = valid[s] && lo <= hi;  // the slot attends at least one key
+    t0[s] = has[s] ? lo / BN : 1;
+    t1[s] = has[s] ? hi / BN : 0;
   }
-  const int jt0 = valid[1] ? min(t0[0], t0[1]) : t0[0];
-  const int jt1 = valid[1] ? max(t1[0], t1[1]) : t1[0];
-  auto active = [&](int s, int j) { return valid[s] && j >= t0[s] && j <= t1[s]; };
+  const int jt0 = has[0] ? (has[1] ? min(t0[0], t0[1]) : t0[0]) : t0[1];
+  const int jt1 = has[0] ? (has[1] ? max(t1[0], t1[1]) : t1[0]) : t1[1];
+  auto active = [&](int s, int j) { return has[s] && j >= t0[s] && j <= t1[s]; };
 
   // ---- set-up: barriers, tensor memory
   if (tid == 0) {
@@ -338,20 +353,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (!mbar_wait(q_full, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
     if (p.rope.on)
       for (int s = 0; s < 2; ++s)
-        if (valid[s]) krot.rotate(sQ + s * C::Q_BYTES, p.pos0 + qs[s], p.rope);
+        if (valid[s]) krot.rotate(sQ + s * C::Q_BYTES, qrope0 + qs[s], p.rope);
     fence_proxy_async();
     mbar_arrive(q_rot);
     // hd = 128: key-tile start angles by recurrence; hd = 64 (half the rotation work per
     // tile, and registers are tighter) computes each accurately
     if constexpr (HD == 128)
-      if (p.rope.on) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
+      if (p.rope.on && !CHUNK) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
     int u = 0, tcnt = 0;
     for (int j = jt0; j <= jt1; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++u) {
         const int st = u % C::NS, n = u / C::NS;
         if (!mbar_wait(kv_full + st, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
         if (tid == WARP_ROPE0 * 32) TRACE(3, tcnt, 20 + kv);
-        if (kv == 0 && p.rope.on) {
+        if (kv == 0 && p.rope.on && !CHUNK) {  // cached keys are already rotated
           if constexpr (HD == 128)
             krot.rotate_next(sKV + st * C::KV_BYTES);
           else
@@ -394,6 +409,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       int cnt[2] = {0, 0};
       if (!mbar_wait(q_rot, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
+      if (jt1 < jt0) goto mma_drain;  // no key tile at all
       // K of the first tile
       if (!mbar_wait(k_rot + 0, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
       tc_fence_after();
@@ -476,12 +492,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int q0s = qs[s];  // first query row of the slot
         const int hs = head[s];
         const int i = q0s + r;
+        const int ip = qoff + i;  // the query's key index
         const uint32_t tS = tmem + lane_off + s * BN;
         const int key0 = j * BN + kq * 32;  // first of my 32 keys
         const float slope = p.alibi.on ? p.alibi.slope[hs] * LOG2E : 0.f;
         // does any row of this slot need per-element masking in my keys of this tile?
-        const bool need_mask = (key0 + 32 > p.T) || (p.causal && key0 + 31 > q0s) ||
-                               (p.window > 0 && q0s + BM - 1 - key0 >= p.window);
+        const bool need_mask = (key0 + 32 > Tk) || (p.causal && key0 + 31 > qoff + q0s) ||
+                               (p.window > 0 && qoff + q0s + BM - 1 - key0 >= p.window);
         const bool plain = !need_mask && !p.alibi.on;
         float x[32];
         tmem_ld32(tS + kq * 32, x);
@@ -495,9 +512,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
             const int jk = key0 + k;
-            float v = p.alibi.on ? fmaf(x[k], sc, -slope * fabsf((float)(i - jk))) : x[k] * sc;
+            float v = p.alibi.on ? fmaf(x[k], sc, -slope * fabsf((float)(ip - jk))) : x[k] * sc;
             if (need_mask) {
-              const bool ok = jk < p.T && (!p.causal || jk <= i) && (p.window <= 0 || i - jk < p.window);
+              const bool ok = jk < Tk && (!p.causal || jk <= ip) && (p.window <= 0 || ip - jk < p.window);
               v = ok ? v : -INFINITY;
             }
             x[k] = v;
@@ -581,7 +598,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
     for (int s = 0; s < 2; ++s) {
       const int c = s ? cs1 : cs0;
-      if (c == 0) continue;
+      if (c == 0) {
+        // a slot that attends no key at all (a chunk over an empty range): zero rows, lse -inf
+        const int i = qs[s] + r;
+        if (valid[s] && i < p.T) {
+          if (kq * 32 < HD) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                  (((size_t)b * p.T + i) * p.H + head[s]) * HD + kq * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+          }
+          if (p.lse && kq == 0) p.lse[((size_t)b * p.H + head[s]) * p.T + i] = -INFINITY;
+        }
+        continue;
+      }
       const float m_ref = s ? m_ref1 : m_ref0;
       // the row's total sum: the four warps' partial sums, exchanged through shared memory
       lsum[(s * 4 + kq) * 128 + r] = s ? l1 : l0;
@@ -670,8 +700,9 @@ bool make_map(CUtensorMap* map, const void* base, int B, int T, int heads, int h
 template <int HD>
 cudaError_t launch_hd(const PrefillParams& p, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, p.q, p.B, p.T, p.H, HD) || !make_map(&mk, p.k, p.B, p.T, p.KV, HD) ||
-      !make_map(&mv, p.v, p.B, p.T, p.KV, HD))
+  const int Lk = p.seqlens ? p.Lk : p.T;  // rows of k and v
+  if (!make_map(&mq, p.q, p.B, p.T, p.H, HD) || !make_map(&mk, p.k, p.B, Lk, p.KV, HD) ||
+      !make_map(&mv, p.v, p.B, Lk, p.KV, HD))
     return cudaErrorInvalidValue;
   TcArgs a;
   a.p = p;
@@ -683,10 +714,10 @@ cudaError_t launch_hd(const PrefillParams& p, cudaStream_t s) {
   a.scale_log2 = p.scale * LOG2E;
   const long long units = (long long)p.B * p.KV * a.npairs * a.nqb;
   if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Cfg<HD>::SMEM);
+  auto kern = p.seqlens ? prefill_tc_kernel<HD, true> : prefill_tc_kernel<HD, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<HD>::SMEM);
   if (e != cudaSuccess) return e;
-  prefill_tc_kernel<HD><<<(unsigned)units, NUM_THREADS, Cfg<HD>::SMEM, s>>>(mq, mk, mv, a);
+  kern<<<(unsigned)units, NUM_THREADS, Cfg<HD>::SMEM, s>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 

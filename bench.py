@@ -7,10 +7,13 @@ One step = one pass of the whole hot path over one batch of synthetic input:
     uniform in [1024, 8192]) and of its MQA variant (KV=1): split-KV partials and the
     log-sum-exp merge;
   * one pass of the bf16 block around the same attention shape (x [2,4096,4096], weights
-    resident): the x@Wq, x@Wk, x@Wv projections, the attention core, then ctx@Wo.
+    resident): the x@Wq, x@Wk, x@Wv projections, the attention core, then ctx@Wo;
+  * a chunked prefill: the second 2048 rows of the GQA sequences against a cache of their
+    4096 rotated keys (written once, before timing).
 ``value`` is the prefill TFLOP/s (causal FLOPs counted: 4*B*H*hd*allowed pairs); the decode
 GB/s (cache rows read + q + out, per launch pair) ride along under ``decode``, the block's
-TFLOP/s (projection FLOPs 2*M*N*K plus the attention's) under ``block``. Kernels are timed with CUDA events on the stream they
+TFLOP/s (projection FLOPs 2*M*N*K plus the attention's) under ``block``, the chunk's under
+``chunk``. Kernels are timed with CUDA events on the stream they
 are launched on; L2 is flushed (a 256 MiB memset, outside the timed events) before every
 step. ``e2e`` times the same call with the step's inputs copied from pinned host memory and
 its output copied back, all inside the timed region.
@@ -45,11 +48,13 @@ PREFILL = workloads.GQA
 DECODE = workloads.DECODE_GQA
 DECODE_MQA = workloads.DECODE_MQA
 BLOCK = workloads.GQA_BLOCK
+CHUNK = workloads.GQA_CHUNK
 # Algorithmic bytes and launches, stated once (see the design notes):
 #   decode bytes = cache rows read (K and V) + q + out; prefill FLOPs = PREFILL.flops.
 PREFILL_LAUNCHES = 1
 DECODE_LAUNCHES = 2       # split pass + merge, per decode workload
 BLOCK_LAUNCHES = 5        # three projection GEMMs, the prefill, the output GEMM
+CHUNK_LAUNCHES = 1
 
 
 def peaks():
@@ -236,6 +241,7 @@ def run_ours(args, rank, world):
     w = PREFILL
     do_p, do_d = args.only in ("all", "prefill"), args.only in ("all", "decode")
     do_b = args.only in ("all", "block")
+    do_c = args.only in ("all", "chunk")
 
     q, k, v = workloads.prefill_inputs(w)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
@@ -261,6 +267,19 @@ def run_ours(args, rank, world):
                                                                  torch.bfloat16),
                                   dtype=torch.uint8, device="cuda"))
         del hW
+    chk = None
+    if do_c:
+        cw = CHUNK
+        hcq, hck, hcv = workloads.chunk_inputs(cw)
+        ckc = torch.zeros(cw.B, cw.Lmax, cw.KV, cw.hd, dtype=torch.bfloat16, device="cuda")
+        cvc = torch.zeros_like(ckc)
+        art.attn_kv_write(hck.cuda(), hcv.cuda(), ckc, cvc,
+                          torch.zeros(cw.B, dtype=torch.int32, device="cuda"), rope_base=cw.rope_base)
+        chk = dict(w=cw, hq=hcq, q=hcq.cuda(), kc=ckc, vc=cvc,
+                   sl=torch.full((cw.B,), cw.qpos0 + cw.Tq, dtype=torch.int32, device="cuda"),
+                   qp=torch.full((cw.B,), cw.qpos0, dtype=torch.int32, device="cuda"),
+                   out=torch.empty(hcq.shape, dtype=hcq.dtype, device="cuda"))
+        del hck, hcv
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
     def prefill():
@@ -278,16 +297,22 @@ def run_ours(args, rank, world):
                            workspace=blk["ws"], H=bw.H, KV=bw.KV, rope_base=bw.rope_base,
                            causal=bw.causal, window=bw.window)
 
+    def chunk():
+        if chk is not None:
+            art.attn_prefill_chunk(chk["q"], chk["kc"], chk["vc"], chk["sl"], chk["qp"], chk["out"],
+                                   rope_base=chk["w"].rope_base)
+
     for _ in range(max(3, args.warmup)):
         flush.zero_()
         prefill()
         for d in decs:
             decode(d)
         block()
+        chunk()
     torch.cuda.synchronize()
     art.attn_sync_status()
 
-    nev = 2 + 2 * len(decs) + 2
+    nev = 2 + 2 * len(decs) + 4
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
@@ -307,8 +332,12 @@ def run_ours(args, rank, world):
             decode(d)
             ev[s_][3 + 2 * n].record(stream)
         flush.zero_()
-        ev[s_][nev - 2].record(stream)
+        ev[s_][nev - 4].record(stream)
         block()
+        ev[s_][nev - 3].record(stream)
+        flush.zero_()
+        ev[s_][nev - 2].record(stream)
+        chunk()
         ev[s_][nev - 1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -319,7 +348,9 @@ def run_ours(args, rank, world):
     d_tot = [max(1e-9, max_over_ranks(sum(ev[s_][2 + 2 * n].elapsed_time(ev[s_][3 + 2 * n])
                                           for s_ in range(args.steps)), world))
              for n in range(len(decs))]
-    b_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 2].elapsed_time(ev[s_][nev - 1])
+    b_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 4].elapsed_time(ev[s_][nev - 3])
+                                         for s_ in range(args.steps)), world))
+    c_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 2].elapsed_time(ev[s_][nev - 1])
                                          for s_ in range(args.steps)), world))
     region_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
 
@@ -332,6 +363,9 @@ def run_ours(args, rank, world):
     if blk is not None:
         hbx = blk["hx"].pin_memory()
         hbo = torch.empty(blk["hx"].shape, dtype=blk["hx"].dtype).pin_memory()
+    if chk is not None:
+        hcq_p = chk["hq"].pin_memory()
+        hco = torch.empty(chk["hq"].shape, dtype=chk["hq"].dtype).pin_memory()
 
     def e2e_step():
         if do_p:
@@ -348,6 +382,10 @@ def run_ours(args, rank, world):
             blk["x"].copy_(hbx, non_blocking=True)
             block()
             hbo.copy_(blk["out"], non_blocking=True)
+        if chk is not None:
+            chk["q"].copy_(hcq_p, non_blocking=True)
+            chunk()
+            hco.copy_(chk["out"], non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -366,7 +404,7 @@ def run_ours(args, rank, world):
     if args.only != "all":
         print(json.dumps({"only": args.only, "prefill_ms": p_tot / args.steps,
                           "decode_ms": [t / args.steps for t in d_tot],
-                          "block_ms": b_tot / args.steps}), flush=True)
+                          "block_ms": b_tot / args.steps, "chunk_ms": c_tot / args.steps}), flush=True)
         return
     pk = peaks()
     flops_step = w.flops
@@ -398,11 +436,22 @@ def run_ours(args, rank, world):
         "projections_derived": {"tflops": proj_tflops, "ms": proj_ms,
                                 "frac": proj_tflops / pk["bf16_tflops"],
                                 "how": "block time minus the prefill time of the same shape"}}
+    cw = chk["w"]
+    c_ms = c_tot / args.steps
+    c_tflops = cw.flops / (c_ms * 1e-3) / 1e12
+    chunk_out = {
+        "workload": cw.name, "value": aggregate_rate(cw.flops * args.steps, world, c_tot) / 1e12,
+        "unit": "TFLOP/s", "ms": c_ms, "flops": cw.flops,
+        "roofline": {"bound": "tensor", "achieved": c_tflops, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": c_tflops / pk["bf16_tflops"], "traffic": None,
+                     "kernel": "prefill_tc_kernel<128, true>",
+                     "peak_source": f"{pk.get('source')} burst bf16 dense"}}
     xb = blk["hx"].numel() * blk["hx"].element_size()
+    cb = chk["hq"].numel() * chk["hq"].element_size()
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v)) + sum(
-        d["hq"].numel() * d["hq"].element_size() for d in decs) + xb
+        d["hq"].numel() * d["hq"].element_size() for d in decs) + xb + cb
     d2h = q.numel() * q.element_size() + sum(
-        d["hq"].numel() * d["hq"].element_size() for d in decs) + xb
+        d["hq"].numel() * d["hq"].element_size() for d in decs) + xb + cb
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         val, dt, sample = oracle_sample_tflops()
@@ -411,25 +460,28 @@ def run_ours(args, rank, world):
     line = {
         "metric": METRIC, "value": aggregate_rate(flops_step * args.steps, world, p_tot) / 1e12,
         "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": (p_tot + sum(d_tot) + b_tot) / args.steps, "higher_is_better": True,
+        "ms_per_step": (p_tot + sum(d_tot) + b_tot + c_tot) / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "decode_workloads": [d["w"].name for d in decs],
-                   "block_workload": bw.name,
+                   "block_workload": bw.name, "chunk_workload": cw.name,
                    "parallelism": f"replicas{world}",
                    "l2": "flushed: 256 MiB memset before every kernel family, outside the events",
                    "timed_region_ms": region_ms},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                     "traffic": traffic.get(w.name), "kernel": "prefill_tc_kernel<128>",
+                     "traffic": traffic.get(w.name), "kernel": "prefill_tc_kernel<128, false>",
                      "peak_source": f"{pk.get('source')} burst bf16 dense"},
         "decode": decode_out,
         "block": block_out,
+        "chunk": chunk_out,
         "e2e": {"value": aggregate_rate(flops_step * args.steps, world, e2e_ms) / 1e12,
                 "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": e2e_ms / args.steps,
-                "note": "prefill FLOPs over the whole step incl. copies, both decodes and the "
-                        "block (block weights resident; x in, out back)"},
-        "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES * len(decs) + BLOCK_LAUNCHES),
+                "note": "prefill FLOPs over the whole step incl. copies, both decodes, the block "
+                        "(block weights resident; x in, out back) and the chunk (cache resident; "
+                        "its queries in, out back)"},
+        "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES * len(decs) + BLOCK_LAUNCHES
+                                      + CHUNK_LAUNCHES),
         "clocks": clk,
         "cpu_baseline": cpu,
     }
@@ -443,7 +495,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "block"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "block", "chunk"], default="all",
                     help="run one kernel family only (for profiler captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:

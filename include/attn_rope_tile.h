@@ -91,6 +91,28 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
                  int causal, int window, const float* alibi_slopes, int dtype, void* stream);
 
 /*
+ * attn_prefill_chunk -- a chunk of Tq query rows that continues sequences held in a KV
+ * cache ([XF5] "KV caching"; [LAB] exercise 2 with several new tokens at once): the step
+ * between a prefill and a decode, for prompts processed in pieces.
+ *
+ * q: [B,Tq,H,hd] BEFORE rotation; row i of sequence b sits at position qpos0[b] + i and is
+ * turned there. kcache, vcache: [B,Lmax,KV,hd]; slot j holds the key already rotated at
+ * position j (attn_kv_write / attn_kv_append write it that way; write the chunk's own keys
+ * first, so that it attends to itself). Row i attends slots j < seqlens[b] with, when
+ * causal, j <= qpos0[b] + i and, with window W > 0, qpos0[b] + i - j < W; ALiBi adds
+ * -slope_h |qpos0[b] + i - j|. seqlens, qpos0: [B] int32 (device). A row with no allowed
+ * slot gets out = 0, lse = -inf. out: [B,Tq,H,hd] (device, written); lse: [B,H,Tq] or NULL.
+ * seqlens[b] > Lmax, qpos0[b] < 0 or qpos0[b] + Tq > 2^24 is recorded as
+ * ATTN_ERR_DEVICE_ARG (attn_sync_status) and that sequence's rows are zeroed.
+ * Runs the tensor-core prefill kernel: bf16 with hd in {64, 128}; anything else returns
+ * ATTN_ERR_UNSUPPORTED.
+ */
+int attn_prefill_chunk(const void* q, const void* kcache, const void* vcache, const int* seqlens,
+                       const int* qpos0, void* out, float* lse, int B, int Tq, int H, int KV, int hd,
+                       int Lmax, float rope_base, int causal, int window, const float* alibi_slopes,
+                       int dtype, void* stream);
+
+/*
  * attn_decode_workspace_size -- bytes of device scratch attn_decode needs for these
  * sizes (split-KV partial outputs and their softmax statistics). Returns 0 on invalid
  * sizes.
@@ -156,6 +178,16 @@ int attn_decode_noalloc(const void* q, const void* kcache, const void* vcache, c
 int attn_kv_append(const void* k_new, const void* v_new, void* kcache, void* vcache,
                    const int* pos, int B, int KV, int hd, int Lmax, float rope_base, int dtype,
                    void* stream);
+
+/*
+ * attn_kv_write -- write a chunk of Tn tokens per sequence into the cache (the multi-token
+ * form of attn_kv_append, for attn_prefill_chunk): row t of sequence b goes to slot
+ * pos0[b] + t, its key rotated at that position (if rope_base > 0), its value as is.
+ * k_new, v_new: [B,Tn,KV,hd] (device). pos0: [B] int32 (device). 1 <= Tn <= 65535.
+ * A slot outside [0, Lmax) is recorded as ATTN_ERR_DEVICE_ARG and that row is skipped.
+ */
+int attn_kv_write(const void* k_new, const void* v_new, void* kcache, void* vcache, const int* pos0,
+                  int B, int Tn, int KV, int hd, int Lmax, float rope_base, int dtype, void* stream);
 
 /*
  * attn_block_workspace_size -- bytes of device scratch attn_block needs (the q, k, v and

@@ -31,6 +31,7 @@ def declared_functions():
 def test_header_declares_entry_points():
     names = declared_functions()
     for must in ("attn_prefill", "attn_decode", "attn_block", "attn_kv_append",
+                 "attn_prefill_chunk", "attn_kv_write",
                  "attn_decode_workspace_size", "attn_block_workspace_size", "attn_alibi_slopes",
                  "attn_sync_status", "attn_last_error", "attn_version"):
         assert must in names
@@ -115,6 +116,31 @@ def test_block_workspace_error(lib):
     st = lib.attn_block(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 1, 6, 32, 4, 2, 8, 0,
                         10000.0, 1, 0, None, 0, 0x1000, 16, None)
     assert st == -6
+
+
+def test_chunk_and_kv_write_argument_errors(lib):
+    P = 0x1000
+    def chunk(**kw):
+        a = dict(seqlens=P, qpos0=P, B=2, Tq=16, H=8, KV=2, hd=128, Lmax=64, causal=1, window=0,
+                 dtype=1)
+        a.update(kw)
+        return lib.attn_prefill_chunk(P, P, P, a["seqlens"], a["qpos0"], P, None, a["B"], a["Tq"],
+                                      a["H"], a["KV"], a["hd"], a["Lmax"], 10000.0, a["causal"],
+                                      a["window"], None, a["dtype"], None)
+    assert chunk(seqlens=None) == -1                 # NULL lengths
+    assert chunk(causal=0, window=8) == -1          # a window needs the causal mask
+    assert chunk(Lmax=0) == -1
+    assert chunk(H=6, KV=4) == -1                   # H % KV
+    assert chunk(dtype=0) == -3                     # fp32 has no chunk kernel
+    assert chunk(hd=48) == -3                       # neither has hd 48
+    def write(**kw):
+        a = dict(B=2, Tn=4, KV=2, hd=64, Lmax=64)
+        a.update(kw)
+        return lib.attn_kv_write(P, P, P, P, P, a["B"], a["Tn"], a["KV"], a["hd"], a["Lmax"],
+                                 10000.0, 1, None)
+    assert write(Tn=0) == -1
+    assert write(Tn=70000) == -1
+    assert write(hd=7) == -1
 
 
 def test_binding_requires_cuda_tensors(lib):

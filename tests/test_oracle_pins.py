@@ -332,3 +332,8 @@ def test_workload_pair_counts():
     assert workloads.MHA_ROPE.flops == 4 * 4 * 16 * 64 * 524800
     assert abs(workloads.GQA.flops / 1e9 - 274.9) < 0.1
     assert abs(workloads.LONG_WINDOW.flops / 1e9 - 962.1) < 0.1
+    c = workloads.GQA_CHUNK
+    assert c.allowed_pairs == sum(c.qpos0 + i + 1 for i in range(c.Tq))
+    # the chunk's rows are the second half of the GQA prefill's rows: its pairs plus the first
+    # half's make up the whole causal triangle
+    assert c.allowed_pairs + 2048 * 2049 // 2 == workloads.GQA.allowed_pairs

@@ -107,6 +107,31 @@ class Block:
         return self.projection_flops + self.attention.flops
 
 
+@dataclasses.dataclass(frozen=True)
+class Chunk:
+    """Tq query rows of each sequence at positions qpos0 .. qpos0+Tq-1, attending a cache that
+    holds the sequence's first qpos0 + Tq keys (causal)."""
+    name: str
+    B: int
+    Tq: int
+    qpos0: int
+    Lmax: int
+    H: int
+    KV: int
+    hd: int
+    rope_base: float = 10000.0
+    seed: int = 0
+
+    @property
+    def allowed_pairs(self) -> int:
+        """Allowed (query, key) pairs per (batch, head): row i sees qpos0 + i + 1 keys."""
+        return self.Tq * self.qpos0 + self.Tq * (self.Tq + 1) // 2
+
+    @property
+    def flops(self) -> int:
+        return 4 * self.B * self.H * self.hd * self.allowed_pairs
+
+
 # The workloads of this library, named by what they are.
 TINY_BLOCK = Block("tiny_block_fp32_T6_d32_H4_KV2_hd8", B=1, T=6, d=32, H=4, KV=2, hd=8,
                    rope_base=10000.0, causal=True, seed=0)
@@ -122,6 +147,9 @@ DECODE_GQA = Decode("decode_bf16_B64_H32_KV8_hd128_L1024-8192", B=64, H=32, KV=8
                     Lmax=8192, len_lo=1024, len_hi=8192, seed=4)
 DECODE_MQA = Decode("decode_bf16_B64_H32_KV1_hd128_L1024-8192", B=64, H=32, KV=1, hd=128,
                     Lmax=8192, len_lo=1024, len_hi=8192, seed=5)
+# The second half of the GQA prefill's sequences as a chunk over a cache of their 4096 keys.
+GQA_CHUNK = Chunk("gqa_chunk_bf16_B2_Tq2048_at2048_H32_KV8_hd128", B=2, Tq=2048, qpos0=2048,
+                  Lmax=4096, H=32, KV=8, hd=128, rope_base=500000.0, seed=7)
 # A Llama-style bf16 block whose attention is the GQA prefill's shape (d_model 4096).
 GQA_BLOCK = Block("gqa_block_bf16_B2_T4096_d4096_H32_KV8_hd128", B=2, T=4096, d=4096, H=32, KV=8,
                   hd=128, rope_base=500000.0, causal=True, seed=6)
@@ -173,6 +201,17 @@ def block_inputs(w: Block, dtype=torch.bfloat16):
                      ("Wv", (w.d, w.KV * w.hd)), ("Wo", (w.H * w.hd, w.d))):
         Ws[n] = (torch.randn(*shape, generator=gen, dtype=torch.float32) * scale).to(dtype)
     return x, Ws
+
+
+def chunk_inputs(w: Chunk, dtype=torch.bfloat16):
+    """q [B,Tq,H,hd] (the chunk's queries, not rotated) and k, v [B,qpos0+Tq,KV,hd] (the keys
+    and values of every position up to the chunk's end, not rotated), drawn in that order."""
+    gen = torch.Generator().manual_seed(w.seed)
+    n = w.qpos0 + w.Tq
+    q = normal((w.B, w.Tq, w.H, w.hd), w.seed, dtype, gen)
+    k = normal((w.B, n, w.KV, w.hd), w.seed, dtype, gen)
+    v = normal((w.B, n, w.KV, w.hd), w.seed, dtype, gen)
+    return q, k, v
 
 
 def decode_lengths(w: Decode) -> torch.Tensor:
