@@ -171,6 +171,31 @@ def decode(q, kcache, vcache, seqlens, qpos, *, rope_base: float = 0.0, window: 
     return out, lse
 
 
+def gather_pages(pages, block_table, L: int, page_size: int, b: int) -> np.ndarray:
+    """Slots 0..L-1 of sequence b from a paged cache: slot j lives in row j % page_size of
+    page block_table[b][j // page_size]. pages [num_pages, page_size, KV, hd]."""
+    pages = _f64(pages)
+    j = np.arange(L)
+    page = np.asarray(block_table)[b][j // page_size]
+    return pages[page, j % page_size]                          # [L, KV, hd]
+
+
+def decode_paged(q, kpages, vpages, block_table, seqlens, qpos, *, page_size: int,
+                 rope_base: float = 0.0, window: int = 0, slopes=None):
+    """decode() over a paged cache: the cache of sequence b is its pages in block-table order
+    (the serving layout the pages' PagedAttention mention stands for). Returns out, lse."""
+    B = len(seqlens)
+    Lmax = max(1, max(int(x) for x in seqlens))
+    KV, hd = kpages.shape[2], kpages.shape[3]
+    kc = np.zeros((B, Lmax, KV, hd))
+    vc = np.zeros((B, Lmax, KV, hd))
+    for b in range(B):
+        L = int(seqlens[b])
+        kc[b, :L] = gather_pages(kpages, block_table, L, page_size, b)
+        vc[b, :L] = gather_pages(vpages, block_table, L, page_size, b)
+    return decode(q, kc, vc, seqlens, qpos, rope_base=rope_base, window=window, slopes=slopes)
+
+
 def kv_write(k_new, v_new, kcache, vcache, pos0, *, rope_base: float = 0.0):
     """Write a chunk of keys and values into the cache ([XF5] "KV caching"), in fp64.
 

@@ -161,3 +161,31 @@ def chunk(q, kcache, vcache, seqlens, qpos0, *, rope_base=0.0, causal=True, wind
                 out[b][i][h] = o
                 lse[b][h][i] = s
     return out, lse
+
+
+def decode_paged(q, kpages, vpages, block_table, seqlens, qpos, *, page_size, rope_base=0.0,
+                 window=0, slopes=None):
+    """decode() with each cached row looked up through the block table, one slot at a time."""
+    q, kp, vp = _rows(q), _rows(kpages), _rows(vpages)
+    table = _rows(block_table)
+    B, H, KV = len(q), len(q[0]), len(kp[0][0])
+    out, lse = [], []
+    for b in range(B):
+        L, p = int(seqlens[b]), int(qpos[b])
+        ob, lb = [], []
+        for h in range(H):
+            g = h // (H // KV)
+            qv = rotate_vec(q[b][h], p, rope_base) if rope_base > 0 else q[b][h]
+            keys, vals = [], []
+            for j in range(L):
+                page, row = int(table[b][j // page_size]), j % page_size
+                keys.append(kp[page][row][g])
+                vals.append(vp[page][row][g])
+            slope = None if slopes is None else float(slopes[h])
+            o, s = attend_one(qv, keys, vals, p, list(range(L)), causal=False, window=window,
+                              slope=slope)
+            ob.append(o)
+            lb.append(s)
+        out.append(ob)
+        lse.append(lb)
+    return out, lse

@@ -45,6 +45,9 @@ MUTANTS = {
                                  "kb = _f64(kcache[b, :L + 1]).transpose(1, 0, 2)"),
     "kv_write_rotation_position": ("kb = rope(kb, p, rope_base)\n        kc[b, p]",
                                    "kb = rope(kb, p + 1, rope_base)\n        kc[b, p]"),
+    "paged_row_index": ("return pages[page, j % page_size]", "return pages[page, (j + 1) % page_size]"),
+    "paged_block_index": ("page = np.asarray(block_table)[b][j // page_size]",
+                          "page = np.asarray(block_table)[b][j % page_size]"),
     "block_wq_transposed": ("q = (x @ Wq).reshape(B, T, H, hd)", "q = (x @ Wq.T).reshape(B, T, H, hd)"),
     "block_head_split": ("q = (x @ Wq).reshape(B, T, H, hd)",
                          "q = (x @ Wq).reshape(B, T, hd, H).swapaxes(2, 3)"),
@@ -61,6 +64,7 @@ PIN_TESTS = [
     ("test_decode_brute_force_and_empty_cache", False), ("test_chunked_prefill_equals_full", False),
     ("test_chunk_brute_force_and_cache_route", False),
     ("test_chunk_of_one_row_is_a_decode_step_and_empty_cache", False),
+    ("test_paged_decode_brute_force_and_page_order", False),
 ]
 
 

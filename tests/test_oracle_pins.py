@@ -323,6 +323,33 @@ def test_chunk_of_one_row_is_a_decode_step_and_empty_cache():
     assert np.all(o[1] == 0.0) and np.all(np.isneginf(l[1]))
 
 
+def test_paged_decode_brute_force_and_page_order():
+    """Paged decode against slot-by-slot page lookups, and invariance under where the pages sit:
+    the same rows in a shuffled page pool give the contiguous cache's result."""
+    B, H, KV, hd, ps, base = 3, 4, 2, 6, 4, 10000.0
+    seqlens, qpos = [9, 0, 16], [9, 0, 15]
+    npages = 14
+    rng = np.random.default_rng(7)
+    table = rng.permutation(npages)[:12].reshape(3, 4)
+    q, kp, vp = _rand((B, H, hd), 100), _rand((npages, ps, KV, hd), 101), _rand((npages, ps, KV, hd), 102)
+    for window, slopes in [(0, None), (5, A.alibi_slopes(H))]:
+        out, lse = A.decode_paged(q, kp, vp, table, seqlens, qpos, page_size=ps, rope_base=base,
+                                  window=window, slopes=slopes)
+        bo, bl = brute.decode_paged(q, kp, vp, table, seqlens, qpos, page_size=ps, rope_base=base,
+                                    window=window, slopes=slopes)
+        np.testing.assert_allclose(out, np.array(bo), rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse, np.array(bl), rtol=0, atol=1e-13)
+        # contiguous equivalent built by hand, row by row
+        kc = np.zeros((B, 16, KV, hd)); vc = np.zeros((B, 16, KV, hd))
+        for b in range(B):
+            for j in range(seqlens[b]):
+                kc[b, j] = kp[table[b][j // ps], j % ps]
+                vc[b, j] = vp[table[b][j // ps], j % ps]
+        co, cl = A.decode(q, kc, vc, seqlens, qpos, rope_base=base, window=window, slopes=slopes)
+        np.testing.assert_allclose(out, co, rtol=0, atol=1e-13)
+        assert np.all(out[1] == 0.0) and np.all(np.isneginf(lse[1]))
+
+
 # ----------------------------------------------------------------------------- workloads
 def test_workload_pair_counts():
     """FLOP counts used by the bench: causal pairs T(T+1)/2, windowed pairs sum min(i+1, W)."""
