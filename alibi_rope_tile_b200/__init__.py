@@ -38,6 +38,9 @@ SIGNATURES = {
     "attn_prefill_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _FP,
                                 _I, _P]),
     "attn_kv_write": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _FP,
+                               _I, _P, _S, _P]),
+    "attn_kv_write_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "attn_block_workspace_size": (_S, [_I, _I, _I, _I, _I, _I, _I]),
     "attn_block": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _L, _F, _I, _I, _FP, _I,
                         _P, _S, _P]),
@@ -210,6 +213,47 @@ def attn_kv_write(k_new, v_new, kcache, vcache, pos0, *, rope_base: float = 0.0,
     st = lib().attn_kv_write(_dev(k_new, "k_new"), _dev(v_new, "v_new", dt), _dev(kcache, "kcache", dt),
                              _dev(vcache, "vcache", dt), _dev(pos0, "pos0", torch.int32), B, Tn, KV, hd,
                              Lmax, float(rope_base), _dtype(k_new), _stream(stream))
+    _check(st)
+
+
+def attn_decode_paged(q, kpages, vpages, block_table, seqlens, qpos, out=None, lse=None,
+                      workspace=None, *, rope_base: float = 0.0, window: int = 0, alibi_slopes=None,
+                      stream=None):
+    """q [B,H,hd] (not rotated) over page pools [num_pages,page_size,KV,hd] through
+    block_table [B,max_blocks] int32 -> out [B,H,hd]."""
+    B, H, hd = q.shape
+    num_pages, page_size, KV, _ = kpages.shape
+    max_blocks = block_table.shape[1]
+    dt = q.dtype
+    if out is None:
+        out = torch.empty_like(q)
+    need = attn_decode_workspace_size(B, H, KV, hd, max_blocks * page_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib().attn_decode_paged(_dev(q, "q"), _dev(kpages, "kpages", dt), _dev(vpages, "vpages", dt),
+                                 _dev(block_table, "block_table", torch.int32),
+                                 _dev(seqlens, "seqlens", torch.int32), _dev(qpos, "qpos", torch.int32),
+                                 _dev(out, "out", dt), _dev(lse, "lse", torch.float32), B, H, KV, hd,
+                                 page_size, num_pages, max_blocks, float(rope_base), int(window),
+                                 _slopes(alibi_slopes, H), _dtype(q), _dev(workspace, "workspace"),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st)
+    return out
+
+
+def attn_kv_write_paged(k_new, v_new, kpages, vpages, block_table, pos0, *, rope_base: float = 0.0,
+                        stream=None):
+    """Write k_new, v_new [B,Tn,KV,hd] into the page pools at slots pos0[b] .. pos0[b]+Tn-1."""
+    B, Tn, KV, hd = k_new.shape
+    num_pages, page_size = kpages.shape[:2]
+    max_blocks = block_table.shape[1]
+    dt = k_new.dtype
+    st = lib().attn_kv_write_paged(_dev(k_new, "k_new"), _dev(v_new, "v_new", dt),
+                                   _dev(kpages, "kpages", dt), _dev(vpages, "vpages", dt),
+                                   _dev(block_table, "block_table", torch.int32),
+                                   _dev(pos0, "pos0", torch.int32), B, Tn, KV, hd, page_size,
+                                   num_pages, max_blocks, float(rope_base), _dtype(k_new),
+                                   _stream(stream))
     _check(st)
 
 

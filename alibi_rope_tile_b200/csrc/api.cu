@@ -258,6 +258,80 @@ int attn_kv_append(const void* k_new, const void* v_new, void* kcache, void* vca
   return ok();
 }
 
+namespace {
+int check_pages(int page_size, int num_pages, int max_blocks) {
+  if (!(page_size == 8 || page_size == 16 || page_size == 32 || page_size == 64 || page_size == 128))
+    return fail(ATTN_ERR_ARG, "page_size must be 8, 16, 32, 64 or 128 (got %d)", page_size);
+  if (num_pages < 1 || max_blocks < 1) return fail(ATTN_ERR_ARG, "num_pages and max_blocks must be >= 1");
+  if ((long long)max_blocks * page_size >= (1LL << 24) || (long long)num_pages * page_size >= (1LL << 31))
+    return fail(ATTN_ERR_ARG, "max_blocks * page_size must be below 2^24");
+  return ATTN_OK;
+}
+}  // namespace
+
+int attn_decode_paged(const void* q, const void* kpages, const void* vpages, const int* block_table,
+                      const int* seqlens, const int* qpos, void* out, float* lse, int B, int H, int KV,
+                      int hd, int page_size, int num_pages, int max_blocks, float rope_base, int window,
+                      const float* alibi_slopes, int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  int st = check_common(H, KV, hd, dtype, rope_base);
+  if (st) return st;
+  if ((st = check_pages(page_size, num_pages, max_blocks))) return st;
+  if (!q || !kpages || !vpages || !block_table || !seqlens || !qpos || !out)
+    return fail(ATTN_ERR_ARG, "q, kpages, vpages, block_table, seqlens, qpos and out must not be NULL");
+  if (!aligned16(q) || !aligned16(kpages) || !aligned16(vpages) || !aligned16(out) ||
+      (lse && !aligned16(lse)) || (workspace && !aligned16(workspace)))
+    return fail(ATTN_ERR_ALIGN, "q, page pools, out, lse and workspace must be 16-byte aligned");
+  if (B < 1) return fail(ATTN_ERR_ARG, "B=%d must be >= 1", B);
+  if (window < 0) window = 0;
+  const int Lmax = max_blocks * page_size;
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.kcache = kpages; p.vcache = vpages; p.seqlens = seqlens; p.qpos = qpos;
+  p.out = out; p.lse = lse;
+  p.B = B; p.H = H; p.KV = KV; p.hd = hd; p.Lmax = Lmax; p.window = window;
+  p.block_table = block_table; p.page_size = page_size; p.num_pages = num_pages; p.max_blocks = max_blocks;
+  p.scale = (float)(1.0 / std::sqrt((double)hd));
+  p.rope = make_rope(hd, rope_base);
+  if ((st = make_alibi(H, alibi_slopes, &p.alibi))) return st;
+  if (!decode_tc_supported(p, dtype))
+    return fail(ATTN_ERR_UNSUPPORTED, "attn_decode_paged runs bf16 with hd 64 or 128 and H/KV <= 32");
+  const size_t need = decode_workspace_bytes(B, H, KV, hd, Lmax);
+  if (!workspace || ws_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "decode needs %zu bytes of workspace (got %zu)", need, ws_bytes);
+  int err = 0;
+  p.status = device_status(&err);
+  if (!p.status) return err;
+  cudaError_t e = launch_decode(p, dtype, workspace, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_decode_paged launch");
+  return ok();
+}
+
+int attn_kv_write_paged(const void* k_new, const void* v_new, void* kpages, void* vpages,
+                        const int* block_table, const int* pos0, int B, int Tn, int KV, int hd,
+                        int page_size, int num_pages, int max_blocks, float rope_base, int dtype,
+                        void* stream) {
+  int st = check_common(KV, KV, hd, dtype, rope_base);
+  if (st) return st;
+  if ((st = check_pages(page_size, num_pages, max_blocks))) return st;
+  if (!k_new || !v_new || !kpages || !vpages || !block_table || !pos0)
+    return fail(ATTN_ERR_ARG, "k_new, v_new, kpages, vpages, block_table and pos0 must not be NULL");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kpages) || !aligned16(vpages))
+    return fail(ATTN_ERR_ALIGN, "k_new, v_new and the page pools must be 16-byte aligned");
+  if (B < 1 || Tn < 1 || Tn > 65535) return fail(ATTN_ERR_ARG, "B >= 1 and 1 <= Tn <= 65535");
+  AppendParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.k_new = k_new; p.v_new = v_new; p.kcache = kpages; p.vcache = vpages; p.pos = pos0;
+  p.B = B; p.Tn = Tn; p.KV = KV; p.hd = hd; p.Lmax = max_blocks * page_size;
+  p.block_table = block_table; p.page_size = page_size; p.num_pages = num_pages; p.max_blocks = max_blocks;
+  p.rope = make_rope(hd, rope_base);
+  int err = 0;
+  p.status = device_status(&err);
+  if (!p.status) return err;
+  cudaError_t e = launch_kv_append(p, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_kv_write_paged launch");
+  return ok();
+}
+
 int attn_kv_write(const void* k_new, const void* v_new, void* kcache, void* vcache, const int* pos0,
                   int B, int Tn, int KV, int hd, int Lmax, float rope_base, int dtype, void* stream) {
   int st = check_common(KV, KV, hd, dtype, rope_base);

@@ -295,10 +295,19 @@ __global__ void kv_append_kernel(const AppendParams p) {
     return;
   }
   const int half = p.hd / 2;
+  size_t row = (size_t)b * p.Lmax + pos;  // row of the cache viewed as [rows][KV][hd]
+  if (p.block_table) {
+    const int page = p.block_table[(size_t)b * p.max_blocks + pos / p.page_size];
+    if (page < 0 || page >= p.num_pages) {
+      if (threadIdx.x == 0) flag_error(p.status, DEV_BAD_ARG);
+      return;
+    }
+    row = (size_t)page * p.page_size + pos % p.page_size;
+  }
   const T* kn = static_cast<const T*>(p.k_new) + ((size_t)b * p.Tn + t) * p.KV * p.hd;
   const T* vn = static_cast<const T*>(p.v_new) + ((size_t)b * p.Tn + t) * p.KV * p.hd;
-  T* kc = static_cast<T*>(p.kcache) + ((size_t)b * p.Lmax + pos) * p.KV * p.hd;
-  T* vc = static_cast<T*>(p.vcache) + ((size_t)b * p.Lmax + pos) * p.KV * p.hd;
+  T* kc = static_cast<T*>(p.kcache) + row * p.KV * p.hd;
+  T* vc = static_cast<T*>(p.vcache) + row * p.KV * p.hd;
   for (int idx = threadIdx.x; idx < p.KV * half; idx += blockDim.x) {
     const int g = idx / half, c = idx - g * half;
     const size_t off = (size_t)g * p.hd + 2 * c;

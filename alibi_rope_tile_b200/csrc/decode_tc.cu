@@ -171,9 +171,29 @@ __global__ void __launch_bounds__(THREADS, 2)
         const int st = u % NS, n = u / NS, j = jt0 + u / 2;
         if (!mbar_wait(kv_empty + st, (n & 1) ^ 1, abort_flag, p.status, a.wait_ns)) break;
         mbar_expect_tx(kv_full + st, C::KV_BYTES);
-        for (int kb = 0; kb < HD / 64; ++kb)
-          tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, (u & 1) ? &tmV : &tmK, kv_full + st,
-                      kb * 64, kvh, j * BN, b);
+        if (!p.block_table) {
+          for (int kb = 0; kb < HD / 64; ++kb)
+            tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, (u & 1) ? &tmV : &tmK, kv_full + st,
+                        kb * 64, kvh, j * BN, b);
+        } else {
+          // one box per page of the tile; a page past the sequence (or an invalid table
+          // entry) is fetched at an out-of-range page index, which reads zeros
+          const int ppt = BN / p.page_size;
+          for (int i = 0; i < ppt; ++i) {
+            const int blk = j * ppt + i;
+            int page = p.num_pages;
+            if (blk * p.page_size < L) {
+              const int e = p.block_table[(size_t)b * p.max_blocks + blk];
+              if (e >= 0 && e < p.num_pages)
+                page = e;
+              else
+                flag_error(p.status, DEV_BAD_ARG);
+            }
+            for (int kb = 0; kb < HD / 64; ++kb)
+              tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128 + i * p.page_size * 128, (u & 1) ? &tmV : &tmK,
+                          kv_full + st, kb * 64, kvh, 0, page);
+          }
+        }
       }
       // The loads of the last NS uses land before the CTA exits (immediate when the MMA
       // warp consumed them; after an abort they may still be in flight).
@@ -362,11 +382,29 @@ bool make_cache_map(CUtensorMap* map, const void* base, int B, int Lmax, int KV,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D map over a page pool [num_pages][page_size][KV][hd] with a box of one page x 64 features.
+bool make_page_map(CUtensorMap* map, const void* base, int num_pages, int page_size, int KV, int hd) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)KV, (cuuint64_t)page_size, (cuuint64_t)num_pages};
+  const cuuint64_t strides[3] = {(cuuint64_t)hd * 2, (cuuint64_t)KV * hd * 2,
+                                 (cuuint64_t)page_size * KV * hd * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)page_size, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int HD>
 cudaError_t launch_hd(const DecodeParams& p, int chunk, int nsplit, void* ws, cudaStream_t s) {
   CUtensorMap mk, mv;
-  if (!make_cache_map(&mk, p.kcache, p.B, p.Lmax, p.KV, HD) || !make_cache_map(&mv, p.vcache, p.B, p.Lmax, p.KV, HD))
-    return cudaErrorInvalidValue;
+  const bool ok = p.block_table
+                      ? make_page_map(&mk, p.kcache, p.num_pages, p.page_size, p.KV, HD) &&
+                            make_page_map(&mv, p.vcache, p.num_pages, p.page_size, p.KV, HD)
+                      : make_cache_map(&mk, p.kcache, p.B, p.Lmax, p.KV, HD) &&
+                            make_cache_map(&mv, p.vcache, p.B, p.Lmax, p.KV, HD);
+  if (!ok) return cudaErrorInvalidValue;
   DecArgs a;
   a.p = p;
   a.chunk = chunk;

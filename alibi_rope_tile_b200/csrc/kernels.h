@@ -52,6 +52,11 @@ struct DecodeParams {
   int* status;
   RopeFreqs rope;
   Alibi alibi;
+  // Paged cache (block_table != nullptr): kcache, vcache are page pools
+  // [num_pages][page_size][KV][hd]; slot j of sequence b is row j % page_size of page
+  // block_table[b * max_blocks + j / page_size]; Lmax = max_blocks * page_size.
+  const int* block_table;
+  int page_size, num_pages, max_blocks;
 };
 
 // Split-KV geometry: keys per split and number of splits for these sizes.
@@ -72,6 +77,9 @@ struct AppendParams {
   int B, Tn, KV, hd, Lmax;  // Tn rows per sequence
   int* status;
   RopeFreqs rope;
+  // paged cache, as in DecodeParams (block_table == nullptr: contiguous [B][Lmax][KV][hd])
+  const int* block_table;
+  int page_size, num_pages, max_blocks;
 };
 cudaError_t launch_kv_append(const AppendParams& p, int dtype, cudaStream_t s);
 

@@ -190,6 +190,35 @@ int attn_kv_write(const void* k_new, const void* v_new, void* kcache, void* vcac
                   int B, int Tn, int KV, int hd, int Lmax, float rope_base, int dtype, void* stream);
 
 /*
+ * attn_decode_paged -- attn_decode over a paged KV cache (the block-table layout of the
+ * PagedAttention the pages mention for serving): the caches are page pools
+ * kpages, vpages [num_pages, page_size, KV, hd]; slot j of sequence b is row j % page_size
+ * of page block_table[b * max_blocks + j / page_size] (block_table: [B, max_blocks] int32,
+ * device). page_size in {8, 16, 32, 64, 128}; seqlens[b] <= max_blocks * page_size. Entries
+ * the sequence does not reach are not read. A table entry outside [0, num_pages) is
+ * recorded as ATTN_ERR_DEVICE_ARG and its page reads as zeros. Everything else (q rotated
+ * at qpos[b], window, ALiBi, outputs, workspace = attn_decode_workspace_size(B, H, KV, hd,
+ * max_blocks * page_size)) is as attn_decode. Runs the tensor-core split pass: bf16, hd 64
+ * or 128, H/KV <= 32; anything else returns ATTN_ERR_UNSUPPORTED.
+ */
+int attn_decode_paged(const void* q, const void* kpages, const void* vpages, const int* block_table,
+                      const int* seqlens, const int* qpos, void* out, float* lse, int B, int H, int KV,
+                      int hd, int page_size, int num_pages, int max_blocks, float rope_base, int window,
+                      const float* alibi_slopes, int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * attn_kv_write_paged -- attn_kv_write into page pools: row t of sequence b goes to slot
+ * pos0[b] + t, i.e. row (pos0[b] + t) % page_size of page block_table[b * max_blocks +
+ * (pos0[b] + t) / page_size], its key rotated at that position. A slot past
+ * max_blocks * page_size or a table entry outside [0, num_pages) is recorded as
+ * ATTN_ERR_DEVICE_ARG and that row is skipped.
+ */
+int attn_kv_write_paged(const void* k_new, const void* v_new, void* kpages, void* vpages,
+                        const int* block_table, const int* pos0, int B, int Tn, int KV, int hd,
+                        int page_size, int num_pages, int max_blocks, float rope_base, int dtype,
+                        void* stream);
+
+/*
  * attn_block_workspace_size -- bytes of device scratch attn_block needs (the q, k, v and
  * context activations). Returns 0 on invalid sizes.
  */

@@ -31,7 +31,7 @@ def declared_functions():
 def test_header_declares_entry_points():
     names = declared_functions()
     for must in ("attn_prefill", "attn_decode", "attn_block", "attn_kv_append",
-                 "attn_prefill_chunk", "attn_kv_write",
+                 "attn_prefill_chunk", "attn_kv_write", "attn_decode_paged", "attn_kv_write_paged",
                  "attn_decode_workspace_size", "attn_block_workspace_size", "attn_alibi_slopes",
                  "attn_sync_status", "attn_last_error", "attn_version"):
         assert must in names
@@ -141,6 +141,29 @@ def test_chunk_and_kv_write_argument_errors(lib):
     assert write(Tn=0) == -1
     assert write(Tn=70000) == -1
     assert write(hd=7) == -1
+
+
+def test_paged_argument_errors(lib):
+    P = 0x1000
+    def dec(**kw):
+        a = dict(B=2, H=8, KV=2, hd=128, ps=16, npages=64, mb=8, dtype=1, table=P)
+        a.update(kw)
+        return lib.attn_decode_paged(P, P, P, a["table"], P, P, P, None, a["B"], a["H"], a["KV"], a["hd"],
+                                     a["ps"], a["npages"], a["mb"], 10000.0, 0, None, a["dtype"], P,
+                                     1 << 30, None)
+    assert dec(ps=24) == -1          # page size not a power of two dividing 128
+    assert dec(ps=256) == -1
+    assert dec(npages=0) == -1
+    assert dec(table=None) == -1
+    assert dec(dtype=0) == -3        # fp32 has no paged kernel
+    assert dec(hd=32) == -3
+    def write(**kw):
+        a = dict(Tn=4, ps=64)
+        a.update(kw)
+        return lib.attn_kv_write_paged(P, P, P, P, P, P, 2, a["Tn"], 2, 64, a["ps"], 8, 4, 10000.0, 1,
+                                       None)
+    assert write(Tn=0) == -1
+    assert write(ps=4) == -1
 
 
 def test_binding_requires_cuda_tensors(lib):
