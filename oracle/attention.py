@@ -196,6 +196,61 @@ def decode_paged(q, kpages, vpages, block_table, seqlens, qpos, *, page_size: in
     return decode(q, kc, vc, seqlens, qpos, rope_base=rope_base, window=window, slopes=slopes)
 
 
+def latent_decode(q, ccache, W_uk, W_uv, seqlens, qpos, *, window: int = 0, slopes=None):
+    """Decode over a latent cache, unfolded ([LAB] exercise 5, latent attention): each cached
+    token holds a latent c_j [dc]; head h's key and value are c_j W_uk[h] and c_j W_uv[h]
+    (W_uk, W_uv [H, dc, hd]). No rotary embedding on this path (a position rotation between c
+    and W_uk would not fold into the query). q [B,H,hd]; ccache [B,Lmax,dc].
+    Returns out [B,H,hd], lse [B,H]."""
+    q, c = _f64(q), _f64(ccache)
+    W_uk, W_uv = _f64(W_uk), _f64(W_uv)
+    B, H, hd = q.shape
+    out = np.zeros((B, H, hd))
+    lse = np.full((B, H), -np.inf)
+    for b in range(B):
+        L, p = int(seqlens[b]), int(qpos[b])
+        if L == 0:
+            continue
+        j = np.arange(L)
+        ok = (p - j) < window if window > 0 else np.ones(L, dtype=bool)
+        for h in range(H):
+            k = c[b, :L] @ W_uk[h]                             # [L, hd]
+            v = c[b, :L] @ W_uv[h]
+            s = k @ q[b, h] / np.sqrt(hd)
+            if slopes is not None:
+                s = s - float(slopes[h]) * np.abs(p - j)
+            w, row_lse = _masked_softmax_rows(s[None, :], ok[None, :])
+            lse[b, h] = row_lse[0]
+            out[b, h] = (w @ v)[0]
+    return out, lse
+
+
+def latent_decode_folded(q, ccache, W_uk, W_uv, seqlens, qpos, *, window: int = 0, slopes=None):
+    """The same with the key up-projection folded into the query ([LAB] exercise 5): scores
+    (W_uk[h] q_h) . c_j / sqrt(hd) against the latent itself, and the value up-projection
+    applied once to the weighted latent sum. Returns out [B,H,hd], lse [B,H]."""
+    q, c = _f64(q), _f64(ccache)
+    W_uk, W_uv = _f64(W_uk), _f64(W_uv)
+    B, H, hd = q.shape
+    out = np.zeros((B, H, hd))
+    lse = np.full((B, H), -np.inf)
+    for b in range(B):
+        L, p = int(seqlens[b]), int(qpos[b])
+        if L == 0:
+            continue
+        j = np.arange(L)
+        ok = (p - j) < window if window > 0 else np.ones(L, dtype=bool)
+        for h in range(H):
+            qlat = W_uk[h] @ q[b, h]                           # [dc]
+            s = c[b, :L] @ qlat / np.sqrt(hd)
+            if slopes is not None:
+                s = s - float(slopes[h]) * np.abs(p - j)
+            w, row_lse = _masked_softmax_rows(s[None, :], ok[None, :])
+            lse[b, h] = row_lse[0]
+            out[b, h] = (w @ c[b, :L])[0] @ W_uv[h]
+    return out, lse
+
+
 def kv_write(k_new, v_new, kcache, vcache, pos0, *, rope_base: float = 0.0):
     """Write a chunk of keys and values into the cache ([XF5] "KV caching"), in fp64.
 

@@ -48,6 +48,8 @@ MUTANTS = {
     "paged_row_index": ("return pages[page, j % page_size]", "return pages[page, (j + 1) % page_size]"),
     "paged_block_index": ("page = np.asarray(block_table)[b][j // page_size]",
                           "page = np.asarray(block_table)[b][j % page_size]"),
+    "latent_scale_by_dc": ("s = k @ q[b, h] / np.sqrt(hd)", "s = k @ q[b, h] / np.sqrt(c.shape[2])"),
+    "latent_value_projection": ("v = c[b, :L] @ W_uv[h]", "v = c[b, :L] @ W_uk[h]"),
     "block_wq_transposed": ("q = (x @ Wq).reshape(B, T, H, hd)", "q = (x @ Wq.T).reshape(B, T, H, hd)"),
     "block_head_split": ("q = (x @ Wq).reshape(B, T, H, hd)",
                          "q = (x @ Wq).reshape(B, T, hd, H).swapaxes(2, 3)"),
@@ -65,6 +67,7 @@ PIN_TESTS = [
     ("test_chunk_brute_force_and_cache_route", False),
     ("test_chunk_of_one_row_is_a_decode_step_and_empty_cache", False),
     ("test_paged_decode_brute_force_and_page_order", False),
+    ("test_latent_fold_leaves_scores_and_outputs_unchanged", False),
 ]
 
 

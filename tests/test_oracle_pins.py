@@ -350,6 +350,31 @@ def test_paged_decode_brute_force_and_page_order():
         assert np.all(out[1] == 0.0) and np.all(np.isneginf(lse[1]))
 
 
+def test_latent_fold_leaves_scores_and_outputs_unchanged():
+    """[LAB] exercise 5: folding the key up-projection into the query leaves the scores (and so
+    the outputs) unchanged; and the latent decode equals a plain decode over the keys and values
+    the up-projections produce, materialised as an H-head cache."""
+    B, H, hd, dc, Lmax = 3, 4, 8, 5, 11
+    q, c = _rand((B, H, hd), 110), _rand((B, Lmax, dc), 111)
+    W_uk, W_uv = _rand((H, dc, hd), 112) / np.sqrt(dc), _rand((H, dc, hd), 113) / np.sqrt(dc)
+    seqlens, qpos = [7, 0, 11], [7, 0, 10]
+    for window, slopes in [(0, None), (4, A.alibi_slopes(H))]:
+        o1, l1 = A.latent_decode(q, c, W_uk, W_uv, seqlens, qpos, window=window, slopes=slopes)
+        o2, l2 = A.latent_decode_folded(q, c, W_uk, W_uv, seqlens, qpos, window=window, slopes=slopes)
+        np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l2, l1, rtol=0, atol=1e-13)
+        kc = np.einsum("bld,hde->blhe", c, W_uk)               # [B, Lmax, H, hd]
+        vc = np.einsum("bld,hde->blhe", c, W_uv)
+        o3, l3 = A.decode(q, kc, vc, seqlens, qpos, window=window, slopes=slopes)
+        np.testing.assert_allclose(o3, o1, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l3, l1, rtol=0, atol=1e-13)
+        assert np.all(o1[1] == 0.0) and np.all(np.isneginf(l1[1]))
+    # the fold at the level of one score, written out
+    s_unfolded = q[0, 2] @ (c[0, 3] @ W_uk[2])
+    s_folded = (W_uk[2] @ q[0, 2]) @ c[0, 3]
+    assert abs(s_unfolded - s_folded) < 1e-13
+
+
 # ----------------------------------------------------------------------------- workloads
 def test_workload_pair_counts():
     """FLOP counts used by the bench: causal pairs T(T+1)/2, windowed pairs sum min(i+1, W)."""
