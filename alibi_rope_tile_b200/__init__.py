@@ -41,6 +41,9 @@ SIGNATURES = {
     "attn_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _FP,
                                _I, _P, _S, _P]),
     "attn_kv_write_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_decode_latent_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "attn_decode_latent": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _FP, _I, _P, _S,
+                                _P]),
     "attn_block_workspace_size": (_S, [_I, _I, _I, _I, _I, _I, _I]),
     "attn_block": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _L, _F, _I, _I, _FP, _I,
                         _P, _S, _P]),
@@ -255,6 +258,28 @@ def attn_kv_write_paged(k_new, v_new, kpages, vpages, block_table, pos0, *, rope
                                    num_pages, max_blocks, float(rope_base), _dtype(k_new),
                                    _stream(stream))
     _check(st)
+
+
+def attn_decode_latent(q, ccache, W_uk, W_uv, seqlens, qpos, out=None, lse=None, workspace=None, *,
+                       window: int = 0, alibi_slopes=None, stream=None):
+    """q [B,H,hd] over a latent cache ccache [B,Lmax,dc] with per-head up-projections
+    W_uk, W_uv [H,dc,hd] -> out [B,H,hd] (the key up-projection folded into the query)."""
+    B, H, hd = q.shape
+    _, Lmax, dc = ccache.shape
+    dt = q.dtype
+    if out is None:
+        out = torch.empty_like(q)
+    need = int(lib().attn_decode_latent_workspace_size(B, H, hd, dc, Lmax))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib().attn_decode_latent(_dev(q, "q"), _dev(ccache, "ccache", dt), _dev(W_uk, "W_uk", dt),
+                                  _dev(W_uv, "W_uv", dt), _dev(seqlens, "seqlens", torch.int32),
+                                  _dev(qpos, "qpos", torch.int32), _dev(out, "out", dt),
+                                  _dev(lse, "lse", torch.float32), B, H, hd, dc, Lmax, int(window),
+                                  _slopes(alibi_slopes, H), _dtype(q), _dev(workspace, "workspace"),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st)
+    return out
 
 
 def attn_kv_append(k_new, v_new, kcache, vcache, pos, *, rope_base: float = 0.0, stream=None):

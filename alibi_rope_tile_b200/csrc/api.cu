@@ -332,6 +332,60 @@ int attn_kv_write_paged(const void* k_new, const void* v_new, void* kpages, void
   return ok();
 }
 
+namespace {
+size_t r256(size_t x) { return (x + 255) & ~(size_t)255; }
+}  // namespace
+
+size_t attn_decode_latent_workspace_size(int B, int H, int hd, int dc, int Lmax) {
+  if (B < 1 || H < 1 || hd < 2 || (dc != 64 && dc != 128) || Lmax < 1) return 0;
+  const size_t vec = r256((size_t)B * H * dc * 2);  // q' and the latent output, bf16
+  return 2 * vec + decode_workspace_bytes(B, H, 1, dc, Lmax);
+}
+
+int attn_decode_latent(const void* q, const void* ccache, const void* W_uk, const void* W_uv,
+                       const int* seqlens, const int* qpos, void* out, float* lse, int B, int H, int hd,
+                       int dc, int Lmax, int window, const float* alibi_slopes, int dtype, void* workspace,
+                       size_t ws_bytes, void* stream) {
+  int st = check_common(H, 1, hd, dtype, 0.f);
+  if (st) return st;
+  if (!q || !ccache || !W_uk || !W_uv || !seqlens || !qpos || !out)
+    return fail(ATTN_ERR_ARG, "q, ccache, W_uk, W_uv, seqlens, qpos and out must not be NULL");
+  if (!aligned16(q) || !aligned16(ccache) || !aligned16(W_uk) || !aligned16(W_uv) || !aligned16(out) ||
+      (lse && !aligned16(lse)) || (workspace && !aligned16(workspace)))
+    return fail(ATTN_ERR_ALIGN, "q, ccache, weights, out, lse and workspace must be 16-byte aligned");
+  if (B < 1 || Lmax < 1 || Lmax >= (1 << 24)) return fail(ATTN_ERR_ARG, "B >= 1 and 1 <= Lmax < 2^24");
+  if (dtype != ATTN_BF16 || (dc != 64 && dc != 128) || H > 32)
+    return fail(ATTN_ERR_UNSUPPORTED, "attn_decode_latent runs bf16 with dc 64 or 128 and H <= 32");
+  if (window < 0) window = 0;
+  const size_t need = attn_decode_latent_workspace_size(B, H, hd, dc, Lmax);
+  if (!workspace || ws_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "latent decode needs %zu bytes of workspace (got %zu)", need, ws_bytes);
+  char* ws = static_cast<char*>(workspace);
+  const size_t vec = r256((size_t)B * H * dc * 2);
+  void* qlat = ws;
+  void* olat = ws + vec;
+  void* dws = ws + 2 * vec;
+
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = qlat; p.kcache = ccache; p.vcache = ccache;  // keys and values are the same latents
+  p.seqlens = seqlens; p.qpos = qpos; p.out = olat; p.lse = lse;
+  p.B = B; p.H = H; p.KV = 1; p.hd = dc; p.Lmax = Lmax; p.window = window;
+  p.scale = (float)(1.0 / std::sqrt((double)hd));  // the scores are q . k of head dimension hd
+  p.rope = make_rope(dc, 0.f);                      // no rotation on the latent path
+  if ((st = make_alibi(H, alibi_slopes, &p.alibi))) return st;
+  if (!decode_tc_supported(p, dtype)) return fail(ATTN_ERR_UNSUPPORTED, "latent decode kernel unavailable");
+  int err = 0;
+  p.status = device_status(&err);
+  if (!p.status) return err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_head_proj(true, q, W_uk, qlat, B, H, dc, hd, s);
+  if (e == cudaSuccess) e = launch_decode(p, dtype, dws, s);
+  if (e == cudaSuccess) e = launch_head_proj(false, olat, W_uv, out, B, H, dc, hd, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attn_decode_latent launch");
+  return ok();
+}
+
 int attn_kv_write(const void* k_new, const void* v_new, void* kcache, void* vcache, const int* pos0,
                   int B, int Tn, int KV, int hd, int Lmax, float rope_base, int dtype, void* stream) {
   int st = check_common(KV, KV, hd, dtype, rope_base);

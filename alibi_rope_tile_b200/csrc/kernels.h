@@ -83,6 +83,11 @@ struct AppendParams {
 };
 cudaError_t launch_kv_append(const AppendParams& p, int dtype, cudaStream_t s);
 
+// Latent attention's per-head projections (bf16): fold: y[b,h,:] = W[h] x[b,h,:] (hd -> dc);
+// otherwise y[b,h,:] = x[b,h,:] W[h] (dc -> hd). W is [H][dc][hd].
+cudaError_t launch_head_proj(bool fold, const void* x, const void* W, void* y, int B, int H, int dc, int hd,
+                             cudaStream_t s);
+
 // C[M,N] = A[M,K] @ W[K,N], row-major, fp32 accumulation, output in the input dtype.
 cudaError_t launch_gemm_simt(const void* A, const void* W, void* C, int M, int N, int K, int dtype,
                              cudaStream_t s);

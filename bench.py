@@ -49,12 +49,15 @@ DECODE = workloads.DECODE_GQA
 DECODE_MQA = workloads.DECODE_MQA
 BLOCK = workloads.GQA_BLOCK
 CHUNK = workloads.GQA_CHUNK
+LATENT = workloads.LATENT_DECODE
 # Algorithmic bytes and launches, stated once (see the design notes):
 #   decode bytes = cache rows read (K and V) + q + out; prefill FLOPs = PREFILL.flops.
 PREFILL_LAUNCHES = 1
 DECODE_LAUNCHES = 2       # split pass + merge, per decode workload
+PAGE_SIZE = 16            # rows per page of the paged decode (the KV=8 decode workload, pages shuffled)
 BLOCK_LAUNCHES = 5        # three projection GEMMs, the prefill, the output GEMM
 CHUNK_LAUNCHES = 1
+LATENT_LAUNCHES = 4       # the fold, the split pass, the merge, the value up-projection
 
 
 def peaks():
@@ -247,6 +250,8 @@ def run_ours(args, rank, world):
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
     dout = torch.empty_like(dq)
     decs = []
+    paged = None
+    lat = None
     if do_d:
         for dw in (DECODE, DECODE_MQA):
             hq, hkc, hvc, hsl, hqp = workloads.decode_inputs(dw)
@@ -256,7 +261,38 @@ def run_ours(args, rank, world):
                 out=torch.empty(hq.shape, dtype=hq.dtype, device="cuda"),
                 ws=torch.empty(art.attn_decode_workspace_size(dw.B, dw.H, dw.KV, dw.hd, dw.Lmax),
                                dtype=torch.uint8, device="cuda")))
+            if dw is DECODE:
+                # the same cache as a shuffled pool of 16-row pages behind a block table
+                mb = dw.Lmax // PAGE_SIZE
+                need = [mb] * dw.B  # every slot has a page (those past a length are never read)
+                g = torch.Generator().manual_seed(dw.seed + 100)
+                order = torch.randperm(sum(need), generator=g)
+                table = torch.full((dw.B, mb), -1, dtype=torch.int32)
+                at = 0
+                for b in range(dw.B):
+                    table[b, :need[b]] = order[at:at + need[b]].to(torch.int32)
+                    at += need[b]
+                kp = torch.zeros(sum(need), PAGE_SIZE, dw.KV, dw.hd, dtype=hkc.dtype, device="cuda")
+                vp = torch.zeros_like(kp)
+                dtab = table.cuda()
+                zero = torch.zeros(dw.B, dtype=torch.int32, device="cuda")
+                art.attn_kv_write_paged(decs[-1]["kc"], decs[-1]["vc"], kp, vp, dtab, zero, rope_base=0.0)
+                paged = dict(w=dw, bytes=decs[-1]["bytes"], q=decs[-1]["q"], sl=decs[-1]["sl"],
+                             qp=decs[-1]["qp"], kp=kp, vp=vp, table=dtab,
+                             out=torch.empty_like(decs[-1]["out"]),
+                             ws=torch.empty_like(decs[-1]["ws"]))
             del hkc, hvc
+        lw = LATENT
+        lq, lc, luk, luv, lsl = workloads.latent_inputs(lw)
+        lat = dict(w=lw, hq=lq, q=lq.cuda(), c=lc.cuda(), uk=luk.cuda(), uv=luv.cuda(), sl=lsl.cuda(),
+                   out=torch.empty(lq.shape, dtype=lq.dtype, device="cuda"),
+                   ws=torch.empty(int(art.lib().attn_decode_latent_workspace_size(lw.B, lw.H, lw.hd, lw.dc,
+                                                                                  lw.Lmax)),
+                                  dtype=torch.uint8, device="cuda"),
+                   # algorithmic bytes: each latent row read once, q and out, both weights
+                   bytes=int(lsl.sum()) * lw.dc * 2 + 2 * lw.B * lw.H * lw.hd * 2
+                   + 2 * lw.H * lw.dc * lw.hd * 2)
+        del lc
     blk = None
     if do_b:
         bw = BLOCK
@@ -297,6 +333,17 @@ def run_ours(args, rank, world):
                            workspace=blk["ws"], H=bw.H, KV=bw.KV, rope_base=bw.rope_base,
                            causal=bw.causal, window=bw.window)
 
+    def decode_paged():
+        if paged is not None:
+            art.attn_decode_paged(paged["q"], paged["kp"], paged["vp"], paged["table"], paged["sl"],
+                                  paged["qp"], paged["out"], workspace=paged["ws"],
+                                  rope_base=paged["w"].rope_base)
+
+    def decode_latent():
+        if lat is not None:
+            art.attn_decode_latent(lat["q"], lat["c"], lat["uk"], lat["uv"], lat["sl"], lat["sl"], lat["out"],
+                                   workspace=lat["ws"])
+
     def chunk():
         if chk is not None:
             art.attn_prefill_chunk(chk["q"], chk["kc"], chk["vc"], chk["sl"], chk["qp"], chk["out"],
@@ -309,10 +356,12 @@ def run_ours(args, rank, world):
             decode(d)
         block()
         chunk()
+        decode_paged()
+        decode_latent()
     torch.cuda.synchronize()
     art.attn_sync_status()
 
-    nev = 2 + 2 * len(decs) + 4
+    nev = 2 + 2 * len(decs) + 8
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
@@ -332,12 +381,20 @@ def run_ours(args, rank, world):
             decode(d)
             ev[s_][3 + 2 * n].record(stream)
         flush.zero_()
-        ev[s_][nev - 4].record(stream)
+        ev[s_][nev - 8].record(stream)
+        decode_latent()
+        ev[s_][nev - 7].record(stream)
+        flush.zero_()
+        ev[s_][nev - 6].record(stream)
         block()
+        ev[s_][nev - 5].record(stream)
+        flush.zero_()
+        ev[s_][nev - 4].record(stream)
+        chunk()
         ev[s_][nev - 3].record(stream)
         flush.zero_()
         ev[s_][nev - 2].record(stream)
-        chunk()
+        decode_paged()
         ev[s_][nev - 1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -348,9 +405,13 @@ def run_ours(args, rank, world):
     d_tot = [max(1e-9, max_over_ranks(sum(ev[s_][2 + 2 * n].elapsed_time(ev[s_][3 + 2 * n])
                                           for s_ in range(args.steps)), world))
              for n in range(len(decs))]
-    b_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 4].elapsed_time(ev[s_][nev - 3])
+    b_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 6].elapsed_time(ev[s_][nev - 5])
                                          for s_ in range(args.steps)), world))
-    c_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 2].elapsed_time(ev[s_][nev - 1])
+    c_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 4].elapsed_time(ev[s_][nev - 3])
+                                         for s_ in range(args.steps)), world))
+    g_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 2].elapsed_time(ev[s_][nev - 1])
+                                         for s_ in range(args.steps)), world))
+    l_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 8].elapsed_time(ev[s_][nev - 7])
                                          for s_ in range(args.steps)), world))
     region_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
 
@@ -363,6 +424,11 @@ def run_ours(args, rank, world):
     if blk is not None:
         hbx = blk["hx"].pin_memory()
         hbo = torch.empty(blk["hx"].shape, dtype=blk["hx"].dtype).pin_memory()
+    if paged is not None:
+        hpo = torch.empty(paged["out"].shape, dtype=paged["out"].dtype).pin_memory()
+    if lat is not None:
+        hlq = lat["hq"].pin_memory()
+        hlo = torch.empty(lat["hq"].shape, dtype=lat["hq"].dtype).pin_memory()
     if chk is not None:
         hcq_p = chk["hq"].pin_memory()
         hco = torch.empty(chk["hq"].shape, dtype=chk["hq"].dtype).pin_memory()
@@ -386,6 +452,14 @@ def run_ours(args, rank, world):
             chk["q"].copy_(hcq_p, non_blocking=True)
             chunk()
             hco.copy_(chk["out"], non_blocking=True)
+        if paged is not None:
+            # its query tensor is the KV=8 decode's, already copied in above
+            decode_paged()
+            hpo.copy_(paged["out"], non_blocking=True)
+        if lat is not None:
+            lat["q"].copy_(hlq, non_blocking=True)
+            decode_latent()
+            hlo.copy_(lat["out"], non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -436,6 +510,25 @@ def run_ours(args, rank, world):
         "projections_derived": {"tflops": proj_tflops, "ms": proj_ms,
                                 "frac": proj_tflops / pk["bf16_tflops"],
                                 "how": "block time minus the prefill time of the same shape"}}
+    if paged is not None:
+        ms = g_tot / args.steps
+        gbs = paged["bytes"] / (ms * 1e-3) / 1e9
+        decode_out[paged["w"].name + f"_paged{PAGE_SIZE}"] = {
+            "value": aggregate_rate(paged["bytes"] * args.steps, world, g_tot) / 1e9, "unit": "GB/s",
+            "ms": ms, "bytes": paged["bytes"], "page_size": PAGE_SIZE, "pages": "shuffled",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{pk.get('source')} copy"}}
+    if lat is not None:
+        ms = l_tot / args.steps
+        gbs = lat["bytes"] / (ms * 1e-3) / 1e9
+        decode_out[lat["w"].name] = {
+            "value": aggregate_rate(lat["bytes"] * args.steps, world, l_tot) / 1e9, "unit": "GB/s",
+            "ms": ms, "bytes": lat["bytes"],
+            "note": "each latent tile is fetched twice (as keys and as values); bytes count it once",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{pk.get('source')} copy"}}
     cw = chk["w"]
     c_ms = c_tot / args.steps
     c_tflops = cw.flops / (c_ms * 1e-3) / 1e12
@@ -452,6 +545,11 @@ def run_ours(args, rank, world):
         d["hq"].numel() * d["hq"].element_size() for d in decs) + xb + cb
     d2h = q.numel() * q.element_size() + sum(
         d["hq"].numel() * d["hq"].element_size() for d in decs) + xb + cb
+    if paged is not None:
+        d2h += paged["out"].numel() * paged["out"].element_size()
+    if lat is not None:
+        h2d += lat["hq"].numel() * lat["hq"].element_size()
+        d2h += lat["hq"].numel() * lat["hq"].element_size()
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         val, dt, sample = oracle_sample_tflops()
@@ -460,7 +558,8 @@ def run_ours(args, rank, world):
     line = {
         "metric": METRIC, "value": aggregate_rate(flops_step * args.steps, world, p_tot) / 1e12,
         "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": (p_tot + sum(d_tot) + b_tot + c_tot) / args.steps, "higher_is_better": True,
+        "ms_per_step": (p_tot + sum(d_tot) + b_tot + c_tot + g_tot + l_tot) / args.steps,
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "decode_workloads": [d["w"].name for d in decs],
                    "block_workload": bw.name, "chunk_workload": cw.name,
@@ -480,8 +579,8 @@ def run_ours(args, rank, world):
                 "note": "prefill FLOPs over the whole step incl. copies, both decodes, the block "
                         "(block weights resident; x in, out back) and the chunk (cache resident; "
                         "its queries in, out back)"},
-        "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES * len(decs) + BLOCK_LAUNCHES
-                                      + CHUNK_LAUNCHES),
+        "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES * (len(decs) + 1) + BLOCK_LAUNCHES
+                                      + CHUNK_LAUNCHES + LATENT_LAUNCHES),
         "clocks": clk,
         "cpu_baseline": cpu,
     }

@@ -207,6 +207,26 @@ int attn_decode_paged(const void* q, const void* kpages, const void* vpages, con
                       const float* alibi_slopes, int dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * attn_decode_latent -- one decode step of latent attention ([LAB] exercise 5): every cached
+ * token holds a latent c_j of dc numbers, and query head h's key and value are c_j W_uk[h]
+ * and c_j W_uv[h] (W_uk, W_uv: [H, dc, hd] bf16, device). The key up-projection is folded
+ * into the query (q'_h = W_uk[h] q_h), the decode runs over the latents themselves as one
+ * key/value head of dimension dc (score q'_h . c_j / sqrt(hd)), and the value up-projection
+ * is applied once to the weighted latent sum: the result equals attention over the
+ * up-projected keys and values. No rotary embedding on this path (a position rotation
+ * between c and W_uk does not fold into the query); window and ALiBi as attn_decode.
+ * q: [B,H,hd]; ccache: [B,Lmax,dc] (device); out: [B,H,hd]; lse: [B,H] or NULL.
+ * workspace: attn_decode_latent_workspace_size(B,H,hd,dc,Lmax) bytes (device, caller-owned).
+ * bf16 with dc in {64, 128} and H <= 32; anything else returns ATTN_ERR_UNSUPPORTED.
+ * Four launches: the fold, the split pass, the merge, the value up-projection.
+ */
+size_t attn_decode_latent_workspace_size(int B, int H, int hd, int dc, int Lmax);
+int attn_decode_latent(const void* q, const void* ccache, const void* W_uk, const void* W_uv,
+                       const int* seqlens, const int* qpos, void* out, float* lse, int B, int H, int hd,
+                       int dc, int Lmax, int window, const float* alibi_slopes, int dtype, void* workspace,
+                       size_t ws_bytes, void* stream);
+
+/*
  * attn_kv_write_paged -- attn_kv_write into page pools: row t of sequence b goes to slot
  * pos0[b] + t, i.e. row (pos0[b] + t) % page_size of page block_table[b * max_blocks +
  * (pos0[b] + t) / page_size], its key rotated at that position. A slot past

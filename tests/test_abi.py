@@ -32,6 +32,7 @@ def test_header_declares_entry_points():
     names = declared_functions()
     for must in ("attn_prefill", "attn_decode", "attn_block", "attn_kv_append",
                  "attn_prefill_chunk", "attn_kv_write", "attn_decode_paged", "attn_kv_write_paged",
+                 "attn_decode_latent",
                  "attn_decode_workspace_size", "attn_block_workspace_size", "attn_alibi_slopes",
                  "attn_sync_status", "attn_last_error", "attn_version"):
         assert must in names
@@ -164,6 +165,21 @@ def test_paged_argument_errors(lib):
                                        None)
     assert write(Tn=0) == -1
     assert write(ps=4) == -1
+
+
+def test_latent_argument_errors(lib):
+    P = 0x1000
+    def lat(**kw):
+        a = dict(H=32, hd=128, dc=128, dtype=1, W=P)
+        a.update(kw)
+        return lib.attn_decode_latent(P, P, a["W"], P, P, P, P, None, 4, a["H"], a["hd"], a["dc"], 256, 0,
+                                      None, a["dtype"], P, 1 << 30, None)
+    assert lat(W=None) == -1
+    assert lat(dc=96) == -3          # the latent decode runs dc 64 or 128
+    assert lat(H=64) == -3           # one key/value head serves at most 32 query heads here
+    assert lat(dtype=0) == -3
+    assert lib.attn_decode_latent_workspace_size(4, 32, 128, 96, 256) == 0
+    assert lib.attn_decode_latent_workspace_size(4, 32, 128, 64, 256) > 0
 
 
 def test_binding_requires_cuda_tensors(lib):

@@ -132,6 +132,21 @@ class Chunk:
         return 4 * self.B * self.H * self.hd * self.allowed_pairs
 
 
+@dataclasses.dataclass(frozen=True)
+class Latent:
+    """A latent-attention decode step: a cache of dc-number latents per token and per-head
+    up-projections [H, dc, hd]; cache lengths uniform in [len_lo, len_hi]."""
+    name: str
+    B: int
+    H: int
+    hd: int
+    dc: int
+    Lmax: int
+    len_lo: int
+    len_hi: int
+    seed: int = 0
+
+
 # The workloads of this library, named by what they are.
 TINY_BLOCK = Block("tiny_block_fp32_T6_d32_H4_KV2_hd8", B=1, T=6, d=32, H=4, KV=2, hd=8,
                    rope_base=10000.0, causal=True, seed=0)
@@ -147,6 +162,8 @@ DECODE_GQA = Decode("decode_bf16_B64_H32_KV8_hd128_L1024-8192", B=64, H=32, KV=8
                     Lmax=8192, len_lo=1024, len_hi=8192, seed=4)
 DECODE_MQA = Decode("decode_bf16_B64_H32_KV1_hd128_L1024-8192", B=64, H=32, KV=1, hd=128,
                     Lmax=8192, len_lo=1024, len_hi=8192, seed=5)
+LATENT_DECODE = Latent("latent_decode_bf16_B64_H32_hd128_dc128_L1024-8192", B=64, H=32, hd=128, dc=128,
+                       Lmax=8192, len_lo=1024, len_hi=8192, seed=8)
 # The second half of the GQA prefill's sequences as a chunk over a cache of their 4096 keys.
 GQA_CHUNK = Chunk("gqa_chunk_bf16_B2_Tq2048_at2048_H32_KV8_hd128", B=2, Tq=2048, qpos0=2048,
                   Lmax=4096, H=32, KV=8, hd=128, rope_base=500000.0, seed=7)
@@ -212,6 +229,22 @@ def chunk_inputs(w: Chunk, dtype=torch.bfloat16):
     k = normal((w.B, n, w.KV, w.hd), w.seed, dtype, gen)
     v = normal((w.B, n, w.KV, w.hd), w.seed, dtype, gen)
     return q, k, v
+
+
+def latent_inputs(w: Latent, dtype=torch.bfloat16):
+    """seqlens [B]; q [B,H,hd]; latent cache [B,Lmax,dc] (N(0,1) below each length, zero above);
+    W_uk, W_uv [H,dc,hd] ~ N(0,1)/sqrt(dc); drawn in that order."""
+    gen = torch.Generator().manual_seed(w.seed)
+    seqlens = torch.randint(w.len_lo, w.len_hi + 1, (w.B,), generator=gen, dtype=torch.int32)
+    q = normal((w.B, w.H, w.hd), w.seed, dtype, gen)
+    c = torch.zeros(w.B, w.Lmax, w.dc, dtype=dtype)
+    for b in range(w.B):
+        L = int(seqlens[b])
+        c[b, :L] = normal((L, w.dc), 0, dtype, gen)
+    scale = 1.0 / float(np.sqrt(w.dc))
+    W_uk = (torch.randn(w.H, w.dc, w.hd, generator=gen) * scale).to(dtype)
+    W_uv = (torch.randn(w.H, w.dc, w.hd, generator=gen) * scale).to(dtype)
+    return q, c, W_uk, W_uv, seqlens
 
 
 def decode_lengths(w: Decode) -> torch.Tensor:
