@@ -47,7 +47,11 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
   static constexpr int NBAR = 2 * NS + 5;  // kv_full[NS], kv_empty[NS], s_full, p_full, o_done, never, drain
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  // page index of every block of a split (paged cache): a split holds at most
+  // 2048 / page_size <= 256 pages
+  static constexpr int MAX_TAB = 256;
+  static constexpr int OFF_TAB = (OFF_MISC + 16 + 15) / 16 * 16;
+  static constexpr int SMEM = OFF_TAB + MAX_TAB * 4 + 1024;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, 0, 1);
 };
@@ -162,6 +166,26 @@ __global__ void __launch_bounds__(THREADS, 2)
 
   if (warp == 1) {
     // ------------------------------------------------------------ TMA producer
+    int* tab = reinterpret_cast<int*>(smem + C::OFF_TAB);
+    if (p.block_table) {
+      // the split's page indices, fetched by the whole warp at once; a page past the
+      // sequence (or an invalid table entry) becomes an out-of-range index, which reads zeros
+      const int ppt = BN / p.page_size;
+      const int n = min((jt1 - jt0 + 1) * ppt, C::MAX_TAB);
+      for (int idx = lane; idx < n; idx += 32) {
+        const int blk = jt0 * ppt + idx;
+        int page = p.num_pages;
+        if (blk * p.page_size < L) {
+          const int e = p.block_table[(size_t)b * p.max_blocks + blk];
+          if (e >= 0 && e < p.num_pages)
+            page = e;
+          else
+            flag_error(p.status, DEV_BAD_ARG);
+        }
+        tab[idx] = page;
+      }
+      __syncwarp();
+    }
     if (lane == 0) {
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
@@ -176,19 +200,11 @@ __global__ void __launch_bounds__(THREADS, 2)
             tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, (u & 1) ? &tmV : &tmK, kv_full + st,
                         kb * 64, kvh, j * BN, b);
         } else {
-          // one box per page of the tile; a page past the sequence (or an invalid table
-          // entry) is fetched at an out-of-range page index, which reads zeros
+          // one box per page of the tile
           const int ppt = BN / p.page_size;
           for (int i = 0; i < ppt; ++i) {
-            const int blk = j * ppt + i;
-            int page = p.num_pages;
-            if (blk * p.page_size < L) {
-              const int e = p.block_table[(size_t)b * p.max_blocks + blk];
-              if (e >= 0 && e < p.num_pages)
-                page = e;
-              else
-                flag_error(p.status, DEV_BAD_ARG);
-            }
+            const int ti = (j - jt0) * ppt + i;
+            const int page = ti < C::MAX_TAB ? tab[ti] : p.num_pages;
             for (int kb = 0; kb < HD / 64; ++kb)
               tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128 + i * p.page_size * 128, (u & 1) ? &tmV : &tmK,
                           kv_full + st, kb * 64, kvh, 0, page);
