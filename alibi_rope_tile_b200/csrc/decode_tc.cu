@@ -47,11 +47,12 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
   static constexpr int NBAR = 2 * NS + 5;  // kv_full[NS], kv_empty[NS], s_full, p_full, o_done, never, drain
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // page index of every block of a split (paged cache): a split holds at most
-  // 2048 / page_size <= 256 pages
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;  // (two CTAs per SM stay within 196 KB)
+  // paged cache only: the page index of every block of a split (a split holds at most
+  // 2048 / page_size <= 256 pages), reserved only when a paged decode is launched
   static constexpr int MAX_TAB = 256;
   static constexpr int OFF_TAB = (OFF_MISC + 16 + 15) / 16 * 16;
-  static constexpr int SMEM = OFF_TAB + MAX_TAB * 4 + 1024;
+  static constexpr int SMEM_PAGED = OFF_TAB + MAX_TAB * 4 + 1024;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, 0, 1);
 };
@@ -440,12 +441,13 @@ cudaError_t launch_hd(const DecodeParams& p, int chunk, int nsplit, void* ws, cu
       a.test_stall = 1;
     }
   }
+  const int smem = p.block_table ? Cfg<HD>::SMEM_PAGED : Cfg<HD>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Cfg<HD>::SMEM);
+                                       Cfg<HD>::SMEM_PAGED);
   if (e != cudaSuccess) return e;
   // split is the slowest grid dimension: the full leading splits of every sequence are
   // scheduled before the (shorter, often empty) trailing ones
-  decode_tc_kernel<HD><<<dim3(p.KV, p.B, nsplit), THREADS, Cfg<HD>::SMEM, s>>>(mk, mv, a);
+  decode_tc_kernel<HD><<<dim3(p.KV, p.B, nsplit), THREADS, smem, s>>>(mk, mv, a);
   return cudaGetLastError();
 }
 
