@@ -517,7 +517,8 @@ def run_ours(args, rank, world):
             "value": aggregate_rate(paged["bytes"] * args.steps, world, g_tot) / 1e9, "unit": "GB/s",
             "ms": ms, "bytes": paged["bytes"], "page_size": PAGE_SIZE, "pages": "shuffled",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "frac": gbs / pk["hbm_gbs"],
+                         "traffic": traffic.get(paged["w"].name + f"_paged{PAGE_SIZE}"),
                          "peak_source": f"{pk.get('source')} copy"}}
     if lat is not None:
         ms = l_tot / args.steps
@@ -527,7 +528,7 @@ def run_ours(args, rank, world):
             "ms": ms, "bytes": lat["bytes"],
             "note": "each latent tile is fetched twice (as keys and as values); bytes count it once",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "frac": gbs / pk["hbm_gbs"], "traffic": traffic.get(lat["w"].name),
                          "peak_source": f"{pk.get('source')} copy"}}
     cw = chk["w"]
     c_ms = c_tot / args.steps
