@@ -65,7 +65,7 @@ typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_ARG = -1,          /* a size, flag or pointer is invalid */
   ATTN_ERR_ALIGN = -2,        /* a pointer is not 16-byte aligned */
-  ATTN_ERR_UNSUPPORTED = -3,  /* a valid request this build does not implement */
+  ATTN_ERR_UNSUPPORTED = -3,  /* a valid request the library does not implement */
   ATTN_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed */
   ATTN_ERR_TIMEOUT = -5,      /* a device-side wait gave up (reported by attn_sync_status) */
   ATTN_ERR_WORKSPACE = -6,    /* workspace missing or smaller than the size query returned */
