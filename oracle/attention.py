@@ -310,6 +310,37 @@ def chunk(q, kcache, vcache, seqlens, qpos0, *, rope_base: float = 0.0, causal: 
     return out, lse
 
 
+def rmsnorm(x, gamma, eps: float = 1e-6) -> np.ndarray:
+    """RMSNorm ([XF5] "RMSNorm and Pre-LN residuals"): x / sqrt(mean(x^2) + eps) * gamma over
+    the last axis."""
+    x, gamma = _f64(x), _f64(gamma)
+    rms = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return x / rms * gamma
+
+
+def block_fused(x, gamma, Wqkv, Wo, *, H: int, KV: int, pos0: int = 0, rope_base: float = 0.0,
+                causal: bool = True, window: int = 0, slopes=None, eps: float = 1e-6):
+    """The attention sub-layer of a pre-norm decoder block ([XF5] "RMSNorm and Pre-LN
+    residuals": x + attn(norm(x))): RMSNorm, one projection x_n @ Wqkv whose columns are
+    [q heads | k heads | v heads] (Wqkv [d, (H + 2 KV) hd]), attention, ctx @ Wo, plus x.
+    Returns out [B,T,d] and the rows a cache keeps: k turned at positions pos0.., v [B,T,KV,hd]."""
+    x = _f64(x)
+    Wqkv, Wo = _f64(Wqkv), _f64(Wo)
+    B, T, d = x.shape
+    hd = Wqkv.shape[1] // (H + 2 * KV)
+    qkv = rmsnorm(x, gamma, eps) @ Wqkv
+    q = qkv[..., :H * hd].reshape(B, T, H, hd)
+    k = qkv[..., H * hd:(H + KV) * hd].reshape(B, T, KV, hd)
+    v = qkv[..., (H + KV) * hd:].reshape(B, T, KV, hd)
+    ctx, _ = attention(q, k, v, pos0=pos0, rope_base=rope_base, causal=causal, window=window,
+                       slopes=slopes)
+    out = x + ctx.reshape(B, T, H * hd) @ Wo
+    kc = k.transpose(0, 2, 1, 3)                                 # [B,KV,T,hd]
+    if rope_base > 0:
+        kc = rope(kc, pos0 + np.arange(T), rope_base)
+    return out, kc.transpose(0, 2, 1, 3), v
+
+
 def block(x, Wq, Wk, Wv, Wo, *, H: int, KV: int, pos0: int = 0, rope_base: float = 0.0,
           causal: bool = True, window: int = 0, slopes=None):
     """Projections, attention and output projection of [LAB] attention(): x [B,T,d] -> [B,T,d].

@@ -50,6 +50,11 @@ MUTANTS = {
                           "page = np.asarray(block_table)[b][j % page_size]"),
     "latent_scale_by_dc": ("s = k @ q[b, h] / np.sqrt(hd)", "s = k @ q[b, h] / np.sqrt(c.shape[2])"),
     "latent_value_projection": ("v = c[b, :L] @ W_uv[h]", "v = c[b, :L] @ W_uk[h]"),
+    "rmsnorm_mean_not_rms": ("rms = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)",
+                             "rms = np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)"),
+    "fused_no_residual": ("out = x + ctx.reshape(B, T, H * hd) @ Wo", "out = ctx.reshape(B, T, H * hd) @ Wo"),
+    "fused_qkv_split": ("k = qkv[..., H * hd:(H + KV) * hd].reshape(B, T, KV, hd)",
+                        "k = qkv[..., (H + KV) * hd:].reshape(B, T, KV, hd)"),
     "block_wq_transposed": ("q = (x @ Wq).reshape(B, T, H, hd)", "q = (x @ Wq.T).reshape(B, T, H, hd)"),
     "block_head_split": ("q = (x @ Wq).reshape(B, T, H, hd)",
                          "q = (x @ Wq).reshape(B, T, hd, H).swapaxes(2, 3)"),
@@ -68,6 +73,8 @@ PIN_TESTS = [
     ("test_chunk_of_one_row_is_a_decode_step_and_empty_cache", False),
     ("test_paged_decode_brute_force_and_page_order", False),
     ("test_latent_fold_leaves_scores_and_outputs_unchanged", False),
+    ("test_rmsnorm_closed_forms", False),
+    ("test_fused_block_is_residual_plus_the_plain_block_on_normalised_input", False),
 ]
 
 

@@ -375,6 +375,42 @@ def test_latent_fold_leaves_scores_and_outputs_unchanged():
     assert abs(s_unfolded - s_folded) < 1e-13
 
 
+def test_rmsnorm_closed_forms():
+    """RMSNorm: a constant vector c maps to sign(c) gamma (for eps -> 0); scaling x by s > 0
+    changes nothing; each normalised row has root-mean-square |gamma| when gamma is constant."""
+    g = np.full(6, 2.5)
+    np.testing.assert_allclose(A.rmsnorm(np.full((1, 6), -3.0), g, eps=0.0), np.full((1, 6), -2.5),
+                               rtol=0, atol=1e-15)
+    x = _rand((4, 6), 120)
+    np.testing.assert_allclose(A.rmsnorm(7.0 * x, g, eps=0.0), A.rmsnorm(x, g, eps=0.0), rtol=0, atol=1e-14)
+    y = A.rmsnorm(x, g, eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(y * y, axis=-1)), 2.5, rtol=0, atol=1e-14)
+    # eps enters under the root: x = 0 rows stay 0, tiny rows are damped
+    assert np.all(A.rmsnorm(np.zeros((1, 6)), g) == 0.0)
+
+
+def test_fused_block_is_residual_plus_the_plain_block_on_normalised_input():
+    """block_fused(x) - x equals the plain block on RMSNorm(x) with Wqkv split into Wq, Wk, Wv;
+    its cache rows are the keys turned at their positions and the values."""
+    B, T, d, H, KV, base, pos0 = 2, 9, 16, 4, 2, 10000.0, 5
+    hd = d // H
+    x, gamma = _rand((B, T, d), 121), 1.0 + 0.1 * _rand((d,), 122)
+    Wqkv, Wo = _rand((d, (H + 2 * KV) * hd), 123) / 4, _rand((H * hd, d), 124) / 4
+    Wq, Wk, Wv = Wqkv[:, :H * hd], Wqkv[:, H * hd:(H + KV) * hd], Wqkv[:, (H + KV) * hd:]
+    for window, slopes in [(0, None), (3, A.alibi_slopes(H))]:
+        out, kc, vc = A.block_fused(x, gamma, Wqkv, Wo, H=H, KV=KV, pos0=pos0, rope_base=base,
+                                    window=window, slopes=slopes)
+        plain = A.block(A.rmsnorm(x, gamma), Wq, Wk, Wv, Wo, H=H, KV=KV, pos0=pos0, rope_base=base,
+                        window=window, slopes=slopes)
+        np.testing.assert_allclose(out - x, plain, rtol=0, atol=1e-12)
+        k = (A.rmsnorm(x, gamma) @ Wk).reshape(B, T, KV, hd)
+        v = (A.rmsnorm(x, gamma) @ Wv).reshape(B, T, KV, hd)
+        ek, ev = A.kv_write(k, v, np.zeros((B, 20, KV, hd)), np.zeros((B, 20, KV, hd)), [pos0] * B,
+                            rope_base=base)
+        np.testing.assert_allclose(kc, ek[:, pos0:pos0 + T], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(vc, ev[:, pos0:pos0 + T], rtol=0, atol=0)
+
+
 # ----------------------------------------------------------------------------- workloads
 def test_workload_pair_counts():
     """FLOP counts used by the bench: causal pairs T(T+1)/2, windowed pairs sum min(i+1, W)."""
