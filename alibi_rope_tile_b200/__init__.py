@@ -42,6 +42,9 @@ SIGNATURES = {
                                _I, _P, _S, _P]),
     "attn_kv_write_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "attn_decode_latent_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "attn_block_fused_workspace_size": (_S, [_I, _I, _I, _I, _I, _I]),
+    "attn_block_fused": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _L, _F, _I, _I,
+                              _FP, _F, _I, _P, _S, _P]),
     "attn_decode_latent": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _FP, _I, _P, _S,
                                 _P]),
     "attn_block_workspace_size": (_S, [_I, _I, _I, _I, _I, _I, _I]),
@@ -316,6 +319,31 @@ def attn_block(x, Wq, Wk, Wv, Wo, out=None, workspace=None, *, H: int, KV: int, 
                           float(rope_base), int(bool(causal)), int(window), _slopes(alibi_slopes, H),
                           _dtype(x), _dev(workspace, "workspace"),
                           workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st)
+    return out
+
+
+def attn_block_fused(x, gamma, Wqkv, Wo, out=None, kcache=None, vcache=None, workspace=None, *,
+                     H: int, KV: int, pos0: int = 0, rope_base: float = 0.0, causal: bool = True,
+                     window: int = 0, alibi_slopes=None, eps: float = 1e-6, stream=None):
+    """x [B,T,d] -> x + attention(RMSNorm(x) Wqkv) Wo (Wqkv [d,(H+2KV)hd] = [q|k|v] heads);
+    with caches [B,Lmax,KV,hd], the turned keys and the values go to slots pos0 .. pos0+T-1."""
+    B, T, d = x.shape
+    hd = Wqkv.shape[1] // (H + 2 * KV)
+    dt = x.dtype
+    if out is None:
+        out = torch.empty_like(x)
+    Lmax = kcache.shape[1] if kcache is not None else 0
+    need = int(lib().attn_block_fused_workspace_size(B, T, d, H, KV, hd))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    st = lib().attn_block_fused(_dev(x, "x"), _dev(gamma, "gamma", dt), _dev(Wqkv, "Wqkv", dt),
+                                _dev(Wo, "Wo", dt), _dev(out, "out", dt), _dev(kcache, "kcache", dt),
+                                _dev(vcache, "vcache", dt), Lmax, B, T, d, H, KV, hd, int(pos0),
+                                float(rope_base), int(bool(causal)), int(window),
+                                _slopes(alibi_slopes, H), float(eps), _dtype(x),
+                                _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                                _stream(stream))
     _check(st)
     return out
 

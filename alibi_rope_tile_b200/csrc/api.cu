@@ -473,6 +473,93 @@ int attn_block(const void* x, const void* Wq, const void* Wk, const void* Wv, co
   return ok();
 }
 
+namespace {
+struct FusedLayout {
+  size_t xn, q, k, v, ctx, cs, total;
+};
+FusedLayout fused_layout(int B, int T, int d, int H, int KV, int hd) {
+  FusedLayout L;
+  const size_t M = (size_t)B * T;
+  L.xn = 0;
+  L.q = L.xn + round256(M * d * 2);
+  L.k = L.q + round256(M * H * hd * 2);
+  L.v = L.k + round256(M * KV * hd * 2);
+  L.ctx = L.v + round256(M * KV * hd * 2);
+  L.cs = L.ctx + round256(M * H * hd * 2);
+  L.total = L.cs + round256((size_t)T * (hd / 2) * sizeof(float2));
+  return L;
+}
+}  // namespace
+
+size_t attn_block_fused_workspace_size(int B, int T, int d, int H, int KV, int hd) {
+  if (B < 1 || T < 1 || d < 1 || H < 1 || KV < 1 || H % KV || hd < 2) return 0;
+  return fused_layout(B, T, d, H, KV, hd).total;
+}
+
+int attn_block_fused(const void* x, const void* gamma, const void* Wqkv, const void* Wo, void* out,
+                     void* kcache, void* vcache, int Lmax, int B, int T, int d, int H, int KV, int hd,
+                     long long pos0, float rope_base, int causal, int window, const float* alibi_slopes,
+                     float eps, int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  int st = check_common(H, KV, hd, dtype, rope_base);
+  if (st) return st;
+  if (!x || !gamma || !Wqkv || !Wo || !out)
+    return fail(ATTN_ERR_ARG, "x, gamma, Wqkv, Wo and out must not be NULL");
+  if ((kcache == nullptr) != (vcache == nullptr)) return fail(ATTN_ERR_ARG, "give both caches or neither");
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(Wqkv) || !aligned16(Wo) || !aligned16(out) ||
+      (kcache && (!aligned16(kcache) || !aligned16(vcache))) || (workspace && !aligned16(workspace)))
+    return fail(ATTN_ERR_ALIGN, "tensors and workspace must be 16-byte aligned");
+  if (B < 1 || T < 1 || d < 8 || d % 8) return fail(ATTN_ERR_ARG, "B, T >= 1 and d a multiple of 8");
+  if (!std::isfinite(eps) || eps < 0.f) return fail(ATTN_ERR_ARG, "eps must be finite and >= 0");
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
+  if (window < 0) window = 0;
+  if (window > 0 && !causal) return fail(ATTN_ERR_ARG, "a window requires the causal mask");
+  if (pos0 < 0 || pos0 + (long long)T >= (1LL << 24))
+    return fail(ATTN_ERR_ARG, "positions pos0..pos0+T-1 must lie in [0, 2^24)");
+  if (kcache && (Lmax < 1 || pos0 + (long long)T > Lmax))
+    return fail(ATTN_ERR_ARG, "the cache must hold slots pos0..pos0+T-1 (Lmax=%d)", Lmax);
+  const int M = B * T, Nqkv = (H + 2 * KV) * hd;
+  if ((long long)B * T * (H + 2 * KV) * hd >= (1LL << 40) || (long long)B * T * d >= (1LL << 40))
+    return fail(ATTN_ERR_ARG, "tensor too large");
+  if (dtype != ATTN_BF16 || (hd != 64 && hd != 128) || !gemm_tc_supported(M, Nqkv, d, dtype) ||
+      !gemm_tc_supported(M, d, H * hd, dtype))
+    return fail(ATTN_ERR_UNSUPPORTED, "attn_block_fused runs bf16 with hd 64 or 128 on the tensor-core GEMM");
+  const FusedLayout L = fused_layout(B, T, d, H, KV, hd);
+  if (!workspace || ws_bytes < L.total)
+    return fail(ATTN_ERR_WORKSPACE, "fused block needs %zu bytes of workspace (got %zu)", L.total, ws_bytes);
+  int err = 0;
+  int* status = device_status(&err);
+  if (!status) return err;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const RopeFreqs rope = make_rope(hd, rope_base);
+  float2* cs = reinterpret_cast<float2*>(ws + L.cs);
+  cudaError_t e = cudaSuccess;
+  if (rope.on) e = launch_rope_table(cs, T, (int)pos0, rope, hd, s);
+  if (e == cudaSuccess) e = launch_rmsnorm(x, gamma, ws + L.xn, M, d, eps, s);
+  if (e != cudaSuccess) return cuda_fail(e, "fused block norm");
+  GemmEpilogue qkv;
+  std::memset(&qkv, 0, sizeof(qkv));
+  qkv.mode = 1;
+  qkv.T = T; qkv.H = H; qkv.KV = KV; qkv.hd = hd;
+  qkv.rope_cs = rope.on ? cs : nullptr;
+  qkv.q = ws + L.q; qkv.k = ws + L.k; qkv.v = ws + L.v;
+  qkv.kcache = kcache; qkv.vcache = vcache; qkv.Lmax = Lmax; qkv.pos0 = (int)pos0;
+  if ((e = launch_gemm_tc(ws + L.xn, Wqkv, nullptr, M, Nqkv, d, status, s, &qkv)) != cudaSuccess)
+    return cuda_fail(e, "fused block QKV GEMM");
+  // q and k are already turned: the attention runs without rotation (its masks and ALiBi depend
+  // only on i - j)
+  st = attn_prefill(ws + L.q, ws + L.k, ws + L.v, ws + L.ctx, nullptr, B, T, H, KV, hd, pos0, 0.f, causal,
+                    window, alibi_slopes, dtype, stream);
+  if (st) return st;
+  GemmEpilogue res;
+  std::memset(&res, 0, sizeof(res));
+  res.mode = 2;
+  res.residual = x;
+  if ((e = launch_gemm_tc(ws + L.ctx, Wo, out, M, d, H * hd, status, s, &res)) != cudaSuccess)
+    return cuda_fail(e, "fused block Wo GEMM");
+  return ok();
+}
+
 void attn_alibi_slopes(int H, float* host_out) {
   if (!host_out || H < 1) return;
   for (int h = 0; h < H; ++h) host_out[h] = (float)std::pow(2.0, -8.0 * (h + 1.0) / H);

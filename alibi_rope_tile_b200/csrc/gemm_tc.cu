@@ -9,7 +9,14 @@
 // loads, warp 5 allocates TMEM and issues the M=128, N=256, K=16 MMAs (four per stage),
 // warps 0-3 read the accumulator back (one TMEM lane = one row of C per thread) and store
 // bf16. Rows and columns past M, N are zero-filled on load and not stored.
+//
+// Epilogues (GemmEpilogue): a plain store; the fused block's QKV scatter, which sends each
+// 32-column chunk (within one head, since hd is 64 or 128 and tiles start at multiples of 256)
+// to q, k or v, turns q and k pairwise by the (cos, sin) table of its row's position, and
+// also writes k and v rows into a KV cache; or the output projection plus a residual.
 #include <cudaTypedefs.h>
+
+#include <cstring>
 
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -35,7 +42,16 @@ struct GemmArgs {
   __nv_bfloat16* C;
   int M, N, K;
   int* status;
+  GemmEpilogue ep;
 };
+
+__device__ __forceinline__ void store32(__nv_bfloat16* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(dst + 8 * q) =
+        make_uint4(f2_to_bf2(v[8 * q], v[8 * q + 1]), f2_to_bf2(v[8 * q + 2], v[8 * q + 3]),
+                   f2_to_bf2(v[8 * q + 4], v[8 * q + 5]), f2_to_bf2(v[8 * q + 6], v[8 * q + 7]));
+}
 
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
@@ -121,8 +137,49 @@ __global__ void __launch_bounds__(THREADS, 1)
         float v[32];
         tmem_ld32(t + c0, v);
         tmem_wait_ld();
-        if (row < g.M) {
+        if (row < g.M && g.ep.mode == 1) {
+          const GemmEpilogue& e = g.ep;
+          const int n = n0 + c0;
+          if (n < g.N) {
+            const int b = row / e.T, t = row - b * e.T;
+            const int hh = n / e.hd, d = n - hh * e.hd;
+            const int region = hh < e.H ? 0 : (hh < e.H + e.KV ? 1 : 2);
+            const int head = region == 0 ? hh : (region == 1 ? hh - e.H : hh - e.H - e.KV);
+            if (region < 2 && e.rope_cs) {
+              const float2* cs = e.rope_cs + (size_t)t * (e.hd / 2) + d / 2;
+#pragma unroll
+              for (int p = 0; p < 16; ++p) {
+                const float2 c = cs[p];
+                const float x = v[2 * p], y = v[2 * p + 1];
+                v[2 * p] = x * c.x - y * c.y;
+                v[2 * p + 1] = x * c.y + y * c.x;
+              }
+            }
+            const int nh = region == 0 ? e.H : e.KV;
+            __nv_bfloat16* base = static_cast<__nv_bfloat16*>(region == 0 ? e.q : (region == 1 ? e.k : e.v));
+            store32(base + (((size_t)b * e.T + t) * nh + head) * e.hd + d, v);
+            if (region > 0 && e.kcache) {
+              __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(region == 1 ? e.kcache : e.vcache);
+              store32(cache + (((size_t)b * e.Lmax + e.pos0 + t) * e.KV + head) * e.hd + d, v);
+            }
+          }
+        } else if (row < g.M) {
           __nv_bfloat16* dst = g.C + (size_t)row * g.N + n0 + c0;
+          if (g.ep.mode == 2) {
+            const __nv_bfloat16* res = static_cast<const __nv_bfloat16*>(g.ep.residual) + (size_t)row * g.N + n0 + c0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (n0 + c0 + 8 * q + 8 <= g.N) {
+                const uint4 u = *reinterpret_cast<const uint4*>(res + 8 * q);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float2 f = bf2_to_f2(w[i]);
+                  v[8 * q + 2 * i] += f.x;
+                  v[8 * q + 2 * i + 1] += f.y;
+                }
+              }
+          }
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             if (n0 + c0 + 8 * q + 8 <= g.N)
@@ -178,7 +235,7 @@ bool gemm_tc_supported(int M, int N, int K, int dtype) {
 }
 
 cudaError_t launch_gemm_tc(const void* A, const void* W, void* C, int M, int N, int K, int* status,
-                           cudaStream_t s) {
+                           cudaStream_t s, const GemmEpilogue* ep) {
   using namespace tcgemm;
   CUtensorMap ma, mw;
   if (!make_map2d(&ma, A, M, K, BM) || !make_map2d(&mw, W, K, N, BK)) return cudaErrorInvalidValue;
@@ -188,6 +245,8 @@ cudaError_t launch_gemm_tc(const void* A, const void* W, void* C, int M, int N, 
   g.N = N;
   g.K = K;
   g.status = status;
+  std::memset(&g.ep, 0, sizeof(g.ep));
+  if (ep) g.ep = *ep;
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
   gemm_tc_kernel<<<dim3((N + BN - 1) / BN, (M + BM - 1) / BM), THREADS, SMEM, s>>>(ma, mw, g);

@@ -92,9 +92,30 @@ cudaError_t launch_head_proj(bool fold, const void* x, const void* W, void* y, i
 cudaError_t launch_gemm_simt(const void* A, const void* W, void* C, int M, int N, int K, int dtype,
                              cudaStream_t s);
 // Tensor-core (tcgen05) version for bf16 when M, N, K fit its tiles.
+// Epilogues of the tensor-core GEMM beyond a plain store of C (bf16).
+struct GemmEpilogue {
+  int mode;  // 0: C = A W; 1: scatter the columns [q heads | k heads | v heads] of A Wqkv to
+             // q [B,T,H,hd], k, v [B,T,KV,hd] (row m = b*T + t), turning q and k by rope_cs,
+             // and also write k, v to kcache, vcache slot pos0 + t when kcache != nullptr;
+             // 2: C = A W + residual ([M,N])
+  int T, H, KV, hd;
+  const float2* rope_cs;  // [T][hd/2] (cos, sin) of position pos0 + t, or nullptr
+  void* q;
+  void* k;
+  void* v;
+  void* kcache;
+  void* vcache;
+  int Lmax, pos0;
+  const void* residual;
+};
 bool gemm_tc_supported(int M, int N, int K, int dtype);
 cudaError_t launch_gemm_tc(const void* A, const void* W, void* C, int M, int N, int K, int* status,
-                           cudaStream_t s);
+                           cudaStream_t s, const GemmEpilogue* ep = nullptr);
+
+// Pre-norm helpers of the fused block: y = RMSNorm(x) * gamma per row (bf16), and the table of
+// (cos, sin) of every (position pos0 + t, pair) the QKV epilogue turns by.
+cudaError_t launch_rmsnorm(const void* x, const void* gamma, void* y, int M, int d, float eps, cudaStream_t s);
+cudaError_t launch_rope_table(float2* cs, int T, int pos0, const RopeFreqs& rope, int hd, cudaStream_t s);
 
 // Records a failure for attn_last_error() and returns ``code`` (used by entry points
 // defined outside api.cu).

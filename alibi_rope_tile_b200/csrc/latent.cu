@@ -94,3 +94,4 @@ cudaError_t launch_head_proj(bool fold, const void* x, const void* W, void* y, i
 }
 
 }  // namespace attn
+

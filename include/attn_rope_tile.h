@@ -257,6 +257,26 @@ int attn_block(const void* x, const void* Wq, const void* Wk, const void* Wv, co
                float rope_base, int causal, int window, const float* alibi_slopes, int dtype,
                void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * attn_block_fused -- the attention sub-layer of a pre-norm decoder block ([XF5] "RMSNorm and
+ * Pre-LN residuals": x + attn(norm(x))), fused around the attention core:
+ *   xn = x / sqrt(mean(x^2) + eps) * gamma                      (RMSNorm per row)
+ *   [q | k | v] = xn @ Wqkv, Wqkv [d, (H + 2 KV) hd] ([in, out]; columns: q heads, k heads,
+ *                 v heads); q and k are turned at positions pos0 + t in the GEMM's epilogue,
+ *                 which also writes k (turned) and v to kcache, vcache slots pos0 + t
+ *   out = x + attention(q, k, v) @ Wo                           (the residual in the epilogue)
+ * x, out: [B,T,d]; gamma: [d]; Wo: [H*hd, d]; all bf16 (device). kcache, vcache: [B,Lmax,KV,hd]
+ * or both NULL (no cache write); with caches, pos0 + T <= Lmax. Causal, window and ALiBi as
+ * attn_prefill. workspace: attn_block_fused_workspace_size(...) bytes (device, caller-owned).
+ * bf16, hd in {64, 128}, d and (H + 2 KV) hd multiples of 8; anything else returns
+ * ATTN_ERR_UNSUPPORTED. Launches: RoPE table, RMSNorm, QKV GEMM, attention, Wo GEMM.
+ */
+size_t attn_block_fused_workspace_size(int B, int T, int d, int H, int KV, int hd);
+int attn_block_fused(const void* x, const void* gamma, const void* Wqkv, const void* Wo, void* out,
+                     void* kcache, void* vcache, int Lmax, int B, int T, int d, int H, int KV, int hd,
+                     long long pos0, float rope_base, int causal, int window, const float* alibi_slopes,
+                     float eps, int dtype, void* workspace, size_t ws_bytes, void* stream);
+
 /* attn_alibi_slopes -- host_out[h] = 2^(-8(h+1)/H) for h < H ([ALIBI] Step 1; the slope
  * schedule with exponent 8/H). host_out is a HOST buffer of H floats. */
 void attn_alibi_slopes(int H, float* host_out);

@@ -32,7 +32,7 @@ def test_header_declares_entry_points():
     names = declared_functions()
     for must in ("attn_prefill", "attn_decode", "attn_block", "attn_kv_append",
                  "attn_prefill_chunk", "attn_kv_write", "attn_decode_paged", "attn_kv_write_paged",
-                 "attn_decode_latent",
+                 "attn_decode_latent", "attn_block_fused",
                  "attn_decode_workspace_size", "attn_block_workspace_size", "attn_alibi_slopes",
                  "attn_sync_status", "attn_last_error", "attn_version"):
         assert must in names
@@ -180,6 +180,23 @@ def test_latent_argument_errors(lib):
     assert lat(dtype=0) == -3
     assert lib.attn_decode_latent_workspace_size(4, 32, 128, 96, 256) == 0
     assert lib.attn_decode_latent_workspace_size(4, 32, 128, 64, 256) > 0
+
+
+def test_fused_block_argument_errors(lib):
+    P = 0x1000
+    def fused(**kw):
+        a = dict(gamma=P, kc=None, vc=None, Lmax=0, T=16, d=512, H=8, KV=2, hd=64, pos0=0, dtype=1)
+        a.update(kw)
+        return lib.attn_block_fused(P, a["gamma"], P, P, P, a["kc"], a["vc"], a["Lmax"], 2, a["T"], a["d"],
+                                    a["H"], a["KV"], a["hd"], a["pos0"], 10000.0, 1, 0, None, 1e-6,
+                                    a["dtype"], P, 1 << 30, None)
+    assert fused(gamma=None) == -1
+    assert fused(kc=P) == -1                          # one cache without the other
+    assert fused(kc=P, vc=P, Lmax=20, pos0=8) == -1   # slots pos0..pos0+T-1 exceed the cache
+    assert fused(d=500) == -1                         # d not a multiple of 8
+    assert fused(hd=32, d=256) == -3                  # head size without a tensor-core path
+    assert fused(dtype=0) == -3
+    assert lib.attn_block_fused_workspace_size(2, 16, 512, 8, 2, 64) > 0
 
 
 def test_binding_requires_cuda_tensors(lib):
