@@ -58,6 +58,7 @@ PAGE_SIZE = 16            # rows per page of the paged decode (the KV=8 decode w
 BLOCK_LAUNCHES = 5        # three projection GEMMs, the prefill, the output GEMM
 CHUNK_LAUNCHES = 1
 LATENT_LAUNCHES = 4       # the fold, the split pass, the merge, the value up-projection
+FUSED_LAUNCHES = 5        # RoPE table, RMSNorm, QKV GEMM (+ rotation, cache write), prefill, Wo GEMM (+ residual)
 
 
 def peaks():
@@ -302,6 +303,16 @@ def run_ours(args, rank, world):
                    ws=torch.empty(art.attn_block_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV, bw.hd,
                                                                  torch.bfloat16),
                                   dtype=torch.uint8, device="cuda"))
+        # the same block as a fused pre-norm sub-layer: RMSNorm, one Wqkv, cache write, residual
+        fz = dict(gamma=torch.ones(bw.d, dtype=torch.bfloat16, device="cuda"),
+                  Wqkv=torch.cat([blk["W"]["Wq"], blk["W"]["Wk"], blk["W"]["Wv"]], dim=1).contiguous(),
+                  kc=torch.zeros(bw.B, bw.T, bw.KV, bw.hd, dtype=torch.bfloat16, device="cuda"),
+                  out=torch.empty_like(blk["out"]),
+                  ws=torch.empty(int(art.lib().attn_block_fused_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV,
+                                                                               bw.hd)),
+                                 dtype=torch.uint8, device="cuda"))
+        fz["vc"] = torch.zeros_like(fz["kc"])
+        blk["fused"] = fz
         del hW
     chk = None
     if do_c:
@@ -339,6 +350,13 @@ def run_ours(args, rank, world):
                                   paged["qp"], paged["out"], workspace=paged["ws"],
                                   rope_base=paged["w"].rope_base)
 
+    def block_fused():
+        if blk is not None:
+            bw, fz = blk["w"], blk["fused"]
+            art.attn_block_fused(blk["x"], fz["gamma"], fz["Wqkv"], blk["W"]["Wo"], fz["out"], fz["kc"], fz["vc"],
+                                 fz["ws"], H=bw.H, KV=bw.KV, rope_base=bw.rope_base, causal=bw.causal,
+                                 window=bw.window)
+
     def decode_latent():
         if lat is not None:
             art.attn_decode_latent(lat["q"], lat["c"], lat["uk"], lat["uv"], lat["sl"], lat["sl"], lat["out"],
@@ -358,10 +376,11 @@ def run_ours(args, rank, world):
         chunk()
         decode_paged()
         decode_latent()
+        block_fused()
     torch.cuda.synchronize()
     art.attn_sync_status()
 
-    nev = 2 + 2 * len(decs) + 8
+    nev = 2 + 2 * len(decs) + 10
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
@@ -380,6 +399,10 @@ def run_ours(args, rank, world):
             ev[s_][2 + 2 * n].record(stream)
             decode(d)
             ev[s_][3 + 2 * n].record(stream)
+        flush.zero_()
+        ev[s_][nev - 10].record(stream)
+        block_fused()
+        ev[s_][nev - 9].record(stream)
         flush.zero_()
         ev[s_][nev - 8].record(stream)
         decode_latent()
@@ -413,6 +436,8 @@ def run_ours(args, rank, world):
                                          for s_ in range(args.steps)), world))
     l_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 8].elapsed_time(ev[s_][nev - 7])
                                          for s_ in range(args.steps)), world))
+    f_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 10].elapsed_time(ev[s_][nev - 9])
+                                         for s_ in range(args.steps)), world))
     region_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
 
     # end to end through the public API: the step's inputs go host (pinned) -> device, the
@@ -424,6 +449,7 @@ def run_ours(args, rank, world):
     if blk is not None:
         hbx = blk["hx"].pin_memory()
         hbo = torch.empty(blk["hx"].shape, dtype=blk["hx"].dtype).pin_memory()
+        hfo = torch.empty(blk["hx"].shape, dtype=blk["hx"].dtype).pin_memory()
     if paged is not None:
         hpo = torch.empty(paged["out"].shape, dtype=paged["out"].dtype).pin_memory()
     if lat is not None:
@@ -448,6 +474,8 @@ def run_ours(args, rank, world):
             blk["x"].copy_(hbx, non_blocking=True)
             block()
             hbo.copy_(blk["out"], non_blocking=True)
+            block_fused()
+            hfo.copy_(blk["fused"]["out"], non_blocking=True)
         if chk is not None:
             chk["q"].copy_(hcq_p, non_blocking=True)
             chunk()
@@ -510,6 +538,14 @@ def run_ours(args, rank, world):
         "projections_derived": {"tflops": proj_tflops, "ms": proj_ms,
                                 "frac": proj_tflops / pk["bf16_tflops"],
                                 "how": "block time minus the prefill time of the same shape"}}
+    f_ms = f_tot / args.steps
+    f_tflops = bw.flops / (f_ms * 1e-3) / 1e12
+    block_out["fused"] = {
+        "what": "RMSNorm, one QKV GEMM (RoPE and cache write in its epilogue), attention, Wo GEMM + residual",
+        "value": aggregate_rate(bw.flops * args.steps, world, f_tot) / 1e12, "unit": "TFLOP/s", "ms": f_ms,
+        "roofline": {"bound": "tensor", "achieved": f_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": f_tflops / pk["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{pk.get('source')} burst bf16 dense"}}
     if paged is not None:
         ms = g_tot / args.steps
         gbs = paged["bytes"] / (ms * 1e-3) / 1e9
@@ -545,7 +581,7 @@ def run_ours(args, rank, world):
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v)) + sum(
         d["hq"].numel() * d["hq"].element_size() for d in decs) + xb + cb
     d2h = q.numel() * q.element_size() + sum(
-        d["hq"].numel() * d["hq"].element_size() for d in decs) + xb + cb
+        d["hq"].numel() * d["hq"].element_size() for d in decs) + 2 * xb + cb
     if paged is not None:
         d2h += paged["out"].numel() * paged["out"].element_size()
     if lat is not None:
@@ -559,7 +595,7 @@ def run_ours(args, rank, world):
     line = {
         "metric": METRIC, "value": aggregate_rate(flops_step * args.steps, world, p_tot) / 1e12,
         "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": (p_tot + sum(d_tot) + b_tot + c_tot + g_tot + l_tot) / args.steps,
+        "ms_per_step": (p_tot + sum(d_tot) + b_tot + c_tot + g_tot + l_tot + f_tot) / args.steps,
         "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "decode_workloads": [d["w"].name for d in decs],
@@ -581,7 +617,7 @@ def run_ours(args, rank, world):
                         "(block weights resident; x in, out back) and the chunk (cache resident; "
                         "its queries in, out back)"},
         "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES * (len(decs) + 1) + BLOCK_LAUNCHES
-                                      + CHUNK_LAUNCHES + LATENT_LAUNCHES),
+                                      + CHUNK_LAUNCHES + LATENT_LAUNCHES + FUSED_LAUNCHES),
         "clocks": clk,
         "cpu_baseline": cpu,
     }
