@@ -109,6 +109,14 @@ def _dev(t: Optional[torch.Tensor], name: str, dtype=None) -> int:
     return t.data_ptr()
 
 
+def _shape(t: Optional[torch.Tensor], shape, name: str) -> None:
+    """Raise unless ``t`` (when given) has exactly ``shape``: the library derives every index
+    from the sizes it is passed, so a tensor of another shape would be read or written out of
+    bounds."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
 def _stream(stream) -> int:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -139,6 +147,8 @@ def attn_prefill(q, k, v, out=None, lse=None, *, pos0: int = 0, rope_base: float
     KV = k.shape[2]
     if k.shape != (B, T, KV, hd) or v.shape != k.shape:
         raise ValueError(f"k and v must be [B,T,KV,hd] matching q {tuple(q.shape)}")
+    _shape(out, q.shape, "out")
+    _shape(lse, (B, H, T), "lse")
     dt = q.dtype
     if out is None:
         out = torch.empty_like(q)
@@ -150,6 +160,17 @@ def attn_prefill(q, k, v, out=None, lse=None, *, pos0: int = 0, rope_base: float
     return out
 
 
+def _decode_shapes(q, kcache, vcache, seqlens, qpos, out, lse) -> None:
+    B, H, hd = q.shape
+    if kcache.dim() != 4 or kcache.shape[0] != B or kcache.shape[3] != hd:
+        raise ValueError(f"kcache must be [B={B},Lmax,KV,hd={hd}], got {tuple(kcache.shape)}")
+    _shape(vcache, kcache.shape, "vcache")
+    _shape(seqlens, (B,), "seqlens")
+    _shape(qpos, (B,), "qpos")
+    _shape(out, q.shape, "out")
+    _shape(lse, (B, H), "lse")
+
+
 def attn_decode_workspace_size(B: int, H: int, KV: int, hd: int, Lmax: int) -> int:
     return int(lib().attn_decode_workspace_size(B, H, KV, hd, Lmax))
 
@@ -159,6 +180,7 @@ def attn_decode(q, kcache, vcache, seqlens, qpos, out=None, lse=None, workspace=
     """q [B,H,hd] (not rotated), caches [B,Lmax,KV,hd], seqlens/qpos [B] int32 -> out [B,H,hd]."""
     B, H, hd = q.shape
     _, Lmax, KV, _ = kcache.shape
+    _decode_shapes(q, kcache, vcache, seqlens, qpos, out, lse)
     dt = q.dtype
     if out is None:
         out = torch.empty_like(q)
@@ -181,6 +203,9 @@ def attn_decode_noalloc(q, kcache, vcache, seqlens, qpos, out, lse=None, *,
     the library's fixed scratch array, so no workspace is passed; ``out`` must be given."""
     B, H, hd = q.shape
     _, Lmax, KV, _ = kcache.shape
+    if out is None:
+        raise ValueError("attn_decode_noalloc writes into a caller-given out [B,H,hd]")
+    _decode_shapes(q, kcache, vcache, seqlens, qpos, out, lse)
     dt = q.dtype
     st = lib().attn_decode_noalloc(_dev(q, "q"), _dev(kcache, "kcache", dt),
                                    _dev(vcache, "vcache", dt), _dev(seqlens, "seqlens", torch.int32),
@@ -199,6 +224,12 @@ def attn_prefill_chunk(q, kcache, vcache, seqlens, qpos0, out=None, lse=None, *,
     (keys rotated), slots < seqlens[b] -> out [B,Tq,H,hd] (and lse [B,H,Tq])."""
     B, Tq, H, hd = q.shape
     _, Lmax, KV, _ = kcache.shape
+    _shape(kcache, (B, Lmax, KV, hd), "kcache")
+    _shape(vcache, kcache.shape, "vcache")
+    _shape(seqlens, (B,), "seqlens")
+    _shape(qpos0, (B,), "qpos0")
+    _shape(out, q.shape, "out")
+    _shape(lse, (B, H, Tq), "lse")
     dt = q.dtype
     if out is None:
         out = torch.empty_like(q)
@@ -215,6 +246,10 @@ def attn_kv_write(k_new, v_new, kcache, vcache, pos0, *, rope_base: float = 0.0,
     """Write k_new, v_new [B,Tn,KV,hd] into cache slots pos0[b] .. pos0[b]+Tn-1 (keys rotated)."""
     B, Tn, KV, hd = k_new.shape
     Lmax = kcache.shape[1]
+    _shape(v_new, k_new.shape, "v_new")
+    _shape(kcache, (B, Lmax, KV, hd), "kcache")
+    _shape(vcache, kcache.shape, "vcache")
+    _shape(pos0, (B,), "pos0")
     dt = k_new.dtype
     st = lib().attn_kv_write(_dev(k_new, "k_new"), _dev(v_new, "v_new", dt), _dev(kcache, "kcache", dt),
                              _dev(vcache, "vcache", dt), _dev(pos0, "pos0", torch.int32), B, Tn, KV, hd,
@@ -230,6 +265,13 @@ def attn_decode_paged(q, kpages, vpages, block_table, seqlens, qpos, out=None, l
     B, H, hd = q.shape
     num_pages, page_size, KV, _ = kpages.shape
     max_blocks = block_table.shape[1]
+    _shape(kpages, (num_pages, page_size, KV, hd), "kpages")
+    _shape(vpages, kpages.shape, "vpages")
+    _shape(block_table, (B, max_blocks), "block_table")
+    _shape(seqlens, (B,), "seqlens")
+    _shape(qpos, (B,), "qpos")
+    _shape(out, q.shape, "out")
+    _shape(lse, (B, H), "lse")
     dt = q.dtype
     if out is None:
         out = torch.empty_like(q)
@@ -253,6 +295,11 @@ def attn_kv_write_paged(k_new, v_new, kpages, vpages, block_table, pos0, *, rope
     B, Tn, KV, hd = k_new.shape
     num_pages, page_size = kpages.shape[:2]
     max_blocks = block_table.shape[1]
+    _shape(v_new, k_new.shape, "v_new")
+    _shape(kpages, (num_pages, page_size, KV, hd), "kpages")
+    _shape(vpages, kpages.shape, "vpages")
+    _shape(block_table, (B, max_blocks), "block_table")
+    _shape(pos0, (B,), "pos0")
     dt = k_new.dtype
     st = lib().attn_kv_write_paged(_dev(k_new, "k_new"), _dev(v_new, "v_new", dt),
                                    _dev(kpages, "kpages", dt), _dev(vpages, "vpages", dt),
@@ -269,6 +316,13 @@ def attn_decode_latent(q, ccache, W_uk, W_uv, seqlens, qpos, out=None, lse=None,
     W_uk, W_uv [H,dc,hd] -> out [B,H,hd] (the key up-projection folded into the query)."""
     B, H, hd = q.shape
     _, Lmax, dc = ccache.shape
+    _shape(ccache, (B, Lmax, dc), "ccache")
+    _shape(W_uk, (H, dc, hd), "W_uk")
+    _shape(W_uv, (H, dc, hd), "W_uv")
+    _shape(seqlens, (B,), "seqlens")
+    _shape(qpos, (B,), "qpos")
+    _shape(out, q.shape, "out")
+    _shape(lse, (B, H), "lse")
     dt = q.dtype
     if out is None:
         out = torch.empty_like(q)
@@ -289,6 +343,10 @@ def attn_kv_append(k_new, v_new, kcache, vcache, pos, *, rope_base: float = 0.0,
     """Write k_new (rotated at pos[b]) and v_new [B,KV,hd] into cache slot pos[b]."""
     B, KV, hd = k_new.shape
     Lmax = kcache.shape[1]
+    _shape(v_new, k_new.shape, "v_new")
+    _shape(kcache, (B, Lmax, KV, hd), "kcache")
+    _shape(vcache, kcache.shape, "vcache")
+    _shape(pos, (B,), "pos")
     dt = k_new.dtype
     st = lib().attn_kv_append(_dev(k_new, "k_new"), _dev(v_new, "v_new", dt),
                               _dev(kcache, "kcache", dt), _dev(vcache, "vcache", dt),
@@ -307,7 +365,14 @@ def attn_block(x, Wq, Wk, Wv, Wo, out=None, workspace=None, *, H: int, KV: int, 
                stream=None):
     """x [B,T,d] -> out [B,T,d] = attention(x Wq, x Wk, x Wv) Wo (weights [in, out])."""
     B, T, d = x.shape
+    if H < 1 or KV < 1 or Wq.dim() != 2 or Wq.shape[1] % H:
+        raise ValueError(f"Wq must be [d, H*hd] with H={H}, got {tuple(Wq.shape)}")
     hd = Wq.shape[1] // H
+    _shape(Wq, (d, H * hd), "Wq")
+    _shape(Wk, (d, KV * hd), "Wk")
+    _shape(Wv, (d, KV * hd), "Wv")
+    _shape(Wo, (H * hd, d), "Wo")
+    _shape(out, x.shape, "out")
     dt = x.dtype
     if out is None:
         out = torch.empty_like(x)
@@ -329,7 +394,20 @@ def attn_block_fused(x, gamma, Wqkv, Wo, out=None, kcache=None, vcache=None, wor
     """x [B,T,d] -> x + attention(RMSNorm(x) Wqkv) Wo (Wqkv [d,(H+2KV)hd] = [q|k|v] heads);
     with caches [B,Lmax,KV,hd], the turned keys and the values go to slots pos0 .. pos0+T-1."""
     B, T, d = x.shape
+    if H < 1 or KV < 1 or Wqkv.dim() != 2 or Wqkv.shape[1] % (H + 2 * KV):
+        raise ValueError(f"Wqkv must be [d, (H+2KV)*hd] with H={H}, KV={KV}, got {tuple(Wqkv.shape)}")
     hd = Wqkv.shape[1] // (H + 2 * KV)
+    _shape(Wqkv, (d, (H + 2 * KV) * hd), "Wqkv")
+    _shape(Wo, (H * hd, d), "Wo")
+    _shape(gamma, (d,), "gamma")
+    _shape(out, x.shape, "out")
+    if (kcache is None) != (vcache is None):
+        raise ValueError("give both kcache and vcache, or neither")
+    if kcache is not None:
+        if kcache.dim() != 4:
+            raise ValueError(f"kcache must be [B,Lmax,KV,hd], got {tuple(kcache.shape)}")
+        _shape(kcache, (B, kcache.shape[1], KV, hd), "kcache")
+        _shape(vcache, kcache.shape, "vcache")
     dt = x.dtype
     if out is None:
         out = torch.empty_like(x)

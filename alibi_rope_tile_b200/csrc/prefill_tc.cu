@@ -61,21 +61,6 @@ constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;  // own copies/MMAs finish in 
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
-#ifdef ATTN_TRACE
-// Diagnostic build only: SM-clock stamps of pipeline events of one CTA, 16 lanes x 2048.
-__device__ long long g_attn_trace[16][2048];
-#define TRACE(lane_id, counter, tag)                                                      \
-  do {                                                                                    \
-    if (blockIdx.x == ATTN_TRACE && (counter) < 2048)                                     \
-      g_attn_trace[lane_id][(counter)++] = (clock64() << 8) | (long long)(tag);           \
-  } while (0)
-#else
-#define TRACE(lane_id, counter, tag) \
-  do {                               \
-    (void)(counter);                 \
-  } while (0)
-#endif
-
 template <int HD>
 struct Cfg {
   static constexpr int NS = HD == 128 ? 4 : 10;  // key/value ring stages
@@ -327,13 +312,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (valid[s])
           for (int kb = 0; kb < HD / 64; ++kb)
             tma_load_4d(sQ + s * C::Q_BYTES + kb * BM * 128, &tmQ, q_full, kb * 64, head[s], qs[s], b);
-      int tcnt = 0;
       const int total = 2 * (jt1 - jt0 + 1);  // K and V of every tile
       int u = 0;
       for (; u < total; ++u) {
         const int st = u % C::NS, n = u / C::NS, j = jt0 + u / 2, kv = u & 1;
         if (!mbar_wait(kv_empty + st, (n & 1) ^ 1, abort_flag, p.status, WAIT_LIMIT_NS)) break;
-        TRACE(4, tcnt, 30 + kv);
         mbar_expect_tx(kv_full + st, C::KV_BYTES);
         for (int kb = 0; kb < HD / 64; ++kb)
           tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, kv ? &tmV : &tmK, kv_full + st,
@@ -360,12 +343,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // tile, and registers are tighter) computes each accurately
     if constexpr (HD == 128)
       if (p.rope.on && !CHUNK) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
-    int u = 0, tcnt = 0;
+    int u = 0;
     for (int j = jt0; j <= jt1; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++u) {
         const int st = u % C::NS, n = u / C::NS;
         if (!mbar_wait(kv_full + st, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        if (tid == WARP_ROPE0 * 32) TRACE(3, tcnt, 20 + kv);
         if (kv == 0 && p.rope.on && !CHUNK) {  // cached keys are already rotated
           if constexpr (HD == 128)
             krot.rotate_next(sKV + st * C::KV_BYTES);
@@ -374,7 +356,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         fence_proxy_async();
         mbar_arrive(k_rot + st);
-        if (tid == WARP_ROPE0 * 32) TRACE(3, tcnt, 22);
       }
     }
   } else if (warp == WARP_MMA) {
@@ -385,7 +366,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t dQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
       const uint64_t dV = smem_desc_sw128(smem_u32(sKV), BN * 128, 1024);
-      int tcnt = 0;
       auto issue_qk = [&](int s, int st) {
         const uint32_t d = tmem + s * BN;
         const uint64_t a0 = dQ + (uint64_t)((s * C::Q_BYTES) >> 4);
@@ -404,7 +384,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kk = 0; kk < BN / 16; ++kk) {
           umma_ts(d, aP + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
                   (kk > 0 || acc) ? 1u : 0u);
-          if (kk == 0 || kk == 3) TRACE(0, tcnt, 40 + kk);
         }
       };
       int cnt[2] = {0, 0};
@@ -424,26 +403,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int uK = uV + 1, stK = uK % C::NS;
         const bool next = j < jt1;
         if (!mbar_wait(k_rot + stV, (uV / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
-        TRACE(0, tcnt, 8);
         for (int s = 0; s < 2; ++s) {
           if (active(s, j)) {
             if (!mbar_wait(p_full + s, cnt[s] & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
-            TRACE(0, tcnt, 1 + 4 * s);
             tc_fence_after();
             issue_pv(s, stV, cnt[s] > 0);
             umma_commit(o_done + s);
             ++cnt[s];
-            TRACE(0, tcnt, 2 + 4 * s);
           }
           if (next && s == 0) {
             if (!mbar_wait(k_rot + stK, (uK / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
-            TRACE(0, tcnt, 3);
             tc_fence_after();
           }
           if (next && active(s, j + 1)) {
             issue_qk(s, stK);
             umma_commit(s_full + s);
-            TRACE(0, tcnt, 4 + 4 * s);
           }
         }
         umma_commit(kv_empty + stV);
@@ -476,8 +450,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // share of the weights. The reference moves only when a tile's maximum exceeds it by
     // more than 8 (a factor 256), so O is rescaled rarely; weights stay below 2^8.
     float m_ref0 = -INFINITY, m_ref1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    int cs0 = 0, cs1 = 0, t = 0, tcnt = 0;
-    const bool tracer = warp == 0 && lane == 0;
+    int cs0 = 0, cs1 = 0, t = 0;
 #pragma unroll 1
     for (int j = jt0; j <= jt1; ++j) {
 #pragma unroll 1
@@ -487,7 +460,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int c = s ? cs1 : cs0;
         float m_ref = s ? m_ref1 : m_ref0;
         if (!mbar_wait(s_full + s, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        if (tracer) TRACE(1 + s, tcnt, 10);
         tc_fence_after();
         const int q0s = qs[s];  // first query row of the slot
         const int hs = head[s];
@@ -532,7 +504,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float alpha = (m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
         m_ref = m_new;
-        if (tracer) TRACE(1 + s, tcnt, 11);
         f2x RS = pk2(0.f, 0.f);
         uint32_t pk[16];  // column k: keys 2k, 2k+1 of my 32 (low half = even key)
         if (plain) {
@@ -591,7 +562,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full + s);
-        if (tracer) TRACE(1 + s, tcnt, 14);
         ++t;
       }
     }
@@ -654,21 +624,6 @@ done:
 }
 
 // ---------------------------------------------------------------- host side
-#ifdef ATTN_TRACE
-}  // namespace
-}  // namespace tc
-}  // namespace attn
-extern "C" int attn_trace_read(long long* host) {
-  return (int)cudaMemcpyFromSymbol(host, attn::tc::g_attn_trace, sizeof(attn::tc::g_attn_trace));
-}
-extern "C" int attn_trace_clear() {
-  static long long zeros[16][2048];
-  return (int)cudaMemcpyToSymbol(attn::tc::g_attn_trace, zeros, sizeof(zeros));
-}
-namespace attn {
-namespace tc {
-namespace {
-#endif
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;

@@ -1,28 +1,34 @@
-"""Benchmark of the attention core on B200: causal GQA prefill TFLOP/s and decode HBM GB/s.
+"""Benchmark of the attention core on B200: causal prefill TFLOP/s and decode HBM GB/s, each
+against its roofline.
 
-One step = one pass of the whole hot path over one batch of synthetic input:
-  * prefill of the GQA workload (B=2, T=4096, H=32, KV=8, hd=128, causal, RoPE base 5e5):
-    RoPE on load, QK^T, mask, online softmax, PV, epilogue;
-  * one decode step of the KV-cache workload (batch 64, H=32, KV=8, hd=128, cache lengths
-    uniform in [1024, 8192]) and of its MQA variant (KV=1): split-KV partials and the
-    log-sum-exp merge;
-  * one pass of the bf16 block around the same attention shape (x [2,4096,4096], weights
-    resident): the x@Wq, x@Wk, x@Wv projections, the attention core, then ctx@Wo;
-  * a chunked prefill: the second 2048 rows of the GQA sequences against a cache of their
-    4096 rotated keys (written once, before timing).
-``value`` is the prefill TFLOP/s (causal FLOPs counted: 4*B*H*hd*allowed pairs); the decode
-GB/s (cache rows read + q + out, per launch pair) ride along under ``decode``, the block's
-TFLOP/s (projection FLOPs 2*M*N*K plus the attention's) under ``block``, the chunk's under
-``chunk``. Kernels are timed with CUDA events on the stream they
-are launched on; L2 is flushed (a 256 MiB memset, outside the timed events) before every
-step. ``e2e`` times the same call with the step's inputs copied from pinned host memory and
-its output copied back, all inside the timed region.
+One step = one pass of the whole hot path over one batch of synthetic input of every workload
+the attention core is specified on, plus the library's wider entry points:
+  * gqa_prefill   B=2, T=4096, H=32, KV=8, hd=128, causal, RoPE base 5e5 (the headline);
+  * mha_rope      B=4, T=1024, H=KV=16, hd=64, causal, RoPE base 1e4;
+  * mha_alibi     the same shape with no rotation and the ALiBi bias 2^(-8(h+1)/H)(j - i);
+  * long_window   B=1, T=16384, H=32, KV=8, hd=128, causal + window 4096, RoPE base 1e4;
+  * decode_kv8 / decode_mqa   one decode step of 64 sequences, H=32, KV=8 (or 1), hd=128,
+    cache lengths uniform in [1024, 8192]: the split pass and the log-sum-exp merge;
+  * decode_kv8_paged16   the KV=8 decode over the same cache as shuffled 16-row pages;
+  * latent_decode  B=64, H=32, hd=128, latent width 128, lengths U[1024, 8192];
+  * chunk          the second 2048 rows of the GQA sequences over a cache of their 4096 keys;
+  * block / block_fused   the bf16 block around the GQA attention (x [2,4096,4096], d 4096),
+    plain and as the fused pre-norm sub-layer.
+Prefill FLOPs count the allowed (causal / window) pairs only: 4*B*H*hd*pairs. Decode bytes are
+the cache rows read plus q and out. Kernels are timed with CUDA events on the stream they are
+launched on. L2 (126 MB) is flushed with a 256 MiB memset, outside the events, before every
+family, except for the two MHA variants: their inputs (34 MB) are far smaller than L2, so each
+step runs them back to back over ten copies of the inputs (336 MB, more than twice L2, so every
+launch reads inputs that left L2 since their last use) between one pair of events; a flushed
+single launch of each is timed as well (``ms_single``).
+``value`` is the GQA prefill's TFLOP/s; ``e2e`` is the same prefill through the public API with
+q, k, v copied in from pinned host memory and out copied back inside the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-With N > 1 (launched by torchrun) every rank runs its own replica of the step (the path
-shards into independent problems; there is no data-path collective): value = all ranks'
-FLOPs / the slowest rank's time.
+With N > 1 (launched by torchrun) every rank runs its own replica of the step (the path shards
+into independent problems; there is no data-path collective): value = all ranks' FLOPs / the
+slowest rank's time.
 """
 from __future__ import annotations
 
@@ -45,20 +51,10 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "source": "fallback"}
 METRIC = "causal GQA prefill TFLOP/s and decode HBM GB/s on 1 B200, % of roofline"
 PREFILL = workloads.GQA
-DECODE = workloads.DECODE_GQA
-DECODE_MQA = workloads.DECODE_MQA
-BLOCK = workloads.GQA_BLOCK
-CHUNK = workloads.GQA_CHUNK
-LATENT = workloads.LATENT_DECODE
-# Algorithmic bytes and launches, stated once (see the design notes):
-#   decode bytes = cache rows read (K and V) + q + out; prefill FLOPs = PREFILL.flops.
-PREFILL_LAUNCHES = 1
-DECODE_LAUNCHES = 2       # split pass + merge, per decode workload
 PAGE_SIZE = 16            # rows per page of the paged decode (the KV=8 decode workload, pages shuffled)
-BLOCK_LAUNCHES = 5        # three projection GEMMs, the prefill, the output GEMM
-CHUNK_LAUNCHES = 1
-LATENT_LAUNCHES = 4       # the fold, the split pass, the merge, the value up-projection
-FUSED_LAUNCHES = 5        # RoPE table, RMSNorm, QKV GEMM (+ rotation, cache write), prefill, Wo GEMM (+ residual)
+MHA_COPIES = 10           # input copies the MHA variants rotate over (10 x 33.6 MB > 2 x L2)
+L2_NOTE = ("flushed: 256 MiB memset before every family, outside the events; the MHA variants "
+           "rotate over 10 input copies (336 MB) back to back instead")
 
 
 def peaks():
@@ -83,8 +79,8 @@ def csrc_sha256() -> str:
 
 
 def measured_traffic() -> dict:
-    """Per-launch DRAM bytes (read + write) from profiles/traffic.json, or {} when the file
-    was written for different kernel sources."""
+    """Per-launch DRAM bytes (read + write) of each family's dominant kernel from
+    profiles/traffic.json, or {} when the file was written for different kernel sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return {}
@@ -134,6 +130,11 @@ def max_over_ranks(x: float, world, device: str = "cuda") -> float:
 def aggregate_rate(units_per_rank: float, world: int, slowest_ms: float) -> float:
     """Whole-job rate: the units all ranks processed over the slowest rank's time (ms)."""
     return world * units_per_rank / (slowest_ms * 1e-3)
+
+
+def base_config(world: int) -> dict:
+    """The configuration both arms report (the headline workload and how it is run)."""
+    return {"workload": PREFILL.name, "parallelism": f"replicas{world}", "l2": L2_NOTE}
 
 
 class Clocks:
@@ -188,48 +189,62 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample_tflops(budget_s: float = 12.0):
-    """The fp64 oracle on a bounded sample of the prefill workload, as TFLOP/s of causal
-    FLOPs: sequence 0, one key/value group (4 query heads) at a time, all 4096 rows, until
-    the time budget is spent (about 1 s per group on 16 cores)."""
+_HOST_INPUTS = []
+
+
+def _prefill_host_inputs():
+    """The headline workload's q, k, v on the host (drawn once)."""
+    if not _HOST_INPUTS:
+        _HOST_INPUTS.extend(workloads.prefill_inputs(PREFILL))
+    return _HOST_INPUTS
+
+
+def oracle_groups(groups) -> tuple:
+    """The fp64 oracle on sequence 0 of the GQA prefill for the given key/value groups (4 query
+    heads each, all 4096 rows): returns (causal FLOPs done, seconds)."""
     from oracle import attention as A
     w = PREFILL
-    q, k, v = workloads.prefill_inputs(w)
+    q, k, v = _prefill_host_inputs()
     group = w.H // w.KV
     pairs = w.T * (w.T + 1) // 2
-    flops = done = 0
     t0 = time.perf_counter()
-    for g in range(w.KV):
-        if time.perf_counter() - t0 >= budget_s:
-            break
+    for g in groups:
         A.attention(q[:1, :, g * group:(g + 1) * group], k[:1, :, g:g + 1], v[:1, :, g:g + 1],
                     rope_base=w.rope_base, causal=True)
-        flops += 4 * group * w.hd * pairs
-        done += 1
     dt = time.perf_counter() - t0
-    sample = (f"GQA prefill, sequence 0, {done} of {w.KV} key/value groups ({done * group} of "
-              f"{w.H} query heads), all {w.T} rows, fp64 numpy/OpenBLAS")
-    return flops / dt / 1e12, dt, sample
+    return 4 * group * w.hd * pairs * len(groups), dt
+
+
+SAMPLE = ("GQA prefill (B=2, T=4096, H=32, KV=8, hd=128, RoPE 5e5): sequence 0, {n} key/value "
+          "group(s) of 4 query heads, all 4096 rows, fp64 numpy/OpenBLAS")
+
+
+def cpu_baseline():
+    """The oracle on a bounded sample of the headline workload: all 8 groups of sequence 0."""
+    flops, dt = oracle_groups(range(PREFILL.KV))
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": SAMPLE.format(n=PREFILL.KV), "seconds": round(dt, 2)}
 
 
 def run_reference(args, rank, world):
-    """Reference arm: the fp64 CPU oracle, as it stands, on the host cores (rank 0 only)."""
+    """Reference arm: the fp64 CPU oracle, as it stands, on the host cores (rank 0 only); each
+    step is one key/value group of sequence 0 of the headline workload (groups in turn)."""
     if rank != 0:
         return
-    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
-    for _ in range(args.warmup):
-        oracle_sample_tflops(min(per_step, 3.0))
-    vals, secs, sample = [], 0.0, ""
-    for _ in range(args.steps):
-        v, dt, sample = oracle_sample_tflops(per_step)
-        vals.append(v)
+    for s in range(args.warmup):
+        oracle_groups([s % PREFILL.KV])
+    flops = secs = 0.0
+    for s in range(args.steps):
+        f, dt = oracle_groups([s % PREFILL.KV])
+        flops += f
         secs += dt
-    value = statistics.median(vals)
+    value = flops / secs / 1e12
+    sample = SAMPLE.format(n=1) + " per step, groups in turn"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * secs / max(1, args.steps), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": PREFILL.name, "sample": sample},
+            "config": base_config(world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -237,389 +252,347 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------------------------ families
+class Family:
+    """One workload of the step: how to run it, what it computes, how it is timed."""
+
+    def __init__(self, key, workload, unit, bound, work, launches, kernel, run, reps=1,
+                 e2e=None, note=None):
+        self.key, self.workload, self.unit, self.bound = key, workload, unit, bound
+        self.work = work              # FLOPs or bytes of one run
+        self.launches = launches      # kernel launches of one run
+        self.kernel = kernel          # the dominant kernel
+        self.run = run                # run(i): one run on input copy i
+        self.reps = reps              # runs per timed bracket (1: flushed before)
+        self.e2e = e2e                # (h2d bytes, d2h bytes, step()) through host buffers
+        self.note = note
+
+
+def tnb(t):
+    return t.numel() * t.element_size()
+
+
+def build_families(art, only):
+    dev = "cuda"
+    fams = []
+    want = (lambda k: True) if only is None else (lambda k: k in only)
+
+    def prefill_family(key, w, copies=1):
+        q, k, v = workloads.prefill_inputs(w)
+        slopes = art.alibi_slopes(w.H) if w.alibi else None
+        ins = [(q.to(dev), k.to(dev), v.to(dev)) for _ in range(copies)]
+        outs = [torch.empty(q.shape, dtype=q.dtype, device=dev) for _ in range(copies)]
+
+        def run(i=0):
+            dq, dk, dv = ins[i % copies]
+            art.attn_prefill(dq, dk, dv, outs[i % copies], rope_base=w.rope_base, causal=w.causal,
+                             window=w.window, alibi_slopes=slopes, pos0=w.pos0)
+
+        hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+        hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+
+        def e2e_step():
+            dq, dk, dv = ins[0]
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            run(0)
+            hout.copy_(outs[0], non_blocking=True)
+
+        kern = f"prefill_tc_kernel<{w.hd}, false>"
+        return Family(key, w.name, "TFLOP/s", "tensor", w.flops, 1, kern, run, reps=copies,
+                      e2e=(tnb(q) + tnb(k) + tnb(v), tnb(q), e2e_step))
+
+    if want("gqa_prefill"):
+        fams.append(prefill_family("gqa_prefill", PREFILL))
+    if want("mha_rope"):
+        fams.append(prefill_family("mha_rope", workloads.MHA_ROPE, MHA_COPIES))
+    if want("mha_alibi"):
+        fams.append(prefill_family("mha_alibi", workloads.MHA_ALIBI, MHA_COPIES))
+    if want("long_window"):
+        fams.append(prefill_family("long_window", workloads.LONG_WINDOW))
+
+    def decode_family(key, dw, paged):
+        hq, hkc, hvc, hsl, hqp = workloads.decode_inputs(dw)
+        d = dict(q=hq.to(dev), kc=hkc.to(dev), vc=hvc.to(dev), sl=hsl.to(dev), qp=hqp.to(dev),
+                 out=torch.empty(hq.shape, dtype=hq.dtype, device=dev),
+                 ws=torch.empty(art.attn_decode_workspace_size(dw.B, dw.H, dw.KV, dw.hd, dw.Lmax),
+                                dtype=torch.uint8, device=dev))
+        del hkc, hvc
+        if paged:
+            # the same cache as a shuffled pool of 16-row pages behind a block table
+            mb = dw.Lmax // PAGE_SIZE
+            g = torch.Generator().manual_seed(dw.seed + 100)
+            order = torch.randperm(dw.B * mb, generator=g).to(torch.int32).reshape(dw.B, mb)
+            kp = torch.zeros(dw.B * mb, PAGE_SIZE, dw.KV, dw.hd, dtype=torch.bfloat16, device=dev)
+            vp = torch.zeros_like(kp)
+            d["table"] = order.to(dev)
+            zero = torch.zeros(dw.B, dtype=torch.int32, device=dev)
+            art.attn_kv_write_paged(d["kc"], d["vc"], kp, vp, d["table"], zero, rope_base=0.0)
+            del d["kc"], d["vc"]
+            d["kp"], d["vp"] = kp, vp
+
+            def run(i=0):
+                art.attn_decode_paged(d["q"], d["kp"], d["vp"], d["table"], d["sl"], d["qp"], d["out"],
+                                      workspace=d["ws"], rope_base=dw.rope_base)
+        else:
+            def run(i=0):
+                art.attn_decode(d["q"], d["kc"], d["vc"], d["sl"], d["qp"], d["out"], workspace=d["ws"],
+                                rope_base=dw.rope_base)
+        hqq = hq.pin_memory()
+        hout = torch.empty(hq.shape, dtype=hq.dtype).pin_memory()
+
+        def e2e_step():
+            d["q"].copy_(hqq, non_blocking=True)
+            run(0)
+            hout.copy_(d["out"], non_blocking=True)
+
+        return Family(key, dw.name + (f"_paged{PAGE_SIZE}" if paged else ""), "GB/s", "hbm",
+                      decode_bytes(hsl, dw), 2, "decode_tc_kernel<128>", run,
+                      e2e=(tnb(hq), tnb(hq), e2e_step))
+
+    if want("decode_kv8"):
+        fams.append(decode_family("decode_kv8", workloads.DECODE_GQA, False))
+    if want("decode_mqa"):
+        fams.append(decode_family("decode_mqa", workloads.DECODE_MQA, False))
+    if want("decode_kv8_paged16"):
+        fams.append(decode_family("decode_kv8_paged16", workloads.DECODE_GQA, True))
+
+    if want("latent_decode"):
+        lw = workloads.LATENT_DECODE
+        lq, lc, luk, luv, lsl = workloads.latent_inputs(lw)
+        L = dict(q=lq.to(dev), c=lc.to(dev), uk=luk.to(dev), uv=luv.to(dev), sl=lsl.to(dev),
+                 out=torch.empty(lq.shape, dtype=lq.dtype, device=dev),
+                 ws=torch.empty(int(art.lib().attn_decode_latent_workspace_size(lw.B, lw.H, lw.hd, lw.dc,
+                                                                                lw.Lmax)),
+                                dtype=torch.uint8, device=dev))
+        del lc
+
+        def run_lat(i=0):
+            art.attn_decode_latent(L["q"], L["c"], L["uk"], L["uv"], L["sl"], L["sl"], L["out"],
+                                   workspace=L["ws"])
+        hlq = lq.pin_memory()
+        hlo = torch.empty(lq.shape, dtype=lq.dtype).pin_memory()
+
+        def e2e_lat():
+            L["q"].copy_(hlq, non_blocking=True)
+            run_lat(0)
+            hlo.copy_(L["out"], non_blocking=True)
+        # algorithmic bytes: each latent row read once, q and out, both weights
+        lbytes = int(lsl.sum()) * lw.dc * 2 + 2 * lw.B * lw.H * lw.hd * 2 + 2 * lw.H * lw.dc * lw.hd * 2
+        fams.append(Family("latent_decode", lw.name, "GB/s", "hbm", lbytes, LATENT_LAUNCHES,
+                           "decode_tc_kernel<128>", run_lat, e2e=(tnb(lq), tnb(lq), e2e_lat)))
+
+    if want("chunk"):
+        cw = workloads.GQA_CHUNK
+        hcq, hck, hcv = workloads.chunk_inputs(cw)
+        ckc = torch.zeros(cw.B, cw.Lmax, cw.KV, cw.hd, dtype=torch.bfloat16, device=dev)
+        cvc = torch.zeros_like(ckc)
+        art.attn_kv_write(hck.to(dev), hcv.to(dev), ckc, cvc,
+                          torch.zeros(cw.B, dtype=torch.int32, device=dev), rope_base=cw.rope_base)
+        C = dict(q=hcq.to(dev), kc=ckc, vc=cvc,
+                 sl=torch.full((cw.B,), cw.qpos0 + cw.Tq, dtype=torch.int32, device=dev),
+                 qp=torch.full((cw.B,), cw.qpos0, dtype=torch.int32, device=dev),
+                 out=torch.empty(hcq.shape, dtype=hcq.dtype, device=dev))
+
+        def run_chunk(i=0):
+            art.attn_prefill_chunk(C["q"], C["kc"], C["vc"], C["sl"], C["qp"], C["out"], rope_base=cw.rope_base)
+        hq = hcq.pin_memory()
+        ho = torch.empty(hcq.shape, dtype=hcq.dtype).pin_memory()
+
+        def e2e_chunk():
+            C["q"].copy_(hq, non_blocking=True)
+            run_chunk(0)
+            ho.copy_(C["out"], non_blocking=True)
+        fams.append(Family("chunk", cw.name, "TFLOP/s", "tensor", cw.flops, 1, "prefill_tc_kernel<128, true>",
+                           run_chunk, e2e=(tnb(hcq), tnb(hcq), e2e_chunk)))
+
+    if want("block") or want("block_fused"):
+        bw = workloads.GQA_BLOCK
+        hx, hW = workloads.block_inputs(bw)
+        X = dict(x=hx.to(dev), W={n: t.to(dev) for n, t in hW.items()},
+                 out=torch.empty(hx.shape, dtype=hx.dtype, device=dev))
+        hxp = hx.pin_memory()
+        ho = torch.empty(hx.shape, dtype=hx.dtype).pin_memory()
+        if want("block"):
+            X["ws"] = torch.empty(art.attn_block_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV, bw.hd,
+                                                                torch.bfloat16), dtype=torch.uint8, device=dev)
+
+            def run_block(i=0):
+                W = X["W"]
+                art.attn_block(X["x"], W["Wq"], W["Wk"], W["Wv"], W["Wo"], X["out"], workspace=X["ws"],
+                               H=bw.H, KV=bw.KV, rope_base=bw.rope_base, causal=bw.causal, window=bw.window)
+
+            def e2e_block():
+                X["x"].copy_(hxp, non_blocking=True)
+                run_block(0)
+                ho.copy_(X["out"], non_blocking=True)
+            fams.append(Family("block", bw.name, "TFLOP/s", "tensor", bw.flops, BLOCK_LAUNCHES,
+                               "gemm_tc_kernel", run_block, e2e=(tnb(hx), tnb(hx), e2e_block),
+                               note="projection FLOPs 2*M*N*K plus the attention's; weights resident"))
+        if want("block_fused"):
+            # the same block as a fused pre-norm sub-layer: RMSNorm, one Wqkv, cache write, residual
+            F = dict(gamma=torch.ones(bw.d, dtype=torch.bfloat16, device=dev),
+                     Wqkv=torch.cat([X["W"]["Wq"], X["W"]["Wk"], X["W"]["Wv"]], dim=1).contiguous(),
+                     kc=torch.zeros(bw.B, bw.T, bw.KV, bw.hd, dtype=torch.bfloat16, device=dev),
+                     out=torch.empty(hx.shape, dtype=hx.dtype, device=dev),
+                     ws=torch.empty(int(art.lib().attn_block_fused_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV,
+                                                                                  bw.hd)),
+                                    dtype=torch.uint8, device=dev))
+            F["vc"] = torch.zeros_like(F["kc"])
+
+            def run_fused(i=0):
+                art.attn_block_fused(X["x"], F["gamma"], F["Wqkv"], X["W"]["Wo"], F["out"], F["kc"], F["vc"],
+                                     F["ws"], H=bw.H, KV=bw.KV, rope_base=bw.rope_base, causal=bw.causal,
+                                     window=bw.window)
+
+            def e2e_fused():
+                X["x"].copy_(hxp, non_blocking=True)
+                run_fused(0)
+                ho.copy_(F["out"], non_blocking=True)
+            fams.append(Family("block_fused", bw.name + "_prenorm", "TFLOP/s", "tensor", bw.flops,
+                               FUSED_LAUNCHES, "gemm_tc_kernel", run_fused, e2e=(tnb(hx), tnb(hx), e2e_fused),
+                               note="RMSNorm, one QKV GEMM (RoPE and cache write in its epilogue), "
+                                    "attention, Wo GEMM + residual"))
+    return fams
+
+
+# kernel launches of one run of the multi-launch families
+LATENT_LAUNCHES = 4       # the fold, the split pass, the merge, the value up-projection
+BLOCK_LAUNCHES = 5        # three projection GEMMs, the prefill, the output GEMM
+FUSED_LAUNCHES = 5        # RoPE table, RMSNorm, QKV GEMM (+ rotation, cache write), prefill, Wo GEMM (+ residual)
+
+
 def run_ours(args, rank, world):
     import alibi_rope_tile_b200 as art
     art.lib()
     dev = torch.cuda.current_device()
     stream = torch.cuda.current_stream()
-    w = PREFILL
-    do_p, do_d = args.only in ("all", "prefill"), args.only in ("all", "decode")
-    do_b = args.only in ("all", "block")
-    do_c = args.only in ("all", "chunk")
-
-    q, k, v = workloads.prefill_inputs(w)
-    dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
-    dout = torch.empty_like(dq)
-    decs = []
-    paged = None
-    lat = None
-    if do_d:
-        for dw in (DECODE, DECODE_MQA):
-            hq, hkc, hvc, hsl, hqp = workloads.decode_inputs(dw)
-            decs.append(dict(
-                w=dw, bytes=decode_bytes(hsl, dw), hq=hq,
-                q=hq.cuda(), kc=hkc.cuda(), vc=hvc.cuda(), sl=hsl.cuda(), qp=hqp.cuda(),
-                out=torch.empty(hq.shape, dtype=hq.dtype, device="cuda"),
-                ws=torch.empty(art.attn_decode_workspace_size(dw.B, dw.H, dw.KV, dw.hd, dw.Lmax),
-                               dtype=torch.uint8, device="cuda")))
-            if dw is DECODE:
-                # the same cache as a shuffled pool of 16-row pages behind a block table
-                mb = dw.Lmax // PAGE_SIZE
-                need = [mb] * dw.B  # every slot has a page (those past a length are never read)
-                g = torch.Generator().manual_seed(dw.seed + 100)
-                order = torch.randperm(sum(need), generator=g)
-                table = torch.full((dw.B, mb), -1, dtype=torch.int32)
-                at = 0
-                for b in range(dw.B):
-                    table[b, :need[b]] = order[at:at + need[b]].to(torch.int32)
-                    at += need[b]
-                kp = torch.zeros(sum(need), PAGE_SIZE, dw.KV, dw.hd, dtype=hkc.dtype, device="cuda")
-                vp = torch.zeros_like(kp)
-                dtab = table.cuda()
-                zero = torch.zeros(dw.B, dtype=torch.int32, device="cuda")
-                art.attn_kv_write_paged(decs[-1]["kc"], decs[-1]["vc"], kp, vp, dtab, zero, rope_base=0.0)
-                paged = dict(w=dw, bytes=decs[-1]["bytes"], q=decs[-1]["q"], sl=decs[-1]["sl"],
-                             qp=decs[-1]["qp"], kp=kp, vp=vp, table=dtab,
-                             out=torch.empty_like(decs[-1]["out"]),
-                             ws=torch.empty_like(decs[-1]["ws"]))
-            del hkc, hvc
-        lw = LATENT
-        lq, lc, luk, luv, lsl = workloads.latent_inputs(lw)
-        lat = dict(w=lw, hq=lq, q=lq.cuda(), c=lc.cuda(), uk=luk.cuda(), uv=luv.cuda(), sl=lsl.cuda(),
-                   out=torch.empty(lq.shape, dtype=lq.dtype, device="cuda"),
-                   ws=torch.empty(int(art.lib().attn_decode_latent_workspace_size(lw.B, lw.H, lw.hd, lw.dc,
-                                                                                  lw.Lmax)),
-                                  dtype=torch.uint8, device="cuda"),
-                   # algorithmic bytes: each latent row read once, q and out, both weights
-                   bytes=int(lsl.sum()) * lw.dc * 2 + 2 * lw.B * lw.H * lw.hd * 2
-                   + 2 * lw.H * lw.dc * lw.hd * 2)
-        del lc
-    blk = None
-    if do_b:
-        bw = BLOCK
-        hx, hW = workloads.block_inputs(bw)
-        blk = dict(w=bw, hx=hx, x=hx.cuda(), W={n: t.cuda() for n, t in hW.items()},
-                   out=torch.empty(hx.shape, dtype=hx.dtype, device="cuda"),
-                   ws=torch.empty(art.attn_block_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV, bw.hd,
-                                                                 torch.bfloat16),
-                                  dtype=torch.uint8, device="cuda"))
-        # the same block as a fused pre-norm sub-layer: RMSNorm, one Wqkv, cache write, residual
-        fz = dict(gamma=torch.ones(bw.d, dtype=torch.bfloat16, device="cuda"),
-                  Wqkv=torch.cat([blk["W"]["Wq"], blk["W"]["Wk"], blk["W"]["Wv"]], dim=1).contiguous(),
-                  kc=torch.zeros(bw.B, bw.T, bw.KV, bw.hd, dtype=torch.bfloat16, device="cuda"),
-                  out=torch.empty_like(blk["out"]),
-                  ws=torch.empty(int(art.lib().attn_block_fused_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV,
-                                                                               bw.hd)),
-                                 dtype=torch.uint8, device="cuda"))
-        fz["vc"] = torch.zeros_like(fz["kc"])
-        blk["fused"] = fz
-        del hW
-    chk = None
-    if do_c:
-        cw = CHUNK
-        hcq, hck, hcv = workloads.chunk_inputs(cw)
-        ckc = torch.zeros(cw.B, cw.Lmax, cw.KV, cw.hd, dtype=torch.bfloat16, device="cuda")
-        cvc = torch.zeros_like(ckc)
-        art.attn_kv_write(hck.cuda(), hcv.cuda(), ckc, cvc,
-                          torch.zeros(cw.B, dtype=torch.int32, device="cuda"), rope_base=cw.rope_base)
-        chk = dict(w=cw, hq=hcq, q=hcq.cuda(), kc=ckc, vc=cvc,
-                   sl=torch.full((cw.B,), cw.qpos0 + cw.Tq, dtype=torch.int32, device="cuda"),
-                   qp=torch.full((cw.B,), cw.qpos0, dtype=torch.int32, device="cuda"),
-                   out=torch.empty(hcq.shape, dtype=hcq.dtype, device="cuda"))
-        del hck, hcv
+    only = None if args.only == "all" else set(args.only.split(","))
+    fams = build_families(art, only)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
-    def prefill():
-        if do_p:
-            art.attn_prefill(dq, dk, dv, dout, rope_base=w.rope_base, causal=True, window=w.window)
-
-    def decode(d):
-        art.attn_decode(d["q"], d["kc"], d["vc"], d["sl"], d["qp"], d["out"], workspace=d["ws"],
-                        rope_base=d["w"].rope_base)
-
-    def block():
-        if blk is not None:
-            bw, W = blk["w"], blk["W"]
-            art.attn_block(blk["x"], W["Wq"], W["Wk"], W["Wv"], W["Wo"], blk["out"],
-                           workspace=blk["ws"], H=bw.H, KV=bw.KV, rope_base=bw.rope_base,
-                           causal=bw.causal, window=bw.window)
-
-    def decode_paged():
-        if paged is not None:
-            art.attn_decode_paged(paged["q"], paged["kp"], paged["vp"], paged["table"], paged["sl"],
-                                  paged["qp"], paged["out"], workspace=paged["ws"],
-                                  rope_base=paged["w"].rope_base)
-
-    def block_fused():
-        if blk is not None:
-            bw, fz = blk["w"], blk["fused"]
-            art.attn_block_fused(blk["x"], fz["gamma"], fz["Wqkv"], blk["W"]["Wo"], fz["out"], fz["kc"], fz["vc"],
-                                 fz["ws"], H=bw.H, KV=bw.KV, rope_base=bw.rope_base, causal=bw.causal,
-                                 window=bw.window)
-
-    def decode_latent():
-        if lat is not None:
-            art.attn_decode_latent(lat["q"], lat["c"], lat["uk"], lat["uv"], lat["sl"], lat["sl"], lat["out"],
-                                   workspace=lat["ws"])
-
-    def chunk():
-        if chk is not None:
-            art.attn_prefill_chunk(chk["q"], chk["kc"], chk["vc"], chk["sl"], chk["qp"], chk["out"],
-                                   rope_base=chk["w"].rope_base)
-
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
-        prefill()
-        for d in decs:
-            decode(d)
-        block()
-        chunk()
-        decode_paged()
-        decode_latent()
-        block_fused()
+        for f in fams:
+            flush.zero_()
+            for r in range(f.reps):
+                f.run(r)
     torch.cuda.synchronize()
     art.attn_sync_status()
 
-    nev = 2 + 2 * len(decs) + 10
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    def evpair():
+        return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    ev = [{f.key: (evpair(), evpair() if f.reps > 1 else None) for f in fams} for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     clocks = Clocks(dev)
     time.sleep(0.3)
-    t_begin = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
+    t_begin, t_end = evpair()
     t_begin.record(stream)
     for s_ in range(args.steps):
-        flush.zero_()
-        ev[s_][0].record(stream)
-        prefill()
-        ev[s_][1].record(stream)
-        for n, d in enumerate(decs):
-            flush.zero_()
-            ev[s_][2 + 2 * n].record(stream)
-            decode(d)
-            ev[s_][3 + 2 * n].record(stream)
-        flush.zero_()
-        ev[s_][nev - 10].record(stream)
-        block_fused()
-        ev[s_][nev - 9].record(stream)
-        flush.zero_()
-        ev[s_][nev - 8].record(stream)
-        decode_latent()
-        ev[s_][nev - 7].record(stream)
-        flush.zero_()
-        ev[s_][nev - 6].record(stream)
-        block()
-        ev[s_][nev - 5].record(stream)
-        flush.zero_()
-        ev[s_][nev - 4].record(stream)
-        chunk()
-        ev[s_][nev - 3].record(stream)
-        flush.zero_()
-        ev[s_][nev - 2].record(stream)
-        decode_paged()
-        ev[s_][nev - 1].record(stream)
+        for f in fams:
+            (e0, e1), single = ev[s_][f.key]
+            if f.reps == 1:
+                flush.zero_()
+            e0.record(stream)
+            for r in range(f.reps):
+                f.run(r)
+            e1.record(stream)
+            if single is not None:
+                flush.zero_()
+                single[0].record(stream)
+                f.run(0)
+                single[1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
     art.attn_sync_status()
-    p_tot = max(1e-9, max_over_ranks(sum(ev[s_][0].elapsed_time(ev[s_][1]) for s_ in range(args.steps)), world))
-    d_tot = [max(1e-9, max_over_ranks(sum(ev[s_][2 + 2 * n].elapsed_time(ev[s_][3 + 2 * n])
-                                          for s_ in range(args.steps)), world))
-             for n in range(len(decs))]
-    b_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 6].elapsed_time(ev[s_][nev - 5])
-                                         for s_ in range(args.steps)), world))
-    c_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 4].elapsed_time(ev[s_][nev - 3])
-                                         for s_ in range(args.steps)), world))
-    g_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 2].elapsed_time(ev[s_][nev - 1])
-                                         for s_ in range(args.steps)), world))
-    l_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 8].elapsed_time(ev[s_][nev - 7])
-                                         for s_ in range(args.steps)), world))
-    f_tot = max(1e-9, max_over_ranks(sum(ev[s_][nev - 10].elapsed_time(ev[s_][nev - 9])
-                                         for s_ in range(args.steps)), world))
     region_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
+    tot, tot_single = {}, {}
+    for f in fams:
+        tot[f.key] = max(1e-9, max_over_ranks(sum(ev[s_][f.key][0][0].elapsed_time(ev[s_][f.key][0][1])
+                                                  for s_ in range(args.steps)), world))
+        if f.reps > 1:
+            tot_single[f.key] = max(1e-9, max_over_ranks(
+                sum(ev[s_][f.key][1][0].elapsed_time(ev[s_][f.key][1][1]) for s_ in range(args.steps)), world))
 
-    # end to end through the public API: the step's inputs go host (pinned) -> device, the
-    # kernels run, the results come back device -> host; all inside the timed region
-    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    hdec = [(d["hq"].pin_memory(), torch.empty(d["hq"].shape, dtype=d["hq"].dtype).pin_memory())
-            for d in decs]
-    if blk is not None:
-        hbx = blk["hx"].pin_memory()
-        hbo = torch.empty(blk["hx"].shape, dtype=blk["hx"].dtype).pin_memory()
-        hfo = torch.empty(blk["hx"].shape, dtype=blk["hx"].dtype).pin_memory()
-    if paged is not None:
-        hpo = torch.empty(paged["out"].shape, dtype=paged["out"].dtype).pin_memory()
-    if lat is not None:
-        hlq = lat["hq"].pin_memory()
-        hlo = torch.empty(lat["hq"].shape, dtype=lat["hq"].dtype).pin_memory()
-    if chk is not None:
-        hcq_p = chk["hq"].pin_memory()
-        hco = torch.empty(chk["hq"].shape, dtype=chk["hq"].dtype).pin_memory()
-
-    def e2e_step():
-        if do_p:
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            prefill()
-            hout.copy_(dout, non_blocking=True)
-        for d, (hdq, hdo) in zip(decs, hdec):
-            d["q"].copy_(hdq, non_blocking=True)
-            decode(d)
-            hdo.copy_(d["out"], non_blocking=True)
-        if blk is not None:
-            blk["x"].copy_(hbx, non_blocking=True)
-            block()
-            hbo.copy_(blk["out"], non_blocking=True)
-            block_fused()
-            hfo.copy_(blk["fused"]["out"], non_blocking=True)
-        if chk is not None:
-            chk["q"].copy_(hcq_p, non_blocking=True)
-            chunk()
-            hco.copy_(chk["out"], non_blocking=True)
-        if paged is not None:
-            # its query tensor is the KV=8 decode's, already copied in above
-            decode_paged()
-            hpo.copy_(paged["out"], non_blocking=True)
-        if lat is not None:
-            lat["q"].copy_(hlq, non_blocking=True)
-            decode_latent()
-            hlo.copy_(lat["out"], non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    # end to end through the public API: each family's per-step inputs go host (pinned) ->
+    # device, the kernels run, the results come back device -> host; all inside the timed region
+    e2e_ms = {}
+    for f in fams:
+        if f.e2e is None:
+            continue
+        for _ in range(2):
+            f.e2e[2]()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = evpair()
+        e0.record(stream)
+        for _ in range(args.steps):
+            f.e2e[2]()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms[f.key] = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
 
     if rank != 0:
         return
     if args.only != "all":
-        print(json.dumps({"only": args.only, "prefill_ms": p_tot / args.steps,
-                          "decode_ms": [t / args.steps for t in d_tot],
-                          "block_ms": b_tot / args.steps, "chunk_ms": c_tot / args.steps}), flush=True)
+        print(json.dumps({"only": args.only, "ms": {f.key: tot[f.key] / (args.steps * f.reps) for f in fams}}),
+              flush=True)
         return
     pk = peaks()
-    flops_step = w.flops
-    per_launch_ms = p_tot / args.steps
-    achieved = flops_step / (per_launch_ms * 1e-3) / 1e12
     traffic = measured_traffic()
-    decode_out = {}
-    for n, d in enumerate(decs):
-        ms = d_tot[n] / args.steps
-        gbs = d["bytes"] / (ms * 1e-3) / 1e9
-        decode_out[d["w"].name] = {
-            "value": aggregate_rate(d["bytes"] * args.steps, world, d_tot[n]) / 1e9, "unit": "GB/s",
-            "ms": ms, "bytes": d["bytes"],
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "traffic": traffic.get(d["w"].name),
-                         "peak_source": f"{pk.get('source')} copy"}}
-    bw = blk["w"]
-    b_ms = b_tot / args.steps
-    b_tflops = bw.flops / (b_ms * 1e-3) / 1e12
-    # the block's attention has the prefill's shape and flags, so its time is the prefill's
-    proj_ms = max(1e-9, b_ms - per_launch_ms)
-    proj_tflops = bw.projection_flops / (proj_ms * 1e-3) / 1e12
-    block_out = {
-        "workload": bw.name, "value": aggregate_rate(bw.flops * args.steps, world, b_tot) / 1e12,
-        "unit": "TFLOP/s", "ms": b_ms, "flops": bw.flops, "projection_flops": bw.projection_flops,
-        "roofline": {"bound": "tensor", "achieved": b_tflops, "peak": pk["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": b_tflops / pk["bf16_tflops"], "traffic": None,
-                     "peak_source": f"{pk.get('source')} burst bf16 dense"},
-        "projections_derived": {"tflops": proj_tflops, "ms": proj_ms,
-                                "frac": proj_tflops / pk["bf16_tflops"],
-                                "how": "block time minus the prefill time of the same shape"}}
-    f_ms = f_tot / args.steps
-    f_tflops = bw.flops / (f_ms * 1e-3) / 1e12
-    block_out["fused"] = {
-        "what": "RMSNorm, one QKV GEMM (RoPE and cache write in its epilogue), attention, Wo GEMM + residual",
-        "value": aggregate_rate(bw.flops * args.steps, world, f_tot) / 1e12, "unit": "TFLOP/s", "ms": f_ms,
-        "roofline": {"bound": "tensor", "achieved": f_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": f_tflops / pk["bf16_tflops"], "traffic": None,
-                     "peak_source": f"{pk.get('source')} burst bf16 dense"}}
-    if paged is not None:
-        ms = g_tot / args.steps
-        gbs = paged["bytes"] / (ms * 1e-3) / 1e9
-        decode_out[paged["w"].name + f"_paged{PAGE_SIZE}"] = {
-            "value": aggregate_rate(paged["bytes"] * args.steps, world, g_tot) / 1e9, "unit": "GB/s",
-            "ms": ms, "bytes": paged["bytes"], "page_size": PAGE_SIZE, "pages": "shuffled",
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"],
-                         "traffic": traffic.get(paged["w"].name + f"_paged{PAGE_SIZE}"),
-                         "peak_source": f"{pk.get('source')} copy"}}
-    if lat is not None:
-        ms = l_tot / args.steps
-        gbs = lat["bytes"] / (ms * 1e-3) / 1e9
-        decode_out[lat["w"].name] = {
-            "value": aggregate_rate(lat["bytes"] * args.steps, world, l_tot) / 1e9, "unit": "GB/s",
-            "ms": ms, "bytes": lat["bytes"],
-            "note": "each latent tile is fetched twice (as keys and as values); bytes count it once",
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "traffic": traffic.get(lat["w"].name),
-                         "peak_source": f"{pk.get('source')} copy"}}
-    cw = chk["w"]
-    c_ms = c_tot / args.steps
-    c_tflops = cw.flops / (c_ms * 1e-3) / 1e12
-    chunk_out = {
-        "workload": cw.name, "value": aggregate_rate(cw.flops * args.steps, world, c_tot) / 1e12,
-        "unit": "TFLOP/s", "ms": c_ms, "flops": cw.flops,
-        "roofline": {"bound": "tensor", "achieved": c_tflops, "peak": pk["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": c_tflops / pk["bf16_tflops"], "traffic": None,
-                     "kernel": "prefill_tc_kernel<128, true>",
-                     "peak_source": f"{pk.get('source')} burst bf16 dense"}}
-    xb = blk["hx"].numel() * blk["hx"].element_size()
-    cb = chk["hq"].numel() * chk["hq"].element_size()
-    h2d = sum(t.numel() * t.element_size() for t in (q, k, v)) + sum(
-        d["hq"].numel() * d["hq"].element_size() for d in decs) + xb + cb
-    d2h = q.numel() * q.element_size() + sum(
-        d["hq"].numel() * d["hq"].element_size() for d in decs) + 2 * xb + cb
-    if paged is not None:
-        d2h += paged["out"].numel() * paged["out"].element_size()
-    if lat is not None:
-        h2d += lat["hq"].numel() * lat["hq"].element_size()
-        d2h += lat["hq"].numel() * lat["hq"].element_size()
+    fam_out, summary = {}, {}
+    for f in fams:
+        ms = tot[f.key] / (args.steps * f.reps)
+        scale = 1e12 if f.unit == "TFLOP/s" else 1e9
+        rate = f.work / (ms * 1e-3) / scale
+        peak = pk["bf16_tflops"] if f.bound == "tensor" else pk["hbm_gbs"]
+        psrc = f"{pk.get('source')} " + ("burst bf16 dense" if f.bound == "tensor" else "copy")
+        entry = {"workload": f.workload, "value": aggregate_rate(f.work * args.steps * f.reps, world, tot[f.key])
+                 / scale, "unit": f.unit, "ms": ms, "work": f.work,
+                 "launches": f.launches,
+                 "roofline": {"bound": f.bound, "achieved": rate, "peak": peak, "unit": f.unit,
+                              "frac": rate / peak, "traffic": traffic.get(f.key), "kernel": f.kernel,
+                              "peak_source": psrc}}
+        if f.reps > 1:
+            ms1 = tot_single[f.key] / args.steps
+            entry["timing"] = f"{f.reps} launches back to back over {f.reps} input copies per step"
+            entry["ms_single"] = ms1
+            entry["value_single"] = f.work / (ms1 * 1e-3) / scale
+        if f.note:
+            entry["note"] = f.note
+        if f.key in e2e_ms:
+            h2d, d2h, _ = f.e2e
+            entry["e2e"] = {"ms": e2e_ms[f.key], "h2d_bytes": h2d, "d2h_bytes": d2h,
+                            "value": f.work / (e2e_ms[f.key] * 1e-3) / scale}
+        fam_out[f.key] = entry
+        summary[f.key] = [round(entry["value"], 1), f.unit, round(rate / peak, 3)]
+    head = fam_out["gqa_prefill"]
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        val, dt, sample = oracle_sample_tflops()
-        cpu = {"value": val, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-               "sample": sample, "seconds": round(dt, 2)}
+        cpu = cpu_baseline()
+    launches = sum(f.launches * (f.reps + (1 if f.reps > 1 else 0)) for f in fams)
+    h2d, d2h, _ = next(f for f in fams if f.key == "gqa_prefill").e2e
     line = {
-        "metric": METRIC, "value": aggregate_rate(flops_step * args.steps, world, p_tot) / 1e12,
-        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": (p_tot + sum(d_tot) + b_tot + c_tot + g_tot + l_tot + f_tot) / args.steps,
-        "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "decode_workloads": [d["w"].name for d in decs],
-                   "block_workload": bw.name, "chunk_workload": cw.name,
-                   "parallelism": f"replicas{world}",
-                   "l2": "flushed: 256 MiB memset before every kernel family, outside the events",
-                   "timed_region_ms": region_ms},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
-                     "traffic": traffic.get(w.name), "kernel": "prefill_tc_kernel<128, false>",
-                     "peak_source": f"{pk.get('source')} burst bf16 dense"},
-        "decode": decode_out,
-        "block": block_out,
-        "chunk": chunk_out,
-        "e2e": {"value": aggregate_rate(flops_step * args.steps, world, e2e_ms) / 1e12,
-                "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "ms_per_step": e2e_ms / args.steps,
-                "note": "prefill FLOPs over the whole step incl. copies, both decodes, the block "
-                        "(block weights resident; x in, out back) and the chunk (cache resident; "
-                        "its queries in, out back)"},
-        "gpu_launches": args.steps * (PREFILL_LAUNCHES + DECODE_LAUNCHES * (len(decs) + 1) + BLOCK_LAUNCHES
-                                      + CHUNK_LAUNCHES + LATENT_LAUNCHES + FUSED_LAUNCHES),
+        "metric": METRIC, "value": head["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": sum(tot.values()) / args.steps + sum(tot_single.values()) / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": base_config(world),
+        "timed_region_ms": region_ms,
+        "families": fam_out,
         "clocks": clk,
         "cpu_baseline": cpu,
+        "gpu_launches": args.steps * launches,
+        "e2e": {"value": aggregate_rate(PREFILL.flops * args.steps, world, e2e_ms["gqa_prefill"] * args.steps)
+                / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": e2e_ms["gqa_prefill"],
+                "note": "the GQA prefill: q, k, v in from pinned host memory, the prefill, out back"},
+        "roofline": {**head["roofline"]},
+        "summary": summary,
     }
     print(json.dumps(line), flush=True)
 
@@ -627,12 +600,12 @@ def run_ours(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "block", "chunk"], default="all",
-                    help="run one kernel family only (for profiler captures; not a bench line)")
+    ap.add_argument("--only", default="all",
+                    help="comma-separated family keys to run (for profiler captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -319,11 +319,12 @@ def rmsnorm(x, gamma, eps: float = 1e-6) -> np.ndarray:
 
 
 def block_fused(x, gamma, Wqkv, Wo, *, H: int, KV: int, pos0: int = 0, rope_base: float = 0.0,
-                causal: bool = True, window: int = 0, slopes=None, eps: float = 1e-6):
+                causal: bool = True, window: int = 0, slopes=None, eps: float = 1e-6, rows=None):
     """The attention sub-layer of a pre-norm decoder block ([XF5] "RMSNorm and Pre-LN
     residuals": x + attn(norm(x))): RMSNorm, one projection x_n @ Wqkv whose columns are
     [q heads | k heads | v heads] (Wqkv [d, (H + 2 KV) hd]), attention, ctx @ Wo, plus x.
-    Returns out [B,T,d] and the rows a cache keeps: k turned at positions pos0.., v [B,T,KV,hd]."""
+    Returns out [B,T,d] and the rows a cache keeps: k turned at positions pos0.., v [B,T,KV,hd].
+    ``rows`` (query row indices) restricts out to those rows: out [B,len(rows),d]."""
     x = _f64(x)
     Wqkv, Wo = _f64(Wqkv), _f64(Wo)
     B, T, d = x.shape
@@ -333,8 +334,9 @@ def block_fused(x, gamma, Wqkv, Wo, *, H: int, KV: int, pos0: int = 0, rope_base
     k = qkv[..., H * hd:(H + KV) * hd].reshape(B, T, KV, hd)
     v = qkv[..., (H + KV) * hd:].reshape(B, T, KV, hd)
     ctx, _ = attention(q, k, v, pos0=pos0, rope_base=rope_base, causal=causal, window=window,
-                       slopes=slopes)
-    out = x + ctx.reshape(B, T, H * hd) @ Wo
+                       slopes=slopes, rows=rows)
+    R = T if rows is None else len(rows)
+    out = (x if rows is None else x[:, np.asarray(rows)]) + ctx.reshape(B, R, H * hd) @ Wo
     kc = k.transpose(0, 2, 1, 3)                                 # [B,KV,T,hd]
     if rope_base > 0:
         kc = rope(kc, pos0 + np.arange(T), rope_base)
@@ -342,11 +344,12 @@ def block_fused(x, gamma, Wqkv, Wo, *, H: int, KV: int, pos0: int = 0, rope_base
 
 
 def block(x, Wq, Wk, Wv, Wo, *, H: int, KV: int, pos0: int = 0, rope_base: float = 0.0,
-          causal: bool = True, window: int = 0, slopes=None):
+          causal: bool = True, window: int = 0, slopes=None, rows=None):
     """Projections, attention and output projection of [LAB] attention(): x [B,T,d] -> [B,T,d].
 
     Weights are [in, out] and applied as x @ W; head h is columns h*hd .. h*hd+hd-1 of
-    x @ Wq (the reshape to heads of [LAB]). No bias, residual or normalisation.
+    x @ Wq (the reshape to heads of [LAB]). No bias, residual or normalisation. ``rows``
+    (query row indices) restricts the result to those rows: [B,len(rows),d].
     """
     x = _f64(x)
     Wq, Wk, Wv, Wo = (_f64(w) for w in (Wq, Wk, Wv, Wo))
@@ -356,5 +359,5 @@ def block(x, Wq, Wk, Wv, Wo, *, H: int, KV: int, pos0: int = 0, rope_base: float
     k = (x @ Wk).reshape(B, T, KV, hd)
     v = (x @ Wv).reshape(B, T, KV, hd)
     ctx, _ = attention(q, k, v, pos0=pos0, rope_base=rope_base, causal=causal, window=window,
-                       slopes=slopes)
-    return ctx.reshape(B, T, H * hd) @ Wo
+                       slopes=slopes, rows=rows)
+    return ctx.reshape(B, T if rows is None else len(rows), H * hd) @ Wo

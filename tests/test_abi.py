@@ -205,3 +205,63 @@ def test_binding_requires_cuda_tensors(lib):
     q = torch.zeros(1, 4, 2, 8, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         art.attn_prefill(q, q, q, out=q)
+
+
+def test_binding_rejects_mismatched_shapes(lib):
+    """The binding checks every tensor's shape against the sizes it passes to the library
+    before any call: the kernels index by those sizes, so a tensor of another shape would be
+    read or written out of bounds. (CPU tensors: the shape check fires before the device check.)"""
+    import torch
+
+    import alibi_rope_tile_b200 as art
+    bf = torch.bfloat16
+    B, T, d, H, KV, hd = 2, 16, 64, 4, 2, 16
+    x = torch.zeros(B, T, d, dtype=bf)
+    gamma = torch.ones(d, dtype=bf)
+    Wqkv = torch.zeros(d, (H + 2 * KV) * hd, dtype=bf)
+    Wo = torch.zeros(H * hd, d, dtype=bf)
+    kc = torch.zeros(B, 32, KV, hd, dtype=bf)
+    cases = [
+        (dict(Wqkv=torch.zeros(d, (H + 2 * KV) * hd + 1, dtype=bf)), "Wqkv"),
+        (dict(Wqkv=torch.zeros(d + 8, (H + 2 * KV) * hd, dtype=bf)), "Wqkv"),
+        (dict(Wo=torch.zeros(H * hd, d + 8, dtype=bf)), "Wo"),
+        (dict(gamma=torch.ones(d - 8, dtype=bf)), "gamma"),
+        (dict(kcache=torch.zeros(B, 32, KV + 1, hd, dtype=bf), vcache=kc), "kcache"),
+        (dict(kcache=kc, vcache=torch.zeros(B, 31, KV, hd, dtype=bf)), "vcache"),
+        (dict(kcache=kc, vcache=None), "both"),
+    ]
+    for change, what in cases:
+        kw = dict(x=x, gamma=gamma, Wqkv=Wqkv, Wo=Wo, kcache=None, vcache=None)
+        kw.update(change)
+        with pytest.raises(ValueError, match=what):
+            art.attn_block_fused(kw.pop("x"), kw.pop("gamma"), kw.pop("Wqkv"), kw.pop("Wo"), H=H, KV=KV, **kw)
+    Wq, Wk = torch.zeros(d, H * hd, dtype=bf), torch.zeros(d, KV * hd, dtype=bf)
+    with pytest.raises(ValueError, match="Wv"):
+        art.attn_block(x, Wq, Wk, torch.zeros(d, KV * hd + 8, dtype=bf), Wo, H=H, KV=KV)
+    with pytest.raises(ValueError, match="Wo"):
+        art.attn_block(x, Wq, Wk, Wk, torch.zeros(H * hd + 8, d, dtype=bf), H=H, KV=KV)
+    q = torch.zeros(B, T, H, hd, dtype=bf)
+    k = torch.zeros(B, T, KV, hd, dtype=bf)
+    with pytest.raises(ValueError, match="out"):
+        art.attn_prefill(q, k, k, out=torch.zeros(B, T, H, hd + 8, dtype=bf))
+    with pytest.raises(ValueError, match="lse"):
+        art.attn_prefill(q, k, k, lse=torch.zeros(B, T, H, dtype=torch.float32))
+    dq = torch.zeros(B, H, hd, dtype=bf)
+    sl = torch.zeros(B, dtype=torch.int32)
+    with pytest.raises(ValueError, match="vcache"):
+        art.attn_decode(dq, kc, torch.zeros(B, 16, KV, hd, dtype=bf), sl, sl)
+    with pytest.raises(ValueError, match="seqlens"):
+        art.attn_decode(dq, kc, kc, torch.zeros(B + 1, dtype=torch.int32), sl)
+    with pytest.raises(ValueError, match="out"):
+        art.attn_decode_noalloc(dq, kc, kc, sl, sl, None)
+    with pytest.raises(ValueError, match="qpos0"):
+        art.attn_prefill_chunk(q, kc, kc, sl, torch.zeros(1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="kcache"):
+        art.attn_kv_write(k, k, torch.zeros(B, 32, KV, hd + 2, dtype=bf), kc, sl)
+    with pytest.raises(ValueError, match="block_table"):
+        art.attn_decode_paged(dq, kc, kc, torch.zeros(B + 1, 4, dtype=torch.int32), sl, sl)
+    with pytest.raises(ValueError, match="W_uv"):
+        art.attn_decode_latent(dq, torch.zeros(B, 32, 64, dtype=bf), torch.zeros(H, 64, hd, dtype=bf),
+                               torch.zeros(H, 64, hd + 2, dtype=bf), sl, sl)
+    with pytest.raises(ValueError, match="pos"):
+        art.attn_kv_append(dq[:, :KV], dq[:, :KV], kc, kc, torch.zeros(B + 1, dtype=torch.int32))

@@ -61,3 +61,43 @@ def test_fused_block_matches_oracle(art, case):
         assert_close(kc[:, pos0:pos0 + T], rk, BF, "cache keys")
         assert_close(vc[:, pos0:pos0 + T], rv, BF, "cache values")
         assert torch.count_nonzero(kc[:, :pos0]) == 0 and torch.count_nonzero(kc[:, pos0 + T:]) == 0
+
+
+def test_fused_block_at_bench_size(art):
+    """The bench's fused sub-layer (x [2,4096,4096], gamma = 1, Wqkv = [Wq|Wk|Wv], caches
+    [2,4096,8,128]) against the oracle on 1,024 sampled rows per sequence, and its cache rows."""
+    from tests.test_block_gpu import sampled_rows
+    bw = workloads.GQA_BLOCK
+    x, W = workloads.block_inputs(bw)
+    Wqkv = torch.cat([W["Wq"], W["Wk"], W["Wv"]], dim=1).contiguous()
+    gamma = torch.ones(bw.d, dtype=BF)
+    kc = torch.zeros(bw.B, bw.T, bw.KV, bw.hd, dtype=BF, device="cuda")
+    vc = torch.zeros_like(kc)
+    out = art.attn_block_fused(x.cuda(), gamma.cuda(), Wqkv.cuda(), W["Wo"].cuda(), kcache=kc, vcache=vc,
+                               H=bw.H, KV=bw.KV, rope_base=bw.rope_base, causal=bw.causal, window=bw.window)
+    torch.cuda.synchronize()
+    assert art.attn_sync_status() == 0
+    rows = sampled_rows(bw.T, 62)
+    ref, rk, rv = A.block_fused(x, gamma, Wqkv, W["Wo"], H=bw.H, KV=bw.KV, rope_base=bw.rope_base,
+                                causal=bw.causal, window=bw.window, rows=rows)
+    assert_close(out[:, torch.from_numpy(rows).cuda()], ref, BF, "bench-size fused block")
+    assert_close(kc, rk, BF, "bench-size cache keys")
+    assert_close(vc, rv, BF, "bench-size cache values")
+
+
+def test_fused_block_rows_near_eps(art):
+    """Rows whose mean square is about eps (x ~ 1e-3 N(0,1), eps = 1e-6): where eps enters
+    RMSNorm shows in the output (under the root it damps these rows by about 1/sqrt(2))."""
+    B, T, d, H, KV = 1, 256, 512, 8, 2
+    hd = d // H
+    g = torch.Generator().manual_seed(77)
+    x = (1e-3 * torch.randn(B, T, d, generator=g)).to(BF)
+    gamma = (1.0 + 0.1 * torch.randn(d, generator=g)).to(BF)
+    Wqkv = (torch.randn(d, (H + 2 * KV) * hd, generator=g) / np.sqrt(d)).to(BF)
+    Wo = (torch.randn(H * hd, d, generator=g) / (2 * np.sqrt(H * hd))).to(BF)
+    out = art.attn_block_fused(x.cuda(), gamma.cuda(), Wqkv.cuda(), Wo.cuda(), H=H, KV=KV, rope_base=1e4)
+    torch.cuda.synchronize()
+    ref, _, _ = A.block_fused(x, gamma, Wqkv, Wo, H=H, KV=KV, rope_base=1e4)
+    assert_close(out, ref, BF, "fused block, rows near eps")
+    wrong, _, _ = A.block_fused(x, gamma, Wqkv, Wo, H=H, KV=KV, rope_base=1e4, eps=0.0)
+    assert np.abs(wrong - ref).max() > 0.05   # the case does tell the readings apart

@@ -62,3 +62,25 @@ def test_bf16_block(art, shape):
     out = run_block(art, W, x, 0, H=H, KV=KV, rope_base=10000.0)
     ref = A.block(x, W["Wq"], W["Wk"], W["Wv"], W["Wo"], H=H, KV=KV, rope_base=10000.0)
     assert_close(out, ref, torch.bfloat16, f"bf16 block {shape}")
+
+
+def sampled_rows(T: int, seed: int) -> np.ndarray:
+    """The first and last 256 query rows and 512 others drawn at random (seeded)."""
+    rng = np.random.default_rng(seed)
+    middle = rng.choice(np.arange(256, T - 256), size=512, replace=False)
+    return np.unique(np.concatenate([np.arange(256), middle, np.arange(T - 256, T)]))
+
+
+def test_bf16_block_at_bench_size(art):
+    """The bench's block (x [2,4096,4096], d 4096, H 32, KV 8, hd 128, RoPE 5e5, causal) in the
+    launch configuration the bench times, against the oracle on 1,024 sampled rows per sequence."""
+    bw = workloads.GQA_BLOCK
+    x, W = workloads.block_inputs(bw)
+    out = art.attn_block(x.cuda(), W["Wq"].cuda(), W["Wk"].cuda(), W["Wv"].cuda(), W["Wo"].cuda(),
+                         H=bw.H, KV=bw.KV, rope_base=bw.rope_base, causal=bw.causal, window=bw.window)
+    torch.cuda.synchronize()
+    assert art.attn_sync_status() == 0
+    rows = sampled_rows(bw.T, 61)
+    ref = A.block(x, W["Wq"], W["Wk"], W["Wv"], W["Wo"], H=bw.H, KV=bw.KV, rope_base=bw.rope_base,
+                  causal=bw.causal, window=bw.window, rows=rows)
+    assert_close(out[:, torch.from_numpy(rows).cuda()], ref, torch.bfloat16, "bench-size block")

@@ -52,7 +52,12 @@ MUTANTS = {
     "latent_value_projection": ("v = c[b, :L] @ W_uv[h]", "v = c[b, :L] @ W_uk[h]"),
     "rmsnorm_mean_not_rms": ("rms = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)",
                              "rms = np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)"),
-    "fused_no_residual": ("out = x + ctx.reshape(B, T, H * hd) @ Wo", "out = ctx.reshape(B, T, H * hd) @ Wo"),
+    "rmsnorm_eps_outside_root": ("rms = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)",
+                                 "rms = np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) + eps"),
+    "rmsnorm_default_eps": ("def rmsnorm(x, gamma, eps: float = 1e-6)", "def rmsnorm(x, gamma, eps: float = 1e-5)"),
+    "fused_default_eps": ("window: int = 0, slopes=None, eps: float = 1e-6):",
+                          "window: int = 0, slopes=None, eps: float = 1e-8):"),
+    "fused_no_residual":("out = x + ctx.reshape(B, T, H * hd) @ Wo", "out = ctx.reshape(B, T, H * hd) @ Wo"),
     "fused_qkv_split": ("k = qkv[..., H * hd:(H + KV) * hd].reshape(B, T, KV, hd)",
                         "k = qkv[..., (H + KV) * hd:].reshape(B, T, KV, hd)"),
     "block_wq_transposed": ("q = (x @ Wq).reshape(B, T, H, hd)", "q = (x @ Wq.T).reshape(B, T, H, hd)"),

@@ -387,6 +387,15 @@ def test_rmsnorm_closed_forms():
     np.testing.assert_allclose(np.sqrt(np.mean(y * y, axis=-1)), 2.5, rtol=0, atol=1e-14)
     # eps enters under the root: x = 0 rows stay 0, tiny rows are damped
     assert np.all(A.rmsnorm(np.zeros((1, 6)), g) == 0.0)
+    # where eps sits: a constant row c with eps = 3 c^2 gives c / sqrt(c^2 + 3 c^2) = sign(c) / 2
+    # (eps added outside the root would give c / (|c| + 3 c^2) instead: -0.1 gamma for c = -3)
+    for c in (-3.0, 0.5, 2.0):
+        np.testing.assert_allclose(A.rmsnorm(np.full((2, 6), c), g, eps=3.0 * c * c),
+                                   np.full((2, 6), np.sign(c) * 1.25), rtol=0, atol=1e-15)
+    # the default eps is 1e-6 (the listing of "RMSNorm and Pre-LN residuals"): a constant row of
+    # 1e-3 has mean square 1e-6, so it maps to gamma / sqrt(2); 1e-5 or 1e-8 would give 0.30 or 0.995
+    np.testing.assert_allclose(A.rmsnorm(np.full((1, 6), 1e-3), g), np.full((1, 6), 2.5 / np.sqrt(2.0)),
+                               rtol=1e-12, atol=0)
 
 
 def test_fused_block_is_residual_plus_the_plain_block_on_normalised_input():
@@ -425,3 +434,26 @@ def test_workload_pair_counts():
     # the chunk's rows are the second half of the GQA prefill's rows: its pairs plus the first
     # half's make up the whole causal triangle
     assert c.allowed_pairs + 2048 * 2049 // 2 == workloads.GQA.allowed_pairs
+
+
+def test_block_row_selection_equals_full_rows():
+    """block(rows=R) and block_fused(rows=R) are rows R of the full results (each query row's
+    output depends on the keys only through the full k, v, which are always computed)."""
+    B, T, d, H, KV, base = 2, 11, 16, 4, 2, 10000.0
+    hd = d // H
+    x = _rand((B, T, d), 130)
+    Wq, Wk, Wv, Wo = (_rand(s, 131 + n) / 4 for n, s in
+                      enumerate([(d, H * hd), (d, KV * hd), (d, KV * hd), (H * hd, d)]))
+    rows = [0, 3, 10, 7]
+    for window, slopes in [(0, None), (4, A.alibi_slopes(H))]:
+        full = A.block(x, Wq, Wk, Wv, Wo, H=H, KV=KV, pos0=3, rope_base=base, window=window, slopes=slopes)
+        part = A.block(x, Wq, Wk, Wv, Wo, H=H, KV=KV, pos0=3, rope_base=base, window=window, slopes=slopes,
+                       rows=rows)
+        np.testing.assert_array_equal(part, full[:, rows])
+        Wqkv = np.concatenate([Wq, Wk, Wv], axis=1)
+        gamma = 1.0 + 0.1 * _rand((d,), 140)
+        ffull, _, _ = A.block_fused(x, gamma, Wqkv, Wo, H=H, KV=KV, pos0=3, rope_base=base, window=window,
+                                    slopes=slopes)
+        fpart, _, _ = A.block_fused(x, gamma, Wqkv, Wo, H=H, KV=KV, pos0=3, rope_base=base, window=window,
+                                    slopes=slopes, rows=rows)
+        np.testing.assert_allclose(fpart, ffull[:, rows], rtol=0, atol=1e-13)
