@@ -55,8 +55,8 @@ MUTANTS = {
     "rmsnorm_eps_outside_root": ("rms = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)",
                                  "rms = np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) + eps"),
     "rmsnorm_default_eps": ("def rmsnorm(x, gamma, eps: float = 1e-6)", "def rmsnorm(x, gamma, eps: float = 1e-5)"),
-    "fused_default_eps": ("window: int = 0, slopes=None, eps: float = 1e-6):",
-                          "window: int = 0, slopes=None, eps: float = 1e-8):"),
+    "fused_default_eps": ("window: int = 0, slopes=None, eps: float = 1e-6, rows=None):",
+                          "window: int = 0, slopes=None, eps: float = 1e-8, rows=None):"),
     "fused_no_residual":("out = x + ctx.reshape(B, T, H * hd) @ Wo", "out = ctx.reshape(B, T, H * hd) @ Wo"),
     "fused_qkv_split": ("k = qkv[..., H * hd:(H + KV) * hd].reshape(B, T, KV, hd)",
                         "k = qkv[..., (H + KV) * hd:].reshape(B, T, KV, hd)"),
