@@ -57,7 +57,8 @@ MUTANTS = {
     "rmsnorm_default_eps": ("def rmsnorm(x, gamma, eps: float = 1e-6)", "def rmsnorm(x, gamma, eps: float = 1e-5)"),
     "fused_default_eps": ("window: int = 0, slopes=None, eps: float = 1e-6, rows=None):",
                           "window: int = 0, slopes=None, eps: float = 1e-8, rows=None):"),
-    "fused_no_residual":("out = x + ctx.reshape(B, T, H * hd) @ Wo", "out = ctx.reshape(B, T, H * hd) @ Wo"),
+    "fused_no_residual": ("out = (x if rows is None else x[:, np.asarray(rows)]) + ctx.reshape(B, R, H * hd) @ Wo",
+                          "out = ctx.reshape(B, R, H * hd) @ Wo"),
     "fused_qkv_split": ("k = qkv[..., H * hd:(H + KV) * hd].reshape(B, T, KV, hd)",
                         "k = qkv[..., (H + KV) * hd:].reshape(B, T, KV, hd)"),
     "block_wq_transposed": ("q = (x @ Wq).reshape(B, T, H, hd)", "q = (x @ Wq.T).reshape(B, T, H, hd)"),
