@@ -359,101 +359,113 @@ def build_families(art, only):
         fams.append(decode_family("decode_kv8_paged16", workloads.DECODE_GQA, True))
 
     if want("latent_decode"):
-        lw = workloads.LATENT_DECODE
-        lq, lc, luk, luv, lsl = workloads.latent_inputs(lw)
-        L = dict(q=lq.to(dev), c=lc.to(dev), uk=luk.to(dev), uv=luv.to(dev), sl=lsl.to(dev),
-                 out=torch.empty(lq.shape, dtype=lq.dtype, device=dev),
-                 ws=torch.empty(int(art.lib().attn_decode_latent_workspace_size(lw.B, lw.H, lw.hd, lw.dc,
-                                                                                lw.Lmax)),
-                                dtype=torch.uint8, device=dev))
-        del lc
-
-        def run_lat(i=0):
-            art.attn_decode_latent(L["q"], L["c"], L["uk"], L["uv"], L["sl"], L["sl"], L["out"],
-                                   workspace=L["ws"])
-        hlq = lq.pin_memory()
-        hlo = torch.empty(lq.shape, dtype=lq.dtype).pin_memory()
-
-        def e2e_lat():
-            L["q"].copy_(hlq, non_blocking=True)
-            run_lat(0)
-            hlo.copy_(L["out"], non_blocking=True)
-        # algorithmic bytes: each latent row read once, q and out, both weights
-        lbytes = int(lsl.sum()) * lw.dc * 2 + 2 * lw.B * lw.H * lw.hd * 2 + 2 * lw.H * lw.dc * lw.hd * 2
-        fams.append(Family("latent_decode", lw.name, "GB/s", "hbm", lbytes, LATENT_LAUNCHES,
-                           "decode_tc_kernel<128>", run_lat, e2e=(tnb(lq), tnb(lq), e2e_lat)))
-
+        fams.append(latent_family(art))
     if want("chunk"):
-        cw = workloads.GQA_CHUNK
-        hcq, hck, hcv = workloads.chunk_inputs(cw)
-        ckc = torch.zeros(cw.B, cw.Lmax, cw.KV, cw.hd, dtype=torch.bfloat16, device=dev)
-        cvc = torch.zeros_like(ckc)
-        art.attn_kv_write(hck.to(dev), hcv.to(dev), ckc, cvc,
-                          torch.zeros(cw.B, dtype=torch.int32, device=dev), rope_base=cw.rope_base)
-        C = dict(q=hcq.to(dev), kc=ckc, vc=cvc,
-                 sl=torch.full((cw.B,), cw.qpos0 + cw.Tq, dtype=torch.int32, device=dev),
-                 qp=torch.full((cw.B,), cw.qpos0, dtype=torch.int32, device=dev),
-                 out=torch.empty(hcq.shape, dtype=hcq.dtype, device=dev))
-
-        def run_chunk(i=0):
-            art.attn_prefill_chunk(C["q"], C["kc"], C["vc"], C["sl"], C["qp"], C["out"], rope_base=cw.rope_base)
-        hq = hcq.pin_memory()
-        ho = torch.empty(hcq.shape, dtype=hcq.dtype).pin_memory()
-
-        def e2e_chunk():
-            C["q"].copy_(hq, non_blocking=True)
-            run_chunk(0)
-            ho.copy_(C["out"], non_blocking=True)
-        fams.append(Family("chunk", cw.name, "TFLOP/s", "tensor", cw.flops, 1, "prefill_tc_kernel<128, true>",
-                           run_chunk, e2e=(tnb(hcq), tnb(hcq), e2e_chunk)))
-
+        fams.append(chunk_family(art))
     if want("block") or want("block_fused"):
-        bw = workloads.GQA_BLOCK
-        hx, hW = workloads.block_inputs(bw)
-        X = dict(x=hx.to(dev), W={n: t.to(dev) for n, t in hW.items()},
-                 out=torch.empty(hx.shape, dtype=hx.dtype, device=dev))
-        hxp = hx.pin_memory()
+        fams.extend(block_families(art, want))
+    return fams
+
+
+def latent_family(art):
+    dev = "cuda"
+    lw = workloads.LATENT_DECODE
+    lq, lc, luk, luv, lsl = workloads.latent_inputs(lw)
+    L = dict(q=lq.to(dev), c=lc.to(dev), uk=luk.to(dev), uv=luv.to(dev), sl=lsl.to(dev),
+             out=torch.empty(lq.shape, dtype=lq.dtype, device=dev),
+             ws=torch.empty(int(art.lib().attn_decode_latent_workspace_size(lw.B, lw.H, lw.hd, lw.dc, lw.Lmax)),
+                            dtype=torch.uint8, device=dev))
+    del lc
+
+    def run(i=0):
+        art.attn_decode_latent(L["q"], L["c"], L["uk"], L["uv"], L["sl"], L["sl"], L["out"], workspace=L["ws"])
+    hq = lq.pin_memory()
+    ho = torch.empty(lq.shape, dtype=lq.dtype).pin_memory()
+
+    def e2e_step():
+        L["q"].copy_(hq, non_blocking=True)
+        run(0)
+        ho.copy_(L["out"], non_blocking=True)
+    # algorithmic bytes: each latent row read once, q and out, both weights
+    nbytes = int(lsl.sum()) * lw.dc * 2 + 2 * lw.B * lw.H * lw.hd * 2 + 2 * lw.H * lw.dc * lw.hd * 2
+    return Family("latent_decode", lw.name, "GB/s", "hbm", nbytes, LATENT_LAUNCHES, "decode_tc_kernel<128>",
+                  run, e2e=(tnb(lq), tnb(lq), e2e_step))
+
+
+def chunk_family(art):
+    dev = "cuda"
+    cw = workloads.GQA_CHUNK
+    hcq, hck, hcv = workloads.chunk_inputs(cw)
+    kc = torch.zeros(cw.B, cw.Lmax, cw.KV, cw.hd, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    art.attn_kv_write(hck.to(dev), hcv.to(dev), kc, vc, torch.zeros(cw.B, dtype=torch.int32, device=dev),
+                      rope_base=cw.rope_base)
+    C = dict(q=hcq.to(dev), kc=kc, vc=vc,
+             sl=torch.full((cw.B,), cw.qpos0 + cw.Tq, dtype=torch.int32, device=dev),
+             qp=torch.full((cw.B,), cw.qpos0, dtype=torch.int32, device=dev),
+             out=torch.empty(hcq.shape, dtype=hcq.dtype, device=dev))
+
+    def run(i=0):
+        art.attn_prefill_chunk(C["q"], C["kc"], C["vc"], C["sl"], C["qp"], C["out"], rope_base=cw.rope_base)
+    hq = hcq.pin_memory()
+    ho = torch.empty(hcq.shape, dtype=hcq.dtype).pin_memory()
+
+    def e2e_step():
+        C["q"].copy_(hq, non_blocking=True)
+        run(0)
+        ho.copy_(C["out"], non_blocking=True)
+    return Family("chunk", cw.name, "TFLOP/s", "tensor", cw.flops, 1, "prefill_tc_kernel<128, true>", run,
+                  e2e=(tnb(hcq), tnb(hcq), e2e_step))
+
+
+def block_families(art, want):
+    dev = "cuda"
+    fams = []
+    bw = workloads.GQA_BLOCK
+    hx, hW = workloads.block_inputs(bw)
+    X = dict(x=hx.to(dev), W={n: t.to(dev) for n, t in hW.items()})
+    hxp = hx.pin_memory()
+    if want("block"):
+        out = torch.empty(hx.shape, dtype=hx.dtype, device=dev)
+        ws = torch.empty(art.attn_block_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV, bw.hd, torch.bfloat16),
+                         dtype=torch.uint8, device=dev)
         ho = torch.empty(hx.shape, dtype=hx.dtype).pin_memory()
-        if want("block"):
-            X["ws"] = torch.empty(art.attn_block_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV, bw.hd,
-                                                                torch.bfloat16), dtype=torch.uint8, device=dev)
 
-            def run_block(i=0):
-                W = X["W"]
-                art.attn_block(X["x"], W["Wq"], W["Wk"], W["Wv"], W["Wo"], X["out"], workspace=X["ws"],
-                               H=bw.H, KV=bw.KV, rope_base=bw.rope_base, causal=bw.causal, window=bw.window)
+        def run_block(i=0):
+            W = X["W"]
+            art.attn_block(X["x"], W["Wq"], W["Wk"], W["Wv"], W["Wo"], out, workspace=ws, H=bw.H, KV=bw.KV,
+                           rope_base=bw.rope_base, causal=bw.causal, window=bw.window)
 
-            def e2e_block():
-                X["x"].copy_(hxp, non_blocking=True)
-                run_block(0)
-                ho.copy_(X["out"], non_blocking=True)
-            fams.append(Family("block", bw.name, "TFLOP/s", "tensor", bw.flops, BLOCK_LAUNCHES,
-                               "gemm_tc_kernel", run_block, e2e=(tnb(hx), tnb(hx), e2e_block),
-                               note="projection FLOPs 2*M*N*K plus the attention's; weights resident"))
-        if want("block_fused"):
-            # the same block as a fused pre-norm sub-layer: RMSNorm, one Wqkv, cache write, residual
-            F = dict(gamma=torch.ones(bw.d, dtype=torch.bfloat16, device=dev),
-                     Wqkv=torch.cat([X["W"]["Wq"], X["W"]["Wk"], X["W"]["Wv"]], dim=1).contiguous(),
-                     kc=torch.zeros(bw.B, bw.T, bw.KV, bw.hd, dtype=torch.bfloat16, device=dev),
-                     out=torch.empty(hx.shape, dtype=hx.dtype, device=dev),
-                     ws=torch.empty(int(art.lib().attn_block_fused_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV,
-                                                                                  bw.hd)),
-                                    dtype=torch.uint8, device=dev))
-            F["vc"] = torch.zeros_like(F["kc"])
+        def e2e_block():
+            X["x"].copy_(hxp, non_blocking=True)
+            run_block(0)
+            ho.copy_(out, non_blocking=True)
+        fams.append(Family("block", bw.name, "TFLOP/s", "tensor", bw.flops, BLOCK_LAUNCHES, "gemm_tc_kernel",
+                           run_block, e2e=(tnb(hx), tnb(hx), e2e_block),
+                           note="projection FLOPs 2*M*N*K plus the attention's; weights resident"))
+    if want("block_fused"):
+        # the same block as a fused pre-norm sub-layer: RMSNorm, one Wqkv, cache write, residual
+        F = dict(gamma=torch.ones(bw.d, dtype=torch.bfloat16, device=dev),
+                 Wqkv=torch.cat([X["W"]["Wq"], X["W"]["Wk"], X["W"]["Wv"]], dim=1).contiguous(),
+                 kc=torch.zeros(bw.B, bw.T, bw.KV, bw.hd, dtype=torch.bfloat16, device=dev),
+                 out=torch.empty(hx.shape, dtype=hx.dtype, device=dev),
+                 ws=torch.empty(int(art.lib().attn_block_fused_workspace_size(bw.B, bw.T, bw.d, bw.H, bw.KV, bw.hd)),
+                                dtype=torch.uint8, device=dev))
+        F["vc"] = torch.zeros_like(F["kc"])
+        fo = torch.empty(hx.shape, dtype=hx.dtype).pin_memory()
 
-            def run_fused(i=0):
-                art.attn_block_fused(X["x"], F["gamma"], F["Wqkv"], X["W"]["Wo"], F["out"], F["kc"], F["vc"],
-                                     F["ws"], H=bw.H, KV=bw.KV, rope_base=bw.rope_base, causal=bw.causal,
-                                     window=bw.window)
+        def run_fused(i=0):
+            art.attn_block_fused(X["x"], F["gamma"], F["Wqkv"], X["W"]["Wo"], F["out"], F["kc"], F["vc"], F["ws"],
+                                 H=bw.H, KV=bw.KV, rope_base=bw.rope_base, causal=bw.causal, window=bw.window)
 
-            def e2e_fused():
-                X["x"].copy_(hxp, non_blocking=True)
-                run_fused(0)
-                ho.copy_(F["out"], non_blocking=True)
-            fams.append(Family("block_fused", bw.name + "_prenorm", "TFLOP/s", "tensor", bw.flops,
-                               FUSED_LAUNCHES, "gemm_tc_kernel", run_fused, e2e=(tnb(hx), tnb(hx), e2e_fused),
-                               note="RMSNorm, one QKV GEMM (RoPE and cache write in its epilogue), "
-                                    "attention, Wo GEMM + residual"))
+        def e2e_fused():
+            X["x"].copy_(hxp, non_blocking=True)
+            run_fused(0)
+            fo.copy_(F["out"], non_blocking=True)
+        fams.append(Family("block_fused", bw.name + "_prenorm", "TFLOP/s", "tensor", bw.flops, FUSED_LAUNCHES,
+                           "gemm_tc_kernel", run_fused, e2e=(tnb(hx), tnb(hx), e2e_fused),
+                           note="RMSNorm, one QKV GEMM (RoPE and cache write in its epilogue), attention, "
+                                "Wo GEMM + residual"))
     return fams
 
 
