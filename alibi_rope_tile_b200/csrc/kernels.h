@@ -34,9 +34,11 @@ struct PrefillParams {
 // CUDA-core flash prefill: fp32 or bf16 elements, any even hd <= 256.
 cudaError_t launch_prefill_simt(const PrefillParams& p, int dtype, cudaStream_t s);
 
-// Tensor-core (tcgen05 + TMEM + TMA) prefill: bf16, hd in {64, 128}.
+// Tensor-core (tcgen05 + TMEM + TMA) prefill: bf16, hd in {64, 128}. launch_prefill_tc picks
+// the kernel; launch_prefill_pair is the two-slot form it uses for hd = 128 with rotation.
 bool prefill_tc_supported(const PrefillParams& p, int dtype);
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t s);
+cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t s);
 
 struct DecodeParams {
   const void* q;        // [B,H,hd]

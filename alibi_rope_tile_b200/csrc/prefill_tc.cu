@@ -8,49 +8,41 @@
 // grouped-query attention with RoPE and Flash Attention from scratch" (Step 3): a running
 // maximum, a running denominator and a rescaled output accumulator.
 //
-// Work unit (one CTA): two "slots" of 128 query rows that read the same key/value head:
-//   * H/KV even: two query heads of one group at the same rows (GQA sharing);
-//   * H/KV odd (MHA included): one head, two consecutive 128-row tiles.
-// Both slots consume every key/value tile the CTA loads, so each tile is fetched and
-// rotated once per 256 query rows. CTAs are numbered longest-first (causal rows near the
-// end see the most keys) so the block scheduler packs them like an LPT schedule.
+// Work unit (one CTA): 128 query rows of one head. CTAs are numbered longest-first (causal
+// rows near the end see the most keys) so the block scheduler packs them like an LPT
+// schedule, and the heads of one key/value group are adjacent, so the four reads of each
+// K/V tile of a GQA group meet in L2.
+//
+// Operands. The query tile is turned once and moved into tensor memory, so S = Q K^T is a
+// TS-form MMA whose only shared-memory operand is the key tile; O += P V is a TS-form MMA
+// that reads P (bf16) from tensor memory. Both run at N = 128 over whole 128-key tiles,
+// which K/V tiles reach through a TMA ring of NS stages (keys turned in place as they
+// land). S is double-buffered in tensor memory: the tensor core computes the scores of key
+// tile j+1 while the softmax works on tile j. Tensor memory (512 columns): O (hd) | Q
+// (hd/2: bf16 pairs) | ... | S0 (128) | S1 (128) from column 256.
+// Issue order: QK(0); then per tile j: QK(j+1), PV(j). QK(j+1) overwrites the S/P buffer of
+// tile j-1 only after PV(j-1) (the tensor core executes one CTA's MMAs in issue order).
 //
 // Warp roles (22 warps):
-//   warps 0-15  softmax, one slot at a time (slot 0, then slot 1, for every key tile):
-//               warp w owns 32 query rows (TMEM lanes 32*(w%4)..) and 32 keys of the tile
-//               (keys 32*(w/4)..)
-//   warps 16-19 rotary embedding: turns the two Q tiles once, then every K tile in place
-//               in its 128-byte-swizzled shared-memory layout (RoPE on load)
-//   warp 20     TMA producer (Q tiles, then K/V tiles through a ring of NS stages)
+//   warps 0-15  softmax: warp w owns TMEM lanes 32*(w%4).. (32 query rows) and keys
+//               32*(w/4) .. +31 of every tile
+//   warps 16-19 rotary embedding: turns the Q tile in place and moves it into tensor memory,
+//               then turns every K tile in place in its 128-byte-swizzled layout
+//   warp 20     TMA producer (the Q tile, then K/V tiles through the ring)
 //   warp 21     TMEM allocation and UMMA issue
-// Tensor memory (512 columns): S0 | S1 (128 fp32 columns each) | O0 | O1 (hd each).
-// P (bf16, two per 32-bit column) goes over the first 64 columns of the slot's S region
-// once every softmax warp has read its S columns (keys 2c, 2c+1 -> column c), and PV takes
-// P straight from tensor memory (the A operand of the TS-form MMA): P never touches shared
-// memory, which the SS-form QK MMAs, the TMA writes and the in-place key rotation already
-// share (an M=128, N=128 SS MMA reads 8 KB of operands from shared memory). The next
-// QK of a slot overwrites that slot's S/P columns; it is issued after the slot's PV, and
-// the tensor core executes one CTA's MMAs in issue order, so P is read before it is
-// overwritten. Issue order per key tile j: PV0(j), QK0(j+1), PV1(j), QK1(j+1): the tensor
-// core works on one slot while the softmax warps work on the other.
 //
 // Masking: a pair outside the causal/window/length limits gets -inf before the row max,
 // so its weight is exactly 0, and the sums' order depends only on the tile structure;
-// a row's output never depends on the keys it may not see. Tiles outside a slot's key
-// range are skipped entirely.
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
-#include "kernels.h"
-#include "tc_common.cuh"
+// a row's output never depends on the keys it may not see. Tiles outside the key range
+// are skipped entirely.
+#include "prefill_common.cuh"
 
 namespace attn {
 namespace tc {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 128;
+constexpr int BM = PF_BM;  // query rows per CTA
+constexpr int BN = PF_BN;  // keys per tile
 constexpr int NUM_WARPS = 22;
 constexpr int NUM_THREADS = NUM_WARPS * 32;
 constexpr int WARP_ROPE0 = 16;
@@ -63,138 +55,34 @@ constexpr float LN2 = 0.6931471805599453f;
 
 template <int HD>
 struct Cfg {
-  static constexpr int NS = HD == 128 ? 4 : 10;  // key/value ring stages
+  static constexpr int NS = HD == 128 ? 5 : 12;  // key/value ring stages
   static constexpr int Q_BYTES = BM * HD * 2;
   static constexpr int KV_BYTES = BN * HD * 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_KV = OFF_Q + Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
-  static constexpr int NBAR = 3 * NS + 15;
+  static constexpr int NBAR = 3 * NS + 18;
+  // the MMA thread waits for tile j+1's keys before issuing tile j's PV: the ring must hold
+  // more than two tiles so that those keys never wait for a stage only that PV frees
+  static_assert(NS >= 5, "ring depth");
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  // row-max exchange [parity][key quarter][128] and row-sum exchange [slot][key quarter][128]
+  // row-max exchange [parity][key quarter][128] and row-sum exchange [key quarter][128]
   static constexpr int OFF_RED = (OFF_MISC + 16 + 15) / 16 * 16;
-  static constexpr int RED_FLOATS = 2 * 4 * 128 + 2 * 4 * 128;
+  static constexpr int RED_FLOATS = 2 * 4 * 128 + 4 * 128;
   static constexpr int SMEM = OFF_RED + RED_FLOATS * 4 + 1024;  // + slack to align the base
+  // tensor-memory columns
+  static constexpr int COL_O = 0;
+  static constexpr int COL_Q = HD;
+  static constexpr int COL_S = 256;
+  static_assert(COL_Q + HD / 2 <= COL_S && COL_S + 2 * BN <= 512, "tensor memory layout");
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, 0, 1);
 };
 
 struct TcArgs {
   PrefillParams p;
-  int group;       // H / KV
-  int two_heads;   // 1: slots are two heads at the same rows; 0: one head, two row tiles
-  int npairs;      // slot pairs per key/value head
-  int nqb;         // query blocks per (sequence, pair)
+  int nqb;         // query blocks of 128 rows per (sequence, head)
   float scale_log2;
-};
-
-// Rotation of a whole key (or query) tile by the 128 threads of the rotary warpgroup. Thread t owns
-// one 16-byte chunk (4 pairs) of the row and the rows phase, phase + PH, phase + 2 PH ...
-// Along those rows the angle of a pair grows by the fixed step PH * w, so the cosine and
-// sine follow the angle-addition recurrence (c, s) <- (c C - s S, s C + c S) with (C, S)
-// the step's cosine and sine, computed once per CTA. A query tile's start angle is computed
-// accurately; consecutive key tiles take theirs from the previous one by the same recurrence
-// with the step BN * w (rotate_next), so fp32 rounding builds up over the tiles of one CTA
-// (a few hundred steps at most, far below bf16 resolution). Eight threads of a quarter warp
-// cover the 8 chunks of one 128-byte row: shared-memory accesses are free of bank
-// conflicts. Only FMA-pipe arithmetic runs per element.
-template <int HD>
-struct KRot {
-  static constexpr int CH = HD / 8;       // 16-byte chunks per row
-  static constexpr int PH = 128 / CH;     // row step between a thread's rows
-  static constexpr int NR = BN / PH;      // rows per thread
-  int chunk, phase;
-  float stepc[4], steps[4];
-  f2x TC[2], TS[2];  // cosine and sine of the key-tile step BN * w (pairs 0-1, 2-3 of the chunk)
-  f2x KC[2], KS[2];  // start angle of the next key tile
-  __device__ __forceinline__ void init(int t, const RopeFreqs& rope) {
-    chunk = t % CH;
-    phase = t / CH;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int pc = chunk * 4 + e;
-      rope_cos_sin(PH, rope.hi[pc], rope.lo[pc], stepc[e], steps[e]);
-    }
-  }
-  // The key tiles that follow start at position pos_row0 (first tile), pos_row0 + BN, ...
-  __device__ __forceinline__ void start_keys(int pos_row0, const RopeFreqs& rope) {
-    float c[4], sn[4], tc[4], ts[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int pc = chunk * 4 + e;
-      rope_cos_sin(pos_row0 + phase, rope.hi[pc], rope.lo[pc], c[e], sn[e]);
-      rope_cos_sin(BN, rope.hi[pc], rope.lo[pc], tc[e], ts[e]);
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      KC[h] = pk2(c[2 * h], c[2 * h + 1]);
-      KS[h] = pk2(sn[2 * h], sn[2 * h + 1]);
-      TC[h] = pk2(tc[2 * h], tc[2 * h + 1]);
-      TS[h] = pk2(ts[2 * h], ts[2 * h + 1]);
-    }
-  }
-  // Rotate the next key tile, then advance the start angle by BN rows.
-  __device__ __forceinline__ void rotate_next(uint8_t* tile) {
-    rotate_from(tile, KC, KS);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const f2x Cn = fma2(neg2(KS[h]), TS[h], mul2(KC[h], TC[h]));
-      KS[h] = fma2(KC[h], TS[h], mul2(KS[h], TC[h]));
-      KC[h] = Cn;
-    }
-  }
-  // Rotate a tile whose first row sits at position pos_row0 (start angle computed accurately).
-  __device__ __forceinline__ void rotate(uint8_t* tile, int pos_row0, const RopeFreqs& rope) const {
-    float c[4], sn[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int pc = chunk * 4 + e;
-      rope_cos_sin(pos_row0 + phase, rope.hi[pc], rope.lo[pc], c[e], sn[e]);
-    }
-    const f2x C0[2] = {pk2(c[0], c[1]), pk2(c[2], c[3])};
-    const f2x S0[2] = {pk2(sn[0], sn[1]), pk2(sn[2], sn[3])};
-    rotate_from(tile, C0, S0);
-  }
-  __device__ __forceinline__ void rotate_from(uint8_t* tile, const f2x (&C0)[2], const f2x (&S0)[2]) const {
-    // pairs (0, 1) and (2, 3) of the chunk are handled two at a time in packed f32x2 form
-    f2x C[2], S[2], N[2], SC[2], SS[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      C[h] = C0[h];
-      S[h] = S0[h];
-      N[h] = neg2(S[h]);
-      SC[h] = pk2(stepc[2 * h], stepc[2 * h + 1]);
-      SS[h] = pk2(steps[2 * h], steps[2 * h + 1]);
-    }
-    const uint32_t base = smem_u32(tile);
-#pragma unroll 4
-    for (int k = 0; k < NR; ++k) {
-      const int r = phase + PH * k;
-      const uint32_t addr = base + sw128_offset(r, chunk * 8, BN);
-      const uint4 u = lds128(addr);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-      uint32_t o[4];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t wa = w[2 * h], wb = w[2 * h + 1];
-        const f2x X = pk2(__uint_as_float(wa << 16), __uint_as_float(wb << 16));
-        const f2x Y = pk2(__uint_as_float(wa & 0xffff0000u), __uint_as_float(wb & 0xffff0000u));
-        const f2x Xr = fma2(Y, N[h], mul2(X, C[h]));   // x c - y s
-        const f2x Yr = fma2(X, S[h], mul2(Y, C[h]));   // x s + y c
-        float xa, xb, ya, yb;
-        up2(Xr, xa, xb);
-        up2(Yr, ya, yb);
-        o[2 * h] = f2_to_bf2(xa, ya);
-        o[2 * h + 1] = f2_to_bf2(xb, yb);
-        // advance both angles by the step: (c, s) <- (c C - s S, s C + c S)
-        const f2x Cn = fma2(N[h], SS[h], mul2(C[h], SC[h]));
-        S[h] = fma2(C[h], SS[h], mul2(S[h], SC[h]));
-        C[h] = Cn;
-        N[h] = neg2(S[h]);
-      }
-      sts128(addr, make_uint4(o[0], o[1], o[2], o[3]));
-    }
-  }
 };
 
 // CHUNK: the queries continue sequences held in a cache (PrefillParams::seqlens != nullptr).
@@ -212,37 +100,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* kv_empty = bars + C::NS;
   uint64_t* k_rot = bars + 2 * C::NS;
   uint64_t* q_full = bars + 3 * C::NS;
-  uint64_t* q_rot = q_full + 1;
-  uint64_t* s_full = q_full + 2;
-  uint64_t* p_full = q_full + 4;
-  uint64_t* o_done = q_full + 6;
-  uint64_t* drain = q_full + 8;  // the MMA thread's final commit
-  uint64_t* red_bar = q_full + 9;    // [parity of the slot-tile count]: all warps' row maxima written
-  uint64_t* lsum_bar = q_full + 13;  // [slot]: all warps' row sums written
+  uint64_t* q_turned = q_full + 1;  // all rotary threads turned their query chunks in place
+  uint64_t* q_rot = q_full + 2;     // the query tile is in tensor memory
+  uint64_t* s_full = q_full + 3;    // [S buffer]: a QK completed
+  uint64_t* p_full = q_full + 5;    // [S buffer]: P written (and O rescaled)
+  uint64_t* o_done = q_full + 7;    // a PV completed
+  uint64_t* red_bar = q_full + 8;   // [parity of the tile count][lane quarter]: the four warps of
+                                    // those rows wrote their maxima
+  uint64_t* lsum_bar = q_full + 16; // all warps' row sums written
+  uint64_t* drain = q_full + 17;    // the MMA thread's final commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
   const PrefillParams& p = a.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- work unit: longest rows first
-  const int per_qb = p.B * p.KV * a.npairs;
+  // ---- work unit: longest rows first; the heads of a key/value group adjacent
+  const int per_qb = p.B * p.H;
   const int qb = a.nqb - 1 - (int)(blockIdx.x / per_qb);
-  int rest = blockIdx.x % per_qb;
-  const int pair = rest % a.npairs;
-  rest /= a.npairs;
-  const int g = rest % p.KV;
-  const int b = rest / p.KV;
-  int head[2], qs[2];
-  if (a.two_heads) {
-    head[0] = g * a.group + 2 * pair;
-    head[1] = head[0] + 1;
-    qs[0] = qs[1] = qb * BM;
-  } else {
-    head[0] = head[1] = g * a.group + pair;
-    qs[0] = qb * 2 * BM;
-    qs[1] = qs[0] + BM;
-  }
+  const int rest = blockIdx.x % per_qb;
+  const int h = rest % p.H;
+  const int b = rest / p.H;
+  const int g = h / (p.H / p.KV);
+  const int qs = qb * BM;
   // Keys are indexed by position in k/v (a prefill: key j = row j) or by cache slot (chunk
   // mode); qoff is the key index of query row 0 and Tk the number of keys there are.
   int qoff = 0, Tk = p.T, qrope0 = p.pos0;
@@ -256,20 +136,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       Tk = 0;  // nothing is attended: zero rows
     }
   }
-  int t0[2], t1[2];
-  bool valid[2], has[2];
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    valid[s] = qs[s] < p.T;
-    const int lo = p.window > 0 ? max(0, qoff + qs[s] - p.window + 1) : 0;
-    const int hi = p.causal ? min(Tk - 1, qoff + qs[s] + BM - 1) : Tk - 1;
-    has[s] = valid[s] && lo <= hi;  // the slot attends at least one key
-    t0[s] = has[s] ? lo / BN : 1;
-    t1[s] = has[s] ? hi / BN : 0;
-  }
-  const int jt0 = has[0] ? (has[1] ? min(t0[0], t0[1]) : t0[0]) : t0[1];
-  const int jt1 = has[0] ? (has[1] ? max(t1[0], t1[1]) : t1[0]) : t1[1];
-  auto active = [&](int s, int j) { return has[s] && j >= t0[s] && j <= t1[s]; };
+  const int lo = p.window > 0 ? max(0, qoff + qs - p.window + 1) : 0;
+  const int hi = p.causal ? min(Tk - 1, qoff + qs + BM - 1) : Tk - 1;
+  const bool has = lo <= hi;  // the tile attends at least one key
+  const int jt0 = has ? lo / BN : 1, jt1 = has ? hi / BN : 0;
 
   // ---- set-up: barriers, tensor memory
   if (tid == 0) {
@@ -279,14 +149,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(k_rot + i, 128);
     }
     mbar_init(q_full, 1);
+    mbar_init(q_turned, 128);
     mbar_init(q_rot, 128);
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(p_full + s, 16);  // one arrival per softmax warp
-      mbar_init(red_bar + s, 16);
-      mbar_init(lsum_bar + s, 16);
-      mbar_init(o_done + s, 1);
+      mbar_init(p_full + s, 16);   // one arrival per softmax warp
+      for (int qq = 0; qq < 4; ++qq) mbar_init(red_bar + 4 * s + qq, 4);
     }
+    mbar_init(o_done, 1);
+    mbar_init(lsum_bar, 16);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -306,12 +177,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch(&tmQ);
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
-      const uint32_t qbytes = (valid[0] ? C::Q_BYTES : 0) + (valid[1] ? C::Q_BYTES : 0);
-      mbar_expect_tx(q_full, qbytes);
-      for (int s = 0; s < 2; ++s)
-        if (valid[s])
-          for (int kb = 0; kb < HD / 64; ++kb)
-            tma_load_4d(sQ + s * C::Q_BYTES + kb * BM * 128, &tmQ, q_full, kb * 64, head[s], qs[s], b);
+      mbar_expect_tx(q_full, C::Q_BYTES);
+      for (int kb = 0; kb < HD / 64; ++kb)
+        tma_load_4d(sQ + kb * BM * 128, &tmQ, q_full, kb * 64, h, qs, b);
       const int total = 2 * (jt1 - jt0 + 1);  // K and V of every tile
       int u = 0;
       for (; u < total; ++u) {
@@ -330,17 +198,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= WARP_ROPE0 && warp < WARP_ROPE0 + 4) {
     // ------------------------------------------------------------ rotary embedding
-    const int r = tid - WARP_ROPE0 * 32;  // row of a query tile this thread turns
+    const int r = tid - WARP_ROPE0 * 32;  // row of the query tile this thread moves to TMEM
     KRot<HD> krot;
     if (p.rope.on) krot.init(r, p.rope);
     if (!mbar_wait(q_full, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-    if (p.rope.on)
-      for (int s = 0; s < 2; ++s)
-        if (valid[s]) krot.rotate(sQ + s * C::Q_BYTES, qrope0 + qs[s], p.rope);
-    fence_proxy_async();
+    // Turn the query tile in place (thread = 16-byte chunk, rows by the angle recurrence),
+    // then each thread moves one row into the Q columns of tensor memory, where the QK MMAs
+    // read it as their A operand: column c holds features 2c (low half) and 2c + 1, one
+    // rotary pair.
+    if (p.rope.on) krot.rotate(sQ, qrope0 + qs, p.rope);
+    mbar_arrive(q_turned);
+    if (!mbar_wait(q_turned, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+    {
+      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t base = smem_u32(sQ);
+#pragma unroll
+      for (int hb = 0; hb < HD / 64; ++hb) {
+        uint32_t w[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 u = lds128(base + sw128_offset(r, hb * 64 + c * 8, BM));
+          w[4 * c] = u.x;
+          w[4 * c + 1] = u.y;
+          w[4 * c + 2] = u.z;
+          w[4 * c + 3] = u.w;
+        }
+        tmem_st32u(tmem + lane_off + C::COL_Q + hb * 32, w);
+      }
+      tmem_wait_st();
+    }
+    tc_fence_before();
     mbar_arrive(q_rot);
     // hd = 128: key-tile start angles by recurrence; hd = 64 (half the rotation work per
-    // tile, and registers are tighter) computes each accurately
+    // tile) computes each accurately
     if constexpr (HD == 128)
       if (p.rope.on && !CHUNK) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
     int u = 0;
@@ -361,67 +251,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == WARP_MMA) {
     // ------------------------------------------------------------ UMMA issue
     if (lane == 0) {
-      // Descriptors are built once; the start-address field (bits 0-13, in 16-byte
-      // units) is then advanced by plain additions that stay below 2^14.
-      const uint64_t dQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      // Descriptors are built once; the start-address field (bits 0-13, in 16-byte units)
+      // is then advanced by plain additions that stay below 2^14.
       const uint64_t dK = smem_desc_sw128(smem_u32(sKV), 16, 1024);
       const uint64_t dV = smem_desc_sw128(smem_u32(sKV), BN * 128, 1024);
-      auto issue_qk = [&](int s, int st) {
-        const uint32_t d = tmem + s * BN;
-        const uint64_t a0 = dQ + (uint64_t)((s * C::Q_BYTES) >> 4);
+      auto issue_qk = [&](int buf, int st) {
+        const uint32_t d = tmem + C::COL_S + buf * BN;
+        const uint32_t aq = tmem + C::COL_Q;
         const uint64_t b0 = dK + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4;
-          umma_ss(d, a0 + off, b0 + off, C::IDESC_QK, kk > 0);
+          const uint32_t off = ((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4;
+          umma_ts(d, aq + kk * 8, b0 + off, C::IDESC_QK, kk > 0);
         }
       };
-      auto issue_pv = [&](int s, int st, bool acc) {
-        const uint32_t d = tmem + 2 * BN + s * HD;
-        const uint32_t aP = tmem + s * BN;  // P: 64 columns of bf16 pairs over the first half of S
+      auto issue_pv = [&](int buf, int st, bool acc) {
+        const uint32_t d = tmem + C::COL_O;
+        const uint32_t aP = tmem + C::COL_S + buf * BN;  // P: 64 columns of bf16 pairs over S
         const uint64_t b0 = dV + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
+        for (int kk = 0; kk < BN / 16; ++kk)
           umma_ts(d, aP + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
                   (kk > 0 || acc) ? 1u : 0u);
-        }
       };
-      int cnt[2] = {0, 0};
+      // ring use u of tile j: keys at u = 2 (j - jt0), values at u + 1
+      auto wait_rot = [&](int u) -> bool {
+        return mbar_wait(k_rot + u % C::NS, (u / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS);
+      };
       if (!mbar_wait(q_rot, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
-      if (jt1 < jt0) goto mma_drain;  // no key tile at all
-      // K of the first tile
-      if (!mbar_wait(k_rot + 0, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
+      if (!has) goto mma_drain;  // no key at all
+      if (!wait_rot(0)) goto mma_drain;
       tc_fence_after();
-      for (int s = 0; s < 2; ++s)
-        if (active(s, jt0)) {
-          issue_qk(s, 0);
-          umma_commit(s_full + s);
+      issue_qk(0, 0);
+      umma_commit(s_full);
+      umma_commit(kv_empty);
+      for (int i = 0; i <= jt1 - jt0; ++i) {
+        if (i < jt1 - jt0) {
+          const int uK = 2 * (i + 1);
+          if (!wait_rot(uK)) goto mma_drain;  // keys of the next tile, turned
+          tc_fence_after();
+          issue_qk((i + 1) & 1, uK % C::NS);
+          umma_commit(s_full + ((i + 1) & 1));
+          umma_commit(kv_empty + uK % C::NS);
         }
-      umma_commit(kv_empty + 0);
-      for (int j = jt0; j <= jt1; ++j) {
-        const int uV = 2 * (j - jt0) + 1, stV = uV % C::NS;
-        const int uK = uV + 1, stK = uK % C::NS;
-        const bool next = j < jt1;
-        if (!mbar_wait(k_rot + stV, (uV / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
-        for (int s = 0; s < 2; ++s) {
-          if (active(s, j)) {
-            if (!mbar_wait(p_full + s, cnt[s] & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
-            tc_fence_after();
-            issue_pv(s, stV, cnt[s] > 0);
-            umma_commit(o_done + s);
-            ++cnt[s];
-          }
-          if (next && s == 0) {
-            if (!mbar_wait(k_rot + stK, (uK / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
-            tc_fence_after();
-          }
-          if (next && active(s, j + 1)) {
-            issue_qk(s, stK);
-            umma_commit(s_full + s);
-          }
-        }
-        umma_commit(kv_empty + stV);
-        if (next) umma_commit(kv_empty + stK);
+        const int uV = 2 * i + 1;
+        if (!wait_rot(uV)) goto mma_drain;
+        if (!mbar_wait(p_full + (i & 1), (i >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
+        tc_fence_after();
+        issue_pv(i & 1, uV % C::NS, i > 0);
+        umma_commit(o_done);
+        umma_commit(kv_empty + uV % C::NS);
       }
     mma_drain:
       // every MMA issued above completes before tensor memory is released
@@ -430,75 +309,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 0-15)
-    // All sixteen warps work on one slot at a time, slot 0 then slot 1 for every key tile, so
-    // the tensor core runs one slot's PV and next QK while the other slot's weights are
-    // formed. Warp w owns TMEM lanes 32*(w%4).. (32 query rows) and keys kq*32 .. kq*32+31 of
-    // the tile, kq = w/4: one 32-column TMEM load per thread per slot and tile. The four
-    // warps of a row exchange their maxima through shared memory (an mbarrier per parity of
-    // the slot-tile count), all derive the same row reference, and each writes the P (bf16)
-    // of its 32 keys to TMEM columns kq*16 .. kq*16+15 of the slot's S region; every S column
-    // was read before the exchange, so P may overwrite any of them. O is rescaled (rarely)
-    // by column quarter.
+    // Warp w owns TMEM lanes 32*(w%4).. (32 query rows) and keys kq*32 .. kq*32+31 of every
+    // tile, kq = w/4: one 32-column TMEM load per thread and tile. The four warps of a row
+    // exchange their maxima through shared memory (an mbarrier per parity of the tile count
+    // and lane quarter), all derive the same row reference, and each writes the P (bf16) of
+    // its 32 keys to TMEM columns kq*16 .. kq*16+15 of the tile's S buffer; every S column of
+    // those rows was read before the exchange, so P may overwrite any of them. O is rescaled (rarely) by column
+    // quarter, once the previous tile's PV has completed.
     const int kq = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [parity][kq][128] row maxima
-    float* lsum = red + 2 * 4 * 128;                            // [slot][kq][128] row sums
+    float* lsum = red + 2 * 4 * 128;                            // [kq][128] row sums
     const float sc = a.scale_log2;
-    // Row state per slot in the log2 domain: m_ref is the reference the weights are taken
-    // against (-inf until the row has seen an allowed key), l the running sum of this warp's
-    // share of the weights. The reference moves only when a tile's maximum exceeds it by
-    // more than 8 (a factor 256), so O is rescaled rarely; weights stay below 2^8.
-    float m_ref0 = -INFINITY, m_ref1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    int cs0 = 0, cs1 = 0, t = 0;
+    const int i = qs + r;     // query row
+    const int ip = qoff + i;  // the query's key index
+    const float slope = p.alibi.on ? p.alibi.slope[h] * LOG2E : 0.f;
+    // Row state in the log2 domain: m_ref is the reference the weights are taken against
+    // (-inf until the row has seen an allowed key), l the running sum of this warp's share
+    // of the weights. The reference moves only when a tile's maximum exceeds it by more than
+    // 8 (a factor 256), so O is rescaled rarely; weights stay below 2^8.
+    float m_ref = -INFINITY, l = 0.f;
+    int c = 0;
+    if (has) {
 #pragma unroll 1
-    for (int j = jt0; j <= jt1; ++j) {
-#pragma unroll 1
-      for (int s = 0; s < 2; ++s) {
-        if (!active(s, j)) continue;
-        // this slot's row state (scalars selected by slot: no indexed local arrays)
-        const int c = s ? cs1 : cs0;
-        float m_ref = s ? m_ref1 : m_ref0;
-        if (!mbar_wait(s_full + s, c & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      for (int j = jt0; j <= jt1; ++j, ++c) {
+        const int buf = c & 1;
+        if (!mbar_wait(s_full + buf, (c >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
         tc_fence_after();
-        const int q0s = qs[s];  // first query row of the slot
-        const int hs = head[s];
-        const int i = q0s + r;
-        const int ip = qoff + i;  // the query's key index
-        const uint32_t tS = tmem + lane_off + s * BN;
+        const uint32_t tS = tmem + lane_off + C::COL_S + buf * BN;
         const int key0 = j * BN + kq * 32;  // first of my 32 keys
-        const float slope = p.alibi.on ? p.alibi.slope[hs] * LOG2E : 0.f;
-        // does any row of this slot need per-element masking in my keys of this tile?
-        const bool need_mask = (key0 + 32 > Tk) || (p.causal && key0 + 31 > qoff + q0s) ||
-                               (p.window > 0 && qoff + q0s + BM - 1 - key0 >= p.window);
-        const bool plain = !need_mask && !p.alibi.on;
+        // does any row of this tile need per-element masking in my keys? (uniform per warp)
+        const bool need_mask = (key0 + 32 > Tk) || (p.causal && key0 + 31 > qoff + qs) ||
+                               (p.window > 0 && qoff + qs + BM - 1 - key0 >= p.window);
         float x[32];
         tmem_ld32(tS + kq * 32, x);
         tmem_wait_ld();
-        float hx = -INFINITY;
-        if (plain) {
+        if (p.alibi.on) {
+          // -slope |i - j| is, with the causal mask, slope (j - i) on every allowed pair: an
+          // affine function c0 + slope k of the key
+          const float c0 = slope * (float)(key0 - ip);
 #pragma unroll
-          for (int k = 0; k < 16; ++k) hx = max3(hx, x[2 * k], x[2 * k + 1]);
-          hx *= sc;  // a positive scale keeps the order: max then scale is exact
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int jk = key0 + k;
-            float v = p.alibi.on ? fmaf(x[k], sc, -slope * fabsf((float)(ip - jk))) : x[k] * sc;
-            if (need_mask) {
-              const bool ok = jk < Tk && (!p.causal || jk <= ip) && (p.window <= 0 || ip - jk < p.window);
-              v = ok ? v : -INFINITY;
-            }
-            x[k] = v;
-          }
-#pragma unroll
-          for (int k = 0; k < 16; ++k) hx = max3(hx, x[2 * k], x[2 * k + 1]);
+          for (int k = 0; k < 32; ++k)
+            x[k] = p.causal ? fmaf(x[k], sc, fmaf(slope, (float)k, c0))
+                            : fmaf(x[k], sc, -slope * fabsf((float)(ip - key0 - k)));
         }
-        float* rb = red + (t & 1) * 512;
+        if (need_mask) {
+          // my keys allowed for this row: kmin <= k < kmax
+          int kmax = Tk - key0;
+          if (p.causal) kmax = min(kmax, ip - key0 + 1);
+          const int kmin = p.window > 0 ? ip - p.window + 1 - key0 : 0;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) x[k] = (k >= kmin && k < kmax) ? x[k] : -INFINITY;
+        }
+        // without ALiBi the scores are still unscaled: a positive scale keeps the order
+        const float hx = p.alibi.on ? max32(x) : max32(x) * sc;
+        float* rb = red + buf * 512;
         rb[kq * 128 + r] = hx;
         __syncwarp();
-        if (lane == 0) mbar_arrive(red_bar + (t & 1));
-        if (!mbar_wait(red_bar + (t & 1), (t >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+        if (lane == 0) mbar_arrive(red_bar + 4 * buf + (warp & 3));
+        if (!mbar_wait(red_bar + 4 * buf + (warp & 3), (c >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS))
+          goto done;
         const float mt = fmaxf(fmaxf(rb[r], rb[128 + r]), fmaxf(rb[256 + r], rb[384 + r]));
         const float m_new = (mt > m_ref + 8.f) ? mt : m_ref;  // takes mt when m_ref = -inf
         const float alpha = (m_new == m_ref) ? 1.f : ex2(m_ref - m_new);
@@ -506,42 +377,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         m_ref = m_new;
         f2x RS = pk2(0.f, 0.f);
         uint32_t pk[16];  // column k: keys 2k, 2k+1 of my 32 (low half = even key)
-        if (plain) {
-          const f2x SC = pk2(sc, sc), NM = pk2(-mu, -mu);
+        const f2x SC = p.alibi.on ? pk2(1.f, 1.f) : pk2(sc, sc), NM = pk2(-mu, -mu);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            float a0, a1, b0, b1;
-            up2(fma2(pk2(x[4 * k], x[4 * k + 1]), SC, NM), a0, a1);
-            up2(fma2(pk2(x[4 * k + 2], x[4 * k + 3]), SC, NM), b0, b1);
-            const float e0 = ex2(a0), e1 = ex2(a1), e2 = ex2(b0), e3 = ex2(b1);
-            RS = add2(RS, add2(pk2(e0, e1), pk2(e2, e3)));
-            pk[2 * k] = f2_to_bf2(e0, e1);
-            pk[2 * k + 1] = f2_to_bf2(e2, e3);
-          }
-        } else {
-          const f2x NM = pk2(-mu, -mu);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            float a0, a1, b0, b1;
-            up2(add2(pk2(x[4 * k], x[4 * k + 1]), NM), a0, a1);
-            up2(add2(pk2(x[4 * k + 2], x[4 * k + 3]), NM), b0, b1);
-            const float e0 = ex2(a0), e1 = ex2(a1), e2 = ex2(b0), e3 = ex2(b1);
-            RS = add2(RS, add2(pk2(e0, e1), pk2(e2, e3)));
-            pk[2 * k] = f2_to_bf2(e0, e1);
-            pk[2 * k + 1] = f2_to_bf2(e2, e3);
-          }
+        for (int k = 0; k < 8; ++k) {
+          float a0, a1, b0, b1;
+          up2(fma2(pk2(x[4 * k], x[4 * k + 1]), SC, NM), a0, a1);
+          up2(fma2(pk2(x[4 * k + 2], x[4 * k + 3]), SC, NM), b0, b1);
+          const float e0 = ex2(a0), e1 = ex2(a1), e2 = ex2(b0), e3 = ex2(b1);
+          RS = add2(RS, add2(pk2(e0, e1), pk2(e2, e3)));
+          pk[2 * k] = f2_to_bf2(e0, e1);
+          pk[2 * k + 1] = f2_to_bf2(e2, e3);
         }
         tmem_st16u(tS + kq * 16, pk);
-        float rs;
-        {
-          float r0, r1;
-          up2(RS, r0, r1);
-          rs = r0 + r1;
-        }
-        // O is rescaled before this tile's PV is issued. The previous PV of this slot has
-        // completed: it was issued before the QK whose completion this tile waited for.
+        // O is rescaled before this tile's PV is issued, once the previous PV has completed
+        // (the tile before the previous one completed before this tile's QK)
         if (c > 0 && kq * 32 < HD && __any_sync(0xffffffffu, alpha != 1.f)) {
-          const uint32_t tO = tmem + lane_off + 2 * BN + s * HD + kq * 32;
+          if (!mbar_wait(o_done, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+          tc_fence_after();
+          const uint32_t tO = tmem + lane_off + C::COL_O + kq * 32;
           float o[32];
           tmem_ld32(tO, o);
           tmem_wait_ld();
@@ -549,59 +402,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int e = 0; e < 32; ++e) o[e] *= alpha;
           tmem_st32(tO, o);
         }
-        if (s) {
-          l1 = l1 * alpha + rs;
-          m_ref1 = m_ref;
-          cs1 = c + 1;
-        } else {
-          l0 = l0 * alpha + rs;
-          m_ref0 = m_ref;
-          cs0 = c + 1;
+        {
+          float r0, r1;
+          up2(RS, r0, r1);
+          l = l * alpha + (r0 + r1);
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + s);
-        ++t;
+        if (lane == 0) mbar_arrive(p_full + buf);
       }
     }
-#pragma unroll 1
-    for (int s = 0; s < 2; ++s) {
-      const int c = s ? cs1 : cs0;
-      if (c == 0) {
-        // a slot that attends no key at all (a chunk over an empty range): zero rows, lse -inf
-        const int i = qs[s] + r;
-        if (valid[s] && i < p.T) {
-          if (kq * 32 < HD) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                                  (((size_t)b * p.T + i) * p.H + head[s]) * HD + kq * 32);
+    // ---- epilogue: out = O / l (bf16), lse = (m + log2 l) ln 2
+    if (c == 0) {
+      // a tile that attends no key at all (a chunk over an empty range): zero rows, lse -inf
+      if (i < p.T) {
+        if (kq * 32 < HD) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                (((size_t)b * p.T + i) * p.H + h) * HD + kq * 32);
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
-          }
-          if (p.lse && kq == 0) p.lse[((size_t)b * p.H + head[s]) * p.T + i] = -INFINITY;
+          for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
         }
-        continue;
+        if (p.lse && kq == 0) p.lse[((size_t)b * p.H + h) * p.T + i] = -INFINITY;
       }
-      const float m_ref = s ? m_ref1 : m_ref0;
+    } else {
       // the row's total sum: the four warps' partial sums, exchanged through shared memory
-      lsum[(s * 4 + kq) * 128 + r] = s ? l1 : l0;
+      lsum[kq * 128 + r] = l;
       __syncwarp();
-      if (lane == 0) mbar_arrive(lsum_bar + s);
-      if (!mbar_wait(lsum_bar + s, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-      const float* ls = lsum + s * 4 * 128 + r;
-      const float lt = (ls[0] + ls[128]) + (ls[256] + ls[384]);
-      if (!mbar_wait(o_done + s, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      if (lane == 0) mbar_arrive(lsum_bar);
+      if (!mbar_wait(lsum_bar, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      const float lt = (lsum[r] + lsum[128 + r]) + (lsum[256 + r] + lsum[384 + r]);
+      if (!mbar_wait(o_done, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
       tc_fence_after();
-      const int hs = head[s];
-      const int i = qs[s] + r;
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       if (kq * 32 < HD) {
         float o[32];
-        tmem_ld32(tmem + lane_off + 2 * BN + s * HD + kq * 32, o);
+        tmem_ld32(tmem + lane_off + C::COL_O + kq * 32, o);
         tmem_wait_ld();
         if (i < p.T) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                                (((size_t)b * p.T + i) * p.H + hs) * HD + kq * 32);
+                                                (((size_t)b * p.T + i) * p.H + h) * HD + kq * 32);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
             dst[v4] = make_uint4(f2_to_bf2(o[8 * v4] * inv, o[8 * v4 + 1] * inv),
@@ -611,7 +451,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       if (p.lse && i < p.T && kq == 0)
-        p.lse[((size_t)b * p.H + hs) * p.T + i] = lt > 0.f ? (m_ref + __log2f(lt)) * LN2 : -INFINITY;
+        p.lse[((size_t)b * p.H + h) * p.T + i] = lt > 0.f ? (m_ref + __log2f(lt)) * LN2 : -INFINITY;
     }
   }
 done:
@@ -624,34 +464,6 @@ done:
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-// 4-D map over [B][T][heads][hd] bf16 with a box of 128 rows x 64 features of one head.
-bool make_map(CUtensorMap* map, const void* base, int B, int T, int heads, int hd) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)T, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)hd * 2, (cuuint64_t)heads * hd * 2,
-                                 (cuuint64_t)T * heads * hd * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int HD>
 cudaError_t launch_hd(const PrefillParams& p, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
@@ -661,13 +473,9 @@ cudaError_t launch_hd(const PrefillParams& p, cudaStream_t s) {
     return cudaErrorInvalidValue;
   TcArgs a;
   a.p = p;
-  a.group = p.H / p.KV;
-  a.two_heads = (a.group % 2 == 0) ? 1 : 0;
-  a.npairs = a.two_heads ? a.group / 2 : a.group;
-  const int rows = a.two_heads ? BM : 2 * BM;
-  a.nqb = (p.T + rows - 1) / rows;
+  a.nqb = (p.T + BM - 1) / BM;
   a.scale_log2 = p.scale * LOG2E;
-  const long long units = (long long)p.B * p.KV * a.npairs * a.nqb;
+  const long long units = (long long)p.B * p.H * a.nqb;
   if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
   auto kern = p.seqlens ? prefill_tc_kernel<HD, true> : prefill_tc_kernel<HD, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<HD>::SMEM);
@@ -684,6 +492,9 @@ bool prefill_tc_supported(const PrefillParams& p, int dtype) {
 }
 
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t s) {
+  // hd = 128 with the keys turned in the kernel: the two-slot kernel turns each key tile
+  // once per 256 query rows instead of once per 128
+  if (p.hd == 128 && p.rope.on && !p.seqlens) return launch_prefill_pair(p, s);
   return p.hd == 128 ? tc::launch_hd<128>(p, s) : tc::launch_hd<64>(p, s);
 }
 

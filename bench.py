@@ -299,7 +299,9 @@ def build_families(art, only):
             run(0)
             hout.copy_(outs[0], non_blocking=True)
 
-        kern = f"prefill_tc_kernel<{w.hd}, false>"
+        # hd = 128 with the keys turned in the kernel runs the two-slot kernel
+        kern = ("prefill_pair_kernel<128, false>" if w.hd == 128 and w.rope_base > 0
+                else f"prefill_tc_kernel<{w.hd}, false>")
         return Family(key, w.name, "TFLOP/s", "tensor", w.flops, 1, kern, run, reps=copies,
                       e2e=(tnb(q) + tnb(k) + tnb(v), tnb(q), e2e_step))
 
