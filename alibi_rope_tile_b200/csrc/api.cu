@@ -412,7 +412,7 @@ int attn_kv_write(const void* k_new, const void* v_new, void* kcache, void* vcac
 namespace {
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 struct BlockLayout {
-  size_t q, k, v, ctx, total;
+  size_t q, k, v, ctx, cs, total;
 };
 BlockLayout block_layout(int B, int T, int H, int KV, int hd, int dtype) {
   const size_t es = elem_size(dtype);
@@ -422,13 +422,34 @@ BlockLayout block_layout(int B, int T, int H, int KV, int hd, int dtype) {
   L.k = L.q + round256(nq);
   L.v = L.k + round256(nk);
   L.ctx = L.v + round256(nk);
-  L.total = L.ctx + round256(nq);
+  L.cs = L.ctx + round256(nq);
+  L.total = L.cs + round256((size_t)T * (hd / 2) * sizeof(float2));
   return L;
 }
 cudaError_t gemm(const void* A, const void* W, void* C, int M, int N, int K, int dtype, int* status,
                cudaStream_t s) {
   if (gemm_tc_supported(M, N, K, dtype)) return launch_gemm_tc(A, W, C, M, N, K, status, s);
   return launch_gemm_simt(A, W, C, M, N, K, dtype, s);
+}
+// The attention of the blocks: attn_prefill's launch, optionally over keys that the projection
+// epilogue already turned (k_rotated).
+int block_attention(const void* q, const void* k, const void* v, void* out, int B, int T, int H, int KV, int hd,
+                    long long pos0, float rope_base, int causal, int window, const float* alibi_slopes,
+                    int dtype, int k_rotated, int* status, cudaStream_t s) {
+  PrefillParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.k = k; p.v = v; p.out = out;
+  p.B = B; p.T = T; p.H = H; p.KV = KV; p.hd = hd;
+  p.pos0 = (int)pos0; p.causal = causal; p.window = window < 0 ? 0 : window;
+  p.scale = (float)(1.0 / std::sqrt((double)hd));
+  p.rope = make_rope(hd, rope_base);
+  p.k_rotated = k_rotated;
+  p.status = status;
+  int st;
+  if ((st = make_alibi(H, alibi_slopes, &p.alibi))) return st;
+  cudaError_t e = prefill_tc_supported(p, dtype) ? launch_prefill_tc(p, s) : launch_prefill_simt(p, dtype, s);
+  if (e != cudaSuccess) return cuda_fail(e, "block attention launch");
+  return ATTN_OK;
 }
 }  // namespace
 
@@ -451,6 +472,11 @@ int attn_block(const void* x, const void* Wq, const void* Wk, const void* Wv, co
       !aligned16(out) || (workspace && !aligned16(workspace)))
     return fail(ATTN_ERR_ALIGN, "x, weights, out and workspace must be 16-byte aligned");
   if (B < 1 || T < 1 || d < 1) return fail(ATTN_ERR_ARG, "B, T and d must be >= 1");
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
+  if (window < 0) window = 0;
+  if (window > 0 && !causal) return fail(ATTN_ERR_ARG, "a window requires the causal mask");
+  if (pos0 < 0 || pos0 + (long long)T >= (1LL << 24))
+    return fail(ATTN_ERR_ARG, "positions pos0..pos0+T-1 must lie in [0, 2^24)");
   const size_t need = attn_block_workspace_size(B, T, d, H, KV, hd, dtype);
   if (!workspace || ws_bytes < need)
     return fail(ATTN_ERR_WORKSPACE, "block needs %zu bytes of workspace (got %zu)", need, ws_bytes);
@@ -463,11 +489,36 @@ int attn_block(const void* x, const void* Wq, const void* Wk, const void* Wv, co
   int* status = device_status(&err);
   if (!status) return err;
   cudaError_t e;
-  if ((e = gemm(x, Wq, q, M, H * hd, d, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wq GEMM");
-  if ((e = gemm(x, Wk, k, M, KV * hd, d, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wk GEMM");
-  if ((e = gemm(x, Wv, v, M, KV * hd, d, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wv GEMM");
-  st = attn_prefill(q, k, v, ctx, nullptr, B, T, H, KV, hd, pos0, rope_base, causal, window,
-                    alibi_slopes, dtype, stream);
+  int k_rotated = 0;
+  const int Ns[3] = {H * hd, KV * hd, KV * hd};
+  if (gemm_tc_supported(M, H * hd, d, dtype) && gemm_tc_supported(M, KV * hd, d, dtype) &&
+      gemm_tc_segments_fit(3, Ns)) {
+    // x @ Wq, x @ Wk and x @ Wv as one launch over the three weights side by side; the keys
+    // are turned in its epilogue (q, turned once per query tile, is left to the attention)
+    const RopeFreqs rope = make_rope(hd, rope_base);
+    GemmEpilogue ep;
+    std::memset(&ep, 0, sizeof(ep));
+    ep.rot_seg = -1;
+    if (rope.on && (hd == 64 || hd == 128)) {
+      float2* cs = reinterpret_cast<float2*>(ws + L.cs);
+      if ((e = launch_rope_table(cs, T, (int)pos0, rope, hd, s)) != cudaSuccess) return cuda_fail(e, "block table");
+      ep.rot_seg = 1;
+      ep.rope_cs = cs;
+      ep.T = T;
+      ep.hd = hd;
+      k_rotated = 1;
+    }
+    const void* Ws[3] = {Wq, Wk, Wv};
+    void* Cs[3] = {q, k, v};
+    if ((e = launch_gemm_tc_multi(x, 3, Ws, Cs, Ns, M, d, status, s, &ep)) != cudaSuccess)
+      return cuda_fail(e, "block QKV GEMM");
+  } else {
+    if ((e = gemm(x, Wq, q, M, H * hd, d, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wq GEMM");
+    if ((e = gemm(x, Wk, k, M, KV * hd, d, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wk GEMM");
+    if ((e = gemm(x, Wv, v, M, KV * hd, d, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wv GEMM");
+  }
+  st = block_attention(q, k, v, ctx, B, T, H, KV, hd, pos0, rope_base, causal, window, alibi_slopes, dtype,
+                       k_rotated, status, s);
   if (st) return st;
   if ((e = gemm(ctx, Wo, out, M, d, H * hd, dtype, status, s)) != cudaSuccess) return cuda_fail(e, "block Wo GEMM");
   return ok();
@@ -475,13 +526,14 @@ int attn_block(const void* x, const void* Wq, const void* Wk, const void* Wv, co
 
 namespace {
 struct FusedLayout {
-  size_t xn, q, k, v, ctx, cs, total;
+  size_t wg, rinv, q, k, v, ctx, cs, total;
 };
 FusedLayout fused_layout(int B, int T, int d, int H, int KV, int hd) {
   FusedLayout L;
   const size_t M = (size_t)B * T;
-  L.xn = 0;
-  L.q = L.xn + round256(M * d * 2);
+  L.wg = 0;
+  L.rinv = L.wg + round256((size_t)d * (H + 2 * KV) * hd * 2);
+  L.q = L.rinv + round256(M * sizeof(float));
   L.k = L.q + round256(M * H * hd * 2);
   L.v = L.k + round256(M * KV * hd * 2);
   L.ctx = L.v + round256(M * KV * hd * 2);
@@ -520,9 +572,12 @@ int attn_block_fused(const void* x, const void* gamma, const void* Wqkv, const v
   const int M = B * T, Nqkv = (H + 2 * KV) * hd;
   if ((long long)B * T * (H + 2 * KV) * hd >= (1LL << 40) || (long long)B * T * d >= (1LL << 40))
     return fail(ATTN_ERR_ARG, "tensor too large");
-  if (dtype != ATTN_BF16 || (hd != 64 && hd != 128) || !gemm_tc_supported(M, Nqkv, d, dtype) ||
+  const int Ns[3] = {H * hd, KV * hd, KV * hd};
+  if (dtype != ATTN_BF16 || (hd != 64 && hd != 128) || !gemm_tc_supported(M, H * hd, d, dtype) ||
+      !gemm_tc_supported(M, KV * hd, d, dtype) || !gemm_tc_segments_fit(3, Ns) ||
       !gemm_tc_supported(M, d, H * hd, dtype))
-    return fail(ATTN_ERR_UNSUPPORTED, "attn_block_fused runs bf16 with hd 64 or 128 on the tensor-core GEMM");
+    return fail(ATTN_ERR_UNSUPPORTED,
+                "attn_block_fused runs bf16 with hd 64 or 128 on the tensor-core GEMM");
   const FusedLayout L = fused_layout(B, T, d, H, KV, hd);
   if (!workspace || ws_bytes < L.total)
     return fail(ATTN_ERR_WORKSPACE, "fused block needs %zu bytes of workspace (got %zu)", L.total, ws_bytes);
@@ -533,27 +588,38 @@ int attn_block_fused(const void* x, const void* gamma, const void* Wqkv, const v
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const RopeFreqs rope = make_rope(hd, rope_base);
   float2* cs = reinterpret_cast<float2*>(ws + L.cs);
+  float* rinv = reinterpret_cast<float*>(ws + L.rinv);
+  // RMSNorm folded into the projection: 1 / rms per row, gamma into the weights' rows
   cudaError_t e = cudaSuccess;
   if (rope.on) e = launch_rope_table(cs, T, (int)pos0, rope, hd, s);
-  if (e == cudaSuccess) e = launch_rmsnorm(x, gamma, ws + L.xn, M, d, eps, s);
+  if (e == cudaSuccess) e = launch_rms_inverse(x, rinv, M, d, eps, s);
+  if (e == cudaSuccess) e = launch_fold_gamma(Wqkv, gamma, ws + L.wg, d, Nqkv, s);
   if (e != cudaSuccess) return cuda_fail(e, "fused block norm");
+  // (x @ [Wq | Wk | Wv] with gamma folded) / rms, the keys turned, k and v also into the cache
   GemmEpilogue qkv;
   std::memset(&qkv, 0, sizeof(qkv));
-  qkv.mode = 1;
-  qkv.T = T; qkv.H = H; qkv.KV = KV; qkv.hd = hd;
+  qkv.row_scale = rinv;
+  qkv.rot_seg = rope.on ? 1 : -1;
   qkv.rope_cs = rope.on ? cs : nullptr;
-  qkv.q = ws + L.q; qkv.k = ws + L.k; qkv.v = ws + L.v;
-  qkv.kcache = kcache; qkv.vcache = vcache; qkv.Lmax = Lmax; qkv.pos0 = (int)pos0;
-  if ((e = launch_gemm_tc(ws + L.xn, Wqkv, nullptr, M, Nqkv, d, status, s, &qkv)) != cudaSuccess)
+  qkv.T = T;
+  qkv.hd = hd;
+  qkv.cache[1] = kcache;
+  qkv.cache[2] = vcache;
+  qkv.Lmax = Lmax;
+  qkv.pos0 = (int)pos0;
+  const char* wg = ws + L.wg;
+  const void* Ws[3] = {wg, wg + (size_t)H * hd * 2, wg + (size_t)(H + KV) * hd * 2};
+  void* Cs[3] = {ws + L.q, ws + L.k, ws + L.v};
+  if ((e = launch_gemm_tc_multi(x, 3, Ws, Cs, Ns, M, d, status, s, &qkv, Nqkv)) != cudaSuccess)
     return cuda_fail(e, "fused block QKV GEMM");
-  // q and k are already turned: the attention runs without rotation (its masks and ALiBi depend
-  // only on i - j)
-  st = attn_prefill(ws + L.q, ws + L.k, ws + L.v, ws + L.ctx, nullptr, B, T, H, KV, hd, pos0, 0.f, causal,
-                    window, alibi_slopes, dtype, stream);
+  // the keys arrive turned: the attention turns only q (its masks and ALiBi depend on i - j)
+  st = block_attention(ws + L.q, ws + L.k, ws + L.v, ws + L.ctx, B, T, H, KV, hd, pos0, rope_base, causal,
+                       window, alibi_slopes, dtype, 1, status, s);
   if (st) return st;
   GemmEpilogue res;
   std::memset(&res, 0, sizeof(res));
   res.mode = 2;
+  res.rot_seg = -1;
   res.residual = x;
   if ((e = launch_gemm_tc(ws + L.ctx, Wo, out, M, d, H * hd, status, s, &res)) != cudaSuccess)
     return cuda_fail(e, "fused block Wo GEMM");

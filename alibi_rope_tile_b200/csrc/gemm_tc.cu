@@ -10,10 +10,13 @@
 // warps 0-3 read the accumulator back (one TMEM lane = one row of C per thread) and store
 // bf16. Rows and columns past M, N are zero-filled on load and not stored.
 //
-// Epilogues (GemmEpilogue): a plain store; the fused block's QKV scatter, which sends each
-// 32-column chunk (within one head, since hd is 64 or 128 and tiles start at multiples of 256)
-// to q, k or v, turns q and k pairwise by the (cos, sin) table of its row's position, and
-// also writes k and v rows into a KV cache; or the output projection plus a residual.
+// The weights may come as up to three matrices side by side (the block's x @ Wq, x @ Wk, x @ Wv
+// in one launch: a CTA's columns fall in one of them, whose tensor map and output it uses).
+//
+// Epilogues (GemmEpilogue): a store, optionally with each row scaled (the fused block's
+// 1/RMS), one segment's heads turned pairwise by the (cos, sin) table of the row's position
+// (the keys: a 32-column chunk lies in one head, since hd is 64 or 128 and tiles start at
+// multiples of 256), and segments copied into a KV cache; or C = A W plus a residual.
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -38,9 +41,14 @@ constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 1);
 constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;
 
+// Up to three weight matrices side by side (x @ [W0 | W1 | W2] with separate outputs): segment
+// i covers columns [seg_end[i-1], seg_end[i]) of the launch; every boundary but the last is a
+// multiple of 64, so each 64-column W box and each 32-column output chunk lies in one segment.
 struct GemmArgs {
-  __nv_bfloat16* C;
-  int M, N, K;
+  __nv_bfloat16* C[3];
+  int seg_end[3];
+  int nseg;
+  int M, N, K;  // N: all segments' columns
   int* status;
   GemmEpilogue ep;
 };
@@ -54,7 +62,8 @@ __device__ __forceinline__ void store32(__nv_bfloat16* dst, const float (&v)[32]
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW0,
+                   const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
                    const __grid_constant__ GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -66,8 +75,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1) + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  const int gn0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
   const int nk = (g.K + BK - 1) / BK;
+  // the segment of a column of the launch
+  auto seg_of = [&](int col) {
+    return (g.nseg > 1 && col >= g.seg_end[0]) ? ((g.nseg > 2 && col >= g.seg_end[1]) ? 2 : 1) : 0;
+  };
 
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -91,18 +104,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 4) {
     if (lane == 0) {
       tma_prefetch(&tmA);
-      tma_prefetch(&tmW);
+      tma_prefetch(&tmW0);
+      if (g.nseg > 1) tma_prefetch(&tmW1);
+      if (g.nseg > 2) tma_prefetch(&tmW2);
       int kb = 0;
       for (; kb < nk; ++kb) {
         const int st = kb % NS, n = kb / NS;
         if (!mbar_wait(empty + st, (n & 1) ^ 1, abort_flag, g.status, WAIT_LIMIT_NS)) break;
         uint8_t* sa = smem + st * STAGE;
         // W boxes that start past N are not loaded: those columns of C are not stored
-        const int nbv = min(BN / 64, (g.N - n0 + 63) / 64);
+        const int nbv = min(BN / 64, (g.N - gn0 + 63) / 64);
         mbar_expect_tx(full + st, A_BYTES + nbv * (BK * 128));
         tma_load_2d(sa, &tmA, full + st, kb * BK, m0);
         for (int nb = 0; nb < nbv; ++nb)
-          tma_load_2d(sa + A_BYTES + nb * (BK * 128), &tmW, full + st, n0 + nb * 64, kb * BK);
+          {
+            const int col = gn0 + nb * 64, sg = seg_of(col);
+            tma_load_2d(sa + A_BYTES + nb * (BK * 128), sg == 0 ? &tmW0 : (sg == 1 ? &tmW1 : &tmW2), full + st,
+                        col - (sg == 0 ? 0 : g.seg_end[sg - 1]), kb * BK);
+          }
       }
       // the copies issued last land before the CTA exits
       for (int w = (kb > NS ? kb - NS : 0); w < kb; ++w) mbar_wait_drain(full + w % NS, (w / NS) & 1, DRAIN_LIMIT_NS);
@@ -137,39 +156,53 @@ __global__ void __launch_bounds__(THREADS, 1)
         float v[32];
         tmem_ld32(t + c0, v);
         tmem_wait_ld();
-        if (row < g.M && g.ep.mode == 1) {
+        // this chunk's segment, its output and width, and the tile's first column in it
+        const int seg = seg_of(gn0 + c0);
+        const int seg0 = seg == 0 ? 0 : g.seg_end[seg - 1];
+        const int Ns = g.seg_end[seg] - seg0, n0 = gn0 - seg0;
+        __nv_bfloat16* const Cs = g.C[seg];
+        if (row < g.M && g.ep.mode == 0) {
           const GemmEpilogue& e = g.ep;
           const int n = n0 + c0;
-          if (n < g.N) {
-            const int b = row / e.T, t = row - b * e.T;
-            const int hh = n / e.hd, d = n - hh * e.hd;
-            const int region = hh < e.H ? 0 : (hh < e.H + e.KV ? 1 : 2);
-            const int head = region == 0 ? hh : (region == 1 ? hh - e.H : hh - e.H - e.KV);
-            if (region < 2 && e.rope_cs) {
-              const float2* cs = e.rope_cs + (size_t)t * (e.hd / 2) + d / 2;
+          if (n < Ns) {
+            if (e.row_scale) {
+              const float f = e.row_scale[row];
 #pragma unroll
-              for (int p = 0; p < 16; ++p) {
-                const float2 c = cs[p];
-                const float x = v[2 * p], y = v[2 * p + 1];
-                v[2 * p] = x * c.x - y * c.y;
-                v[2 * p + 1] = x * c.y + y * c.x;
+              for (int i = 0; i < 32; ++i) v[i] *= f;
+            }
+            const int bb = e.T > 0 ? row / e.T : 0, tt = row - bb * e.T;  // sequence and position
+            if (seg == e.rot_seg && e.rope_cs) {
+              // turn each pair (2c, 2c+1) of the head by the angle of this row's position
+              const int d = n % e.hd;
+              const float2* cs = e.rope_cs + (size_t)tt * (e.hd / 2) + d / 2;
+#pragma unroll
+              for (int pp = 0; pp < 16; ++pp) {
+                const float2 c = cs[pp];
+                const float x = v[2 * pp], y = v[2 * pp + 1];
+                v[2 * pp] = x * c.x - y * c.y;
+                v[2 * pp + 1] = x * c.y + y * c.x;
               }
             }
-            const int nh = region == 0 ? e.H : e.KV;
-            __nv_bfloat16* base = static_cast<__nv_bfloat16*>(region == 0 ? e.q : (region == 1 ? e.k : e.v));
-            store32(base + (((size_t)b * e.T + t) * nh + head) * e.hd + d, v);
-            if (region > 0 && e.kcache) {
-              __nv_bfloat16* cache = static_cast<__nv_bfloat16*>(region == 1 ? e.kcache : e.vcache);
-              store32(cache + (((size_t)b * e.Lmax + e.pos0 + t) * e.KV + head) * e.hd + d, v);
+            if (n + 32 <= Ns) {
+              store32(Cs + (size_t)row * Ns + n, v);
+              if (e.cache[seg])
+                store32(static_cast<__nv_bfloat16*>(e.cache[seg]) + ((size_t)bb * e.Lmax + e.pos0 + tt) * Ns + n, v);
+            } else {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if (n + 8 * q + 8 <= Ns)
+                  *reinterpret_cast<uint4*>(Cs + (size_t)row * Ns + n + 8 * q) =
+                      make_uint4(f2_to_bf2(v[8 * q], v[8 * q + 1]), f2_to_bf2(v[8 * q + 2], v[8 * q + 3]),
+                                 f2_to_bf2(v[8 * q + 4], v[8 * q + 5]), f2_to_bf2(v[8 * q + 6], v[8 * q + 7]));
             }
           }
         } else if (row < g.M) {
-          __nv_bfloat16* dst = g.C + (size_t)row * g.N + n0 + c0;
-          if (g.ep.mode == 2) {
-            const __nv_bfloat16* res = static_cast<const __nv_bfloat16*>(g.ep.residual) + (size_t)row * g.N + n0 + c0;
+          __nv_bfloat16* dst = Cs + (size_t)row * Ns + n0 + c0;
+          {
+            const __nv_bfloat16* res = static_cast<const __nv_bfloat16*>(g.ep.residual) + (size_t)row * Ns + n0 + c0;
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              if (n0 + c0 + 8 * q + 8 <= g.N) {
+              if (n0 + c0 + 8 * q + 8 <= Ns) {
                 const uint4 u = *reinterpret_cast<const uint4*>(res + 8 * q);
                 const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -182,7 +215,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            if (n0 + c0 + 8 * q + 8 <= g.N)
+            if (n0 + c0 + 8 * q + 8 <= Ns)
               *reinterpret_cast<uint4*>(dst + 8 * q) =
                   make_uint4(f2_to_bf2(v[8 * q], v[8 * q + 1]), f2_to_bf2(v[8 * q + 2], v[8 * q + 3]),
                              f2_to_bf2(v[8 * q + 4], v[8 * q + 5]), f2_to_bf2(v[8 * q + 6], v[8 * q + 7]));
@@ -212,12 +245,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D map over a row-major [rows][cols] bf16 matrix with a box of box_rows x 64 columns.
-bool make_map2d(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+// 2-D map over a row-major [rows][cols] bf16 matrix (rows ld elements apart; 0: cols) with a
+// box of box_rows x 64 columns.
+bool make_map2d(CUtensorMap* map, const void* base, int rows, int cols, int box_rows, int ld = 0) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ld > 0 ? ld : cols) * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
@@ -234,23 +268,49 @@ bool gemm_tc_supported(int M, int N, int K, int dtype) {
          tcgemm::encode_fn() != nullptr;
 }
 
-cudaError_t launch_gemm_tc(const void* A, const void* W, void* C, int M, int N, int K, int* status,
-                           cudaStream_t s, const GemmEpilogue* ep) {
+bool gemm_tc_segments_fit(int nseg, const int* Ns) {
+  for (int i = 0; i + 1 < nseg; ++i)
+    if (Ns[i] % 64) return false;
+  return true;
+}
+
+cudaError_t launch_gemm_tc_multi(const void* A, int nseg, const void* const* Ws, void* const* Cs, const int* Ns,
+                                 int M, int K, int* status, cudaStream_t s, const GemmEpilogue* ep, int ldw) {
   using namespace tcgemm;
-  CUtensorMap ma, mw;
-  if (!make_map2d(&ma, A, M, K, BM) || !make_map2d(&mw, W, K, N, BK)) return cudaErrorInvalidValue;
+  if (nseg < 1 || nseg > 3 || !gemm_tc_segments_fit(nseg, Ns)) return cudaErrorInvalidValue;
+  CUtensorMap ma, mw[3];
+  if (!make_map2d(&ma, A, M, K, BM)) return cudaErrorInvalidValue;
   GemmArgs g;
-  g.C = static_cast<__nv_bfloat16*>(C);
+  std::memset(&g, 0, sizeof(g));
+  int end = 0;
+  for (int i = 0; i < 3; ++i) {
+    const int j = i < nseg ? i : nseg - 1;  // unused maps repeat the last segment's
+    if (!make_map2d(&mw[i], Ws[j], K, Ns[j], BK, ldw)) return cudaErrorInvalidValue;
+    if (i < nseg) {
+      end += Ns[i];
+      g.seg_end[i] = end;
+      g.C[i] = static_cast<__nv_bfloat16*>(Cs[i]);
+    }
+  }
+  g.nseg = nseg;
   g.M = M;
-  g.N = N;
+  g.N = end;
   g.K = K;
   g.status = status;
-  std::memset(&g.ep, 0, sizeof(g.ep));
-  if (ep) g.ep = *ep;
+  if (ep) {
+    g.ep = *ep;
+  } else {
+    g.ep.rot_seg = -1;
+  }
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  gemm_tc_kernel<<<dim3((N + BN - 1) / BN, (M + BM - 1) / BM), THREADS, SMEM, s>>>(ma, mw, g);
+  gemm_tc_kernel<<<dim3((end + BN - 1) / BN, (M + BM - 1) / BM), THREADS, SMEM, s>>>(ma, mw[0], mw[1], mw[2], g);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(const void* A, const void* W, void* C, int M, int N, int K, int* status,
+                           cudaStream_t s, const GemmEpilogue* ep) {
+  return launch_gemm_tc_multi(A, 1, &W, &C, &N, M, K, status, s, ep);
 }
 
 }  // namespace attn

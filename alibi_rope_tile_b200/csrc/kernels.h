@@ -29,6 +29,9 @@ struct PrefillParams {
   const int* seqlens;
   const int* qpos0;
   int Lk;
+  // Keys arrive turned at positions pos0 + j (a block's key projection turned them in its
+  // epilogue): only the queries are turned here.
+  int k_rotated;
 };
 
 // CUDA-core flash prefill: fp32 or bf16 elements, any even hd <= 256.
@@ -96,27 +99,35 @@ cudaError_t launch_gemm_simt(const void* A, const void* W, void* C, int M, int N
 // Tensor-core (tcgen05) version for bf16 when M, N, K fit its tiles.
 // Epilogues of the tensor-core GEMM beyond a plain store of C (bf16).
 struct GemmEpilogue {
-  int mode;  // 0: C = A W; 1: scatter the columns [q heads | k heads | v heads] of A Wqkv to
-             // q [B,T,H,hd], k, v [B,T,KV,hd] (row m = b*T + t), turning q and k by rope_cs,
-             // and also write k, v to kcache, vcache slot pos0 + t when kcache != nullptr;
-             // 2: C = A W + residual ([M,N])
-  int T, H, KV, hd;
-  const float2* rope_cs;  // [T][hd/2] (cos, sin) of position pos0 + t, or nullptr
-  void* q;
-  void* k;
-  void* v;
-  void* kcache;
-  void* vcache;
+  int mode;                // 0: C = A W with the options below; 2: C = A W + residual ([M,N])
+  const float* row_scale;  // [M] or nullptr: row m of C scaled by row_scale[m]
+  int rot_seg;             // segment whose heads are turned (-1: none): pairs (2c, 2c+1) of each
+                           // hd-wide head by the (cos, sin) of the row's position, from rope_cs
+                           // [T][hd/2] with t = m % T
+  const float2* rope_cs;
+  int T, hd;
+  void* cache[3];          // per segment, or nullptr: also written into a cache [B][Lmax][Ns] at
+                           // row slot pos0 + t (B = M / T)
   int Lmax, pos0;
   const void* residual;
 };
 bool gemm_tc_supported(int M, int N, int K, int dtype);
 cudaError_t launch_gemm_tc(const void* A, const void* W, void* C, int M, int N, int K, int* status,
                            cudaStream_t s, const GemmEpilogue* ep = nullptr);
+// One launch over nseg <= 3 weight matrices side by side: C_i [M, Ns[i]] = A @ W_i. Every
+// segment but the last must be a multiple of 64 columns wide (gemm_tc_segments_fit).
+bool gemm_tc_segments_fit(int nseg, const int* Ns);
+// The weights W_i are [K, Ns[i]] with rows ldw elements apart (0: Ns[i]), so they may be column
+// blocks of one matrix.
+cudaError_t launch_gemm_tc_multi(const void* A, int nseg, const void* const* Ws, void* const* Cs, const int* Ns,
+                                 int M, int K, int* status, cudaStream_t s, const GemmEpilogue* ep = nullptr,
+                                 int ldw = 0);
 
-// Pre-norm helpers of the fused block: y = RMSNorm(x) * gamma per row (bf16), and the table of
-// (cos, sin) of every (position pos0 + t, pair) the QKV epilogue turns by.
-cudaError_t launch_rmsnorm(const void* x, const void* gamma, void* y, int M, int d, float eps, cudaStream_t s);
+// Pre-norm helpers of the fused block: the inverse root-mean-square of every row of x, 1 / sqrt(mean
+// (x^2) + eps) (fp32), the weights with gamma folded into their rows, Wg[k][n] = gamma[k] W[k][n]
+// (bf16), and the table of (cos, sin) of every (position pos0 + t, pair) an epilogue turns by.
+cudaError_t launch_rms_inverse(const void* x, float* rinv, int M, int d, float eps, cudaStream_t s);
+cudaError_t launch_fold_gamma(const void* W, const void* gamma, void* Wg, int d, int N, cudaStream_t s);
 cudaError_t launch_rope_table(float2* cs, int T, int pos0, const RopeFreqs& rope, int hd, cudaStream_t s);
 
 // Records a failure for attn_last_error() and returns ``code`` (used by entry points

@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(128) prefill_simt_kernel(const PrefillParams p
         const float2 ke = Elem<T>::load2(k + off);
         const float2 ve = Elem<T>::load2(v + off);
         kx = ke.x; ky = ke.y; vx = ve.x; vy = ve.y;
-        if (p.rope.on) {
+        if (p.rope.on && !p.k_rotated) {
           float cs, sn;
           rope_cos_sin(p.pos0 + j, p.rope.hi[c], p.rope.lo[c], cs, sn);
           rotate_pair(kx, ky, cs, sn);

@@ -232,13 +232,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // hd = 128: key-tile start angles by recurrence; hd = 64 (half the rotation work per
     // tile) computes each accurately
     if constexpr (HD == 128)
-      if (p.rope.on && !CHUNK) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
+      if (p.rope.on && !CHUNK && !p.k_rotated) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
     int u = 0;
     for (int j = jt0; j <= jt1; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++u) {
         const int st = u % C::NS, n = u / C::NS;
         if (!mbar_wait(kv_full + st, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        if (kv == 0 && p.rope.on && !CHUNK) {  // cached keys are already rotated
+        if (kv == 0 && p.rope.on && !CHUNK && !p.k_rotated) {  // cached keys are already rotated
           if constexpr (HD == 128)
             krot.rotate_next(sKV + st * C::KV_BYTES);
           else
@@ -494,7 +494,7 @@ bool prefill_tc_supported(const PrefillParams& p, int dtype) {
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t s) {
   // hd = 128 with the keys turned in the kernel: the two-slot kernel turns each key tile
   // once per 256 query rows instead of once per 128
-  if (p.hd == 128 && p.rope.on && !p.seqlens) return launch_prefill_pair(p, s);
+  if (p.hd == 128 && p.rope.on && !p.seqlens && !p.k_rotated) return launch_prefill_pair(p, s);
   return p.hd == 128 ? tc::launch_hd<128>(p, s) : tc::launch_hd<64>(p, s);
 }
 
