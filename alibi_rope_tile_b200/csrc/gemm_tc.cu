@@ -4,11 +4,13 @@
 // so W is consumed as stored: as the B operand it is MN-major (N contiguous), which the
 // UMMA shared-memory descriptor expresses directly; nothing is transposed.
 //
-// One CTA computes a 128 x 256 tile of C. K is staged by 64 through a 4-stage TMA ring
-// (A: one 128 x 64 box; W: four 64 x 64 boxes, 128-byte swizzle). Warp 4 issues the TMA
-// loads, warp 5 allocates TMEM and issues the M=128, N=256, K=16 MMAs (four per stage),
-// warps 0-3 read the accumulator back (one TMEM lane = one row of C per thread) and store
-// bf16. Rows and columns past M, N are zero-filled on load and not stored.
+// The kernel is persistent: one CTA per SM computes 128 x 256 tiles of C in turn (tile
+// blockIdx.x, then + gridDim.x, ...). K is staged by 64 through a 4-stage TMA ring that runs on
+// across tiles (A: one 128 x 64 box; W: four 64 x 64 boxes, 128-byte swizzle). Warp 4 issues
+// the TMA loads, warp 5 allocates TMEM and issues the M=128, N=256, K=16 MMAs (four per stage)
+// into one of two 256-column accumulators, and warps 0-3 read the other accumulator back (one
+// TMEM lane = one row of C per thread) and store bf16: a tile's epilogue overlaps the next
+// tile's MMAs. Rows and columns past M, N are zero-filled on load and not stored.
 //
 // The weights may come as up to three matrices side by side (the block's x @ Wq, x @ Wk, x @ Wv
 // in one launch: a CTA's columns fall in one of them, whose tensor map and output it uses).
@@ -36,7 +38,7 @@ constexpr int A_BYTES = BM * BK * 2;       // 16 KB
 constexpr int B_BYTES = BK * BN * 2;       // 32 KB
 constexpr int STAGE = A_BYTES + B_BYTES;
 constexpr int OFF_BAR = NS * STAGE;
-constexpr int SMEM = OFF_BAR + (2 * NS + 2) * 8 + 16 + 1024;
+constexpr int SMEM = OFF_BAR + (2 * NS + 5) * 8 + 16 + 1024;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 1);
 constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;
@@ -69,13 +71,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* empty = full + NS;
-  uint64_t* acc_full = full + 2 * NS;
-  uint64_t* drain = acc_full + 1;
+  uint64_t* acc_full = full + 2 * NS;   // [accumulator]: a tile's MMAs completed
+  uint64_t* acc_empty = acc_full + 2;   // [accumulator]: the epilogue read it
+  uint64_t* drain = acc_full + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1) + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gn0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  // persistent: this CTA's tiles are blockIdx.x, blockIdx.x + gridDim.x, ... in the order
+  // (row tile, column tile) with the column tile fastest
+  const int ntn = (g.N + BN - 1) / BN, ntiles = ntn * ((g.M + BM - 1) / BM);
   const int nk = (g.K + BK - 1) / BK;
   // the segment of a column of the launch
   auto seg_of = [&](int col) {
@@ -87,13 +92,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(full + i, 1);
       mbar_init(empty + i, 1);
     }
-    mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, 4);  // one arrival per epilogue warp
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 5) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);  // two 128 x 256 fp32 accumulators
     tmem_relinquish();
   }
   tc_fence_before();
@@ -107,50 +115,81 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_prefetch(&tmW0);
       if (g.nseg > 1) tma_prefetch(&tmW1);
       if (g.nseg > 2) tma_prefetch(&tmW2);
-      int kb = 0;
-      for (; kb < nk; ++kb) {
-        const int st = kb % NS, n = kb / NS;
-        if (!mbar_wait(empty + st, (n & 1) ^ 1, abort_flag, g.status, WAIT_LIMIT_NS)) break;
-        uint8_t* sa = smem + st * STAGE;
+      int u = 0;  // ring uses so far
+      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+        const int gn0 = (tile % ntn) * BN, m0 = (tile / ntn) * BM;
         // W boxes that start past N are not loaded: those columns of C are not stored
         const int nbv = min(BN / 64, (g.N - gn0 + 63) / 64);
-        mbar_expect_tx(full + st, A_BYTES + nbv * (BK * 128));
-        tma_load_2d(sa, &tmA, full + st, kb * BK, m0);
-        for (int nb = 0; nb < nbv; ++nb)
-          {
-            const int col = gn0 + nb * 64, sg = seg_of(col);
-            tma_load_2d(sa + A_BYTES + nb * (BK * 128), sg == 0 ? &tmW0 : (sg == 1 ? &tmW1 : &tmW2), full + st,
-                        col - (sg == 0 ? 0 : g.seg_end[sg - 1]), kb * BK);
+        // the tile's W map, chosen once when the whole tile lies in one segment (choosing it per
+        // box costs ~10% of the GEMM); per box only for a tile across a narrow segment
+        const int sgt = seg_of(gn0);
+        const bool one_seg = sgt == seg_of(min(gn0 + BN, g.N) - 1);
+        const CUtensorMap* tmWt = sgt == 0 ? &tmW0 : (sgt == 1 ? &tmW1 : &tmW2);
+        const int lc0 = gn0 - (sgt == 0 ? 0 : g.seg_end[sgt - 1]);
+        for (int kb = 0; kb < nk; ++kb, ++u) {
+          const int st = u % NS, n = u / NS;
+          if (!mbar_wait(empty + st, (n & 1) ^ 1, abort_flag, g.status, WAIT_LIMIT_NS)) break;
+          uint8_t* sa = smem + st * STAGE;
+          mbar_expect_tx(full + st, A_BYTES + nbv * (BK * 128));
+          tma_load_2d(sa, &tmA, full + st, kb * BK, m0);
+          if (one_seg) {
+            for (int nb = 0; nb < nbv; ++nb)
+              tma_load_2d(sa + A_BYTES + nb * (BK * 128), tmWt, full + st, lc0 + nb * 64, kb * BK);
+          } else {
+            for (int nb = 0; nb < nbv; ++nb) {
+              const int col = gn0 + nb * 64, sg = seg_of(col);
+              tma_load_2d(sa + A_BYTES + nb * (BK * 128), sg == 0 ? &tmW0 : (sg == 1 ? &tmW1 : &tmW2), full + st,
+                          col - (sg == 0 ? 0 : g.seg_end[sg - 1]), kb * BK);
+            }
           }
+        }
       }
       // the copies issued last land before the CTA exits
-      for (int w = (kb > NS ? kb - NS : 0); w < kb; ++w) mbar_wait_drain(full + w % NS, (w / NS) & 1, DRAIN_LIMIT_NS);
+      for (int w = (u > NS ? u - NS : 0); w < u; ++w) mbar_wait_drain(full + w % NS, (w / NS) & 1, DRAIN_LIMIT_NS);
     }
   } else if (warp == 5) {
     if (lane == 0) {
       const uint64_t dA = smem_desc_sw128(smem_u32(smem), 16, 1024);
       const uint64_t dW = smem_desc_sw128(smem_u32(smem + A_BYTES), BK * 128, 1024);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int st = kb % NS, n = kb / NS;
-        if (!mbar_wait(full + st, n & 1, abort_flag, g.status, WAIT_LIMIT_NS)) break;
+      int u = 0, i = 0;  // ring uses and tiles so far
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+        // accumulator i % 2, free once the epilogue has read the tile two before
+        const int ab = i & 1;
+        if (!mbar_wait(acc_empty + ab, ((i >> 1) & 1) ^ 1, abort_flag, g.status, WAIT_LIMIT_NS)) break;
         tc_fence_after();
-        const uint64_t so = (uint64_t)((st * STAGE) >> 4);
+        const uint32_t acc = tmem + ab * BN;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb, ++u) {
+          const int st = u % NS, n = u / NS;
+          if (!mbar_wait(full + st, n & 1, abort_flag, g.status, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t so = (uint64_t)((st * STAGE) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          umma_ss(tmem, dA + so + (uint64_t)((kk * 32) >> 4), dW + so + (uint64_t)((kk * 16 * 128) >> 4),
-                  IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(empty + st);
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_ss(acc, dA + so + (uint64_t)((kk * 32) >> 4), dW + so + (uint64_t)((kk * 16 * 128) >> 4),
+                    IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(empty + st);
+        }
+        if (!ok) break;
+        umma_commit(acc_full + ab);
       }
-      umma_commit(acc_full);
       umma_commit(drain);
       mbar_wait_drain(drain, 0, DRAIN_LIMIT_NS);  // every MMA completes before TMEM is freed
     }
   } else {
-    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = rows m0 + 32*w .. of C
-    if (mbar_wait(acc_full, 0, abort_flag, g.status, WAIT_LIMIT_NS)) {
+    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = rows m0 + 32*w .. of C, tile after
+    // tile, while the MMAs of the next tile fill the other accumulator
+    int it = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+      const int gn0 = (tile % ntn) * BN, m0 = (tile / ntn) * BM;
+      const int ab = it & 1;
+      if (!mbar_wait(acc_full + ab, (it >> 1) & 1, abort_flag, g.status, WAIT_LIMIT_NS)) break;
       tc_fence_after();
       const int row = m0 + warp * 32 + lane;
-      const uint32_t t = tmem + ((uint32_t)(warp * 32) << 16);
+      const uint32_t t = tmem + ab * BN + ((uint32_t)(warp * 32) << 16);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         float v[32];
@@ -221,13 +260,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                              f2_to_bf2(v[8 * q + 4], v[8 * q + 5]), f2_to_bf2(v[8 * q + 6], v[8 * q + 7]));
         }
       }
+      // every TMEM load of this accumulator completed (each chunk waited for its own)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + ab);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -304,7 +347,14 @@ cudaError_t launch_gemm_tc_multi(const void* A, int nseg, const void* const* Ws,
   }
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  gemm_tc_kernel<<<dim3((end + BN - 1) / BN, (M + BM - 1) / BM), THREADS, SMEM, s>>>(ma, mw[0], mw[1], mw[2], g);
+  // persistent: one CTA per SM (its shared memory admits one) over the tiles
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const long long tiles = (long long)((end + BN - 1) / BN) * ((M + BM - 1) / BM);
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const int grid = tiles < sms ? (int)tiles : sms;
+  gemm_tc_kernel<<<grid, THREADS, SMEM, s>>>(ma, mw[0], mw[1], mw[2], g);
   return cudaGetLastError();
 }
 
