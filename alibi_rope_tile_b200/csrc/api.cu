@@ -338,8 +338,8 @@ size_t r256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t attn_decode_latent_workspace_size(int B, int H, int hd, int dc, int Lmax) {
   if (B < 1 || H < 1 || hd < 2 || (dc != 64 && dc != 128) || Lmax < 1) return 0;
-  const size_t vec = r256((size_t)B * H * dc * 2);  // q' and the latent output, bf16
-  return 2 * vec + decode_workspace_bytes(B, H, 1, dc, Lmax);
+  const size_t vec = r256((size_t)B * H * dc * 2);  // q' (bf16)
+  return vec + decode_workspace_bytes(B, H, 1, dc, Lmax);
 }
 
 int attn_decode_latent(const void* q, const void* ccache, const void* W_uk, const void* W_uv,
@@ -354,8 +354,8 @@ int attn_decode_latent(const void* q, const void* ccache, const void* W_uk, cons
       (lse && !aligned16(lse)) || (workspace && !aligned16(workspace)))
     return fail(ATTN_ERR_ALIGN, "q, ccache, weights, out, lse and workspace must be 16-byte aligned");
   if (B < 1 || Lmax < 1 || Lmax >= (1 << 24)) return fail(ATTN_ERR_ARG, "B >= 1 and 1 <= Lmax < 2^24");
-  if (dtype != ATTN_BF16 || (dc != 64 && dc != 128) || H > 32)
-    return fail(ATTN_ERR_UNSUPPORTED, "attn_decode_latent runs bf16 with dc 64 or 128 and H <= 32");
+  if (dtype != ATTN_BF16 || (dc != 64 && dc != 128) || H > 32 || hd % 8)
+    return fail(ATTN_ERR_UNSUPPORTED, "attn_decode_latent runs bf16 with dc 64 or 128, H <= 32 and hd % 8 == 0");
   if (window < 0) window = 0;
   const size_t need = attn_decode_latent_workspace_size(B, H, hd, dc, Lmax);
   if (!workspace || ws_bytes < need)
@@ -363,13 +363,13 @@ int attn_decode_latent(const void* q, const void* ccache, const void* W_uk, cons
   char* ws = static_cast<char*>(workspace);
   const size_t vec = r256((size_t)B * H * dc * 2);
   void* qlat = ws;
-  void* olat = ws + vec;
-  void* dws = ws + 2 * vec;
+  void* dws = ws + vec;
 
   DecodeParams p;
   std::memset(&p, 0, sizeof(p));
   p.q = qlat; p.kcache = ccache; p.vcache = ccache;  // keys and values are the same latents
-  p.seqlens = seqlens; p.qpos = qpos; p.out = olat; p.lse = lse;
+  p.seqlens = seqlens; p.qpos = qpos; p.out = out; p.lse = lse;
+  p.W_out = W_uv; p.hd_out = hd;  // the merge applies the value up-projection
   p.B = B; p.H = H; p.KV = 1; p.hd = dc; p.Lmax = Lmax; p.window = window;
   p.scale = (float)(1.0 / std::sqrt((double)hd));  // the scores are q . k of head dimension hd
   p.rope = make_rope(dc, 0.f);                      // no rotation on the latent path
@@ -379,9 +379,8 @@ int attn_decode_latent(const void* q, const void* ccache, const void* W_uk, cons
   p.status = device_status(&err);
   if (!p.status) return err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_head_proj(true, q, W_uk, qlat, B, H, dc, hd, s);
+  cudaError_t e = launch_latent_fold(q, W_uk, qlat, B, H, dc, hd, s);
   if (e == cudaSuccess) e = launch_decode(p, dtype, dws, s);
-  if (e == cudaSuccess) e = launch_head_proj(false, olat, W_uv, out, B, H, dc, hd, s);
   if (e != cudaSuccess) return cuda_fail(e, "attn_decode_latent launch");
   return ok();
 }

@@ -4,17 +4,22 @@
 // page's FlashAttention equations by the merge kernel in decode.cu.
 //
 // One CTA = one (split of the cache rows, key/value head, sequence); splits are 2048 keys
-// (fewer CTAs amortise the set-up; see decode_chunk). The H/KV query heads
-// served by the key/value head are the rows of a 128-row MMA tile (rows >= H/KV are zero),
-// so the scores S = Q K^T of a 128-key tile land in tensor memory one head per TMEM lane:
-// the softmax of a head is a row-wise online softmax done by one thread, with no
-// cross-thread reduction. P (bf16) is written back over the S columns and PV is the
-// TS-form MMA. The padded rows cost tensor-core time that decode does not miss: the
-// kernel is bound by streaming K and V from HBM, which TMA does through a two-stage ring
-// (two CTAs per SM keep four 32 KB tiles in flight per SM).
+// (fewer CTAs amortise the set-up; see decode_chunk). The H/KV query heads served by the
+// key/value head sit in every 32-row quarter of a 128-row MMA tile (row 32k + i holds head i
+// for i < H/KV, other rows are zero), so the scores S = Q K^T of a 128-key tile land in
+// tensor memory once per TMEM lane quarter. Warp k, which addresses lane quarter k, does the
+// softmax of keys 32k..32k+31 for every head (one head per lane): the four warps sit on the
+// four SM sub-partitions and share a tile's exponentials, where one warp alone would work
+// through all 128 keys. They agree on each head's running maximum through shared memory and
+// write P (bf16) for their quarter of the keys, zeros for the rest, over the S columns of
+// their lanes; the TS-form PV MMA then accumulates in quarter k the part of O that keys of
+// quarter k contribute. The four parts share one reference maximum and are added when the
+// split's partial state is written. The replicated and padded rows cost tensor-core time
+// that decode does not miss: the kernel is bound by streaming K and V from HBM, which TMA
+// does through a two-stage ring (two CTAs per SM keep four 32 KB tiles in flight per SM).
 //
-// Warps: 0 = softmax (lanes 0..H/KV-1 hold one head each) and query set-up, 1 = TMA
-// producer, 2 = TMEM allocation and MMA issue, 3 = query set-up only.
+// Warps: 0-3 = softmax (quarter = warp), 4 = TMA producer, 5 = TMEM allocation and MMA
+// issue; all six set up the query tile.
 // The cached keys are already rotated at their slot positions; only q is rotated here,
 // at qpos[b]. Keys at or beyond seqlens[b] and, with a window, keys j with
 // qpos - j >= window get weight exactly 0.
@@ -34,7 +39,8 @@ using namespace attn::tc;
 constexpr int BN = 128;               // keys per tile
 constexpr int BM = 128;               // MMA rows (query heads, zero padded)
 constexpr int NS = 2;                 // ring stages (K, V alternate)
-constexpr int THREADS = 128;
+constexpr int THREADS = 192;          // 4 softmax warps, the TMA warp, the MMA warp
+constexpr int TMA_WARP = 4, MMA_WARP = 5;
 constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;  // own copies/MMAs finish in microseconds
 constexpr float LOG2E = 1.4426950408889634f;
@@ -45,14 +51,20 @@ struct Cfg {
   static constexpr int KV_BYTES = BN * HD * 2;
   static constexpr int OFF_KV = Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
-  static constexpr int NBAR = 2 * NS + 5;  // kv_full[NS], kv_empty[NS], s_full, p_full, o_done, never, drain
+  // kv_full[NS], kv_empty[NS], s_full, p_full, o_done, never, drain, red_bar[2], fin_bar
+  static constexpr int NBAR = 2 * NS + 8;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;  // (two CTAs per SM stay within 196 KB)
+  // the softmax warps' exchange: running maxima red[2][4][32], row-sum parts lpart[4][32]
+  static constexpr int OFF_RED = (OFF_MISC + 16 + 15) / 16 * 16;
+  static constexpr int RED_BYTES = (2 * 4 * 32 + 4 * 32) * 4;
+  static constexpr int OFF_TAB = OFF_RED + RED_BYTES;
+  static constexpr int SMEM = OFF_TAB + 1024;  // (two CTAs per SM stay within 200 KB)
   // paged cache only: the page index of every block of a split (a split holds at most
   // 2048 / page_size <= 256 pages), reserved only when a paged decode is launched
   static constexpr int MAX_TAB = 256;
-  static constexpr int OFF_TAB = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr int SMEM_PAGED = OFF_TAB + MAX_TAB * 4 + 1024;
+  // the four O parts [4][HD][32] fp32 are added through the K/V ring once it is idle
+  static_assert(4 * HD * 32 * 4 <= NS * KV_BYTES, "O parts do not fit the ring");
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, 0, 1);
 };
@@ -65,6 +77,8 @@ struct DecArgs {
   void* ws;
   unsigned long long wait_ns;  // bound of every wait (4 s unless a test lowers it)
   int test_stall;              // test hook: the MMA warp waits on a barrier nothing signals
+  int kv_same;                 // keys and values are one cache (latent attention): each tile is
+                               // fetched once and serves as K in QK and as V in PV
 };
 
 template <int HD>
@@ -82,10 +96,14 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint64_t* s_full = bars + 2 * NS;
   uint64_t* p_full = s_full + 1;
   uint64_t* o_done = s_full + 2;
-  uint64_t* never = s_full + 3;  // not signalled by anything (test hook)
-  uint64_t* drain = s_full + 4;  // the MMA thread's final commit
+  uint64_t* never = s_full + 3;    // not signalled by anything (test hook)
+  uint64_t* drain = s_full + 4;    // the MMA thread's final commit
+  uint64_t* red_bar = s_full + 5;  // [2]: the four softmax warps posted a tile's maxima
+  uint64_t* fin_bar = s_full + 7;  // the four O parts are in shared memory
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [2][4][32]
+  float* lpart = red + 2 * 4 * 32;                           // [4][32]
 
   const DecodeParams& p = a.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -118,11 +136,11 @@ __global__ void __launch_bounds__(THREADS, 2)
     return;
   }
 
-  // ---- query tile: rows 0..G-1 = this group's heads turned at qpos, other rows zero.
-  // Work items are (row, 16-byte chunk) pairs spread over all threads.
+  // ---- query tile: head i (turned at qpos) in rows i, 32 + i, 64 + i and 96 + i for i < G,
+  // other rows zero. Work items are (head slot, 16-byte chunk) pairs spread over all threads.
   {
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q);
-    for (int it = tid; it < BM * (HD / 8); it += THREADS) {
+    for (int it = tid; it < 32 * (HD / 8); it += THREADS) {
       const int row = it / (HD / 8), c = it % (HD / 8);
       uint32_t w[4] = {0u, 0u, 0u, 0u};
       if (row < G) {
@@ -139,7 +157,9 @@ __global__ void __launch_bounds__(THREADS, 2)
           w[e] = f2_to_bf2(f.x, f.y);
         }
       }
-      sts128(smem_u32(sQ) + sw128_offset(row, c * 8, BM), make_uint4(w[0], w[1], w[2], w[3]));
+      const uint4 v = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sts128(smem_u32(sQ) + sw128_offset(32 * k + row, c * 8, BM), v);
     }
     fence_proxy_async();
   }
@@ -149,14 +169,17 @@ __global__ void __launch_bounds__(THREADS, 2)
       mbar_init(kv_empty + i, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 32);
+    mbar_init(p_full, 128);
     mbar_init(o_done, 1);
     mbar_init(never, 1);
     mbar_init(drain, 1);
+    mbar_init(red_bar, 128);
+    mbar_init(red_bar + 1, 128);
+    mbar_init(fin_bar, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 2) {
+  if (warp == MMA_WARP) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
@@ -165,7 +188,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;  // S: columns 0..127 (P over 0..63), O: 128..128+HD-1
 
-  if (warp == 1) {
+  if (warp == TMA_WARP) {
     // ------------------------------------------------------------ TMA producer
     int* tab = reinterpret_cast<int*>(smem + C::OFF_TAB);
     if (p.block_table) {
@@ -190,15 +213,17 @@ __global__ void __launch_bounds__(THREADS, 2)
     if (lane == 0) {
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
-      const int total = 2 * (jt1 - jt0 + 1);  // K and V of every tile
+      const int per = a.kv_same ? 1 : 2;      // ring uses per tile: K then V, or one for both
+      const int total = per * (jt1 - jt0 + 1);
       int u = 0;
       for (; u < total; ++u) {
-        const int st = u % NS, n = u / NS, j = jt0 + u / 2;
+        const int st = u % NS, n = u / NS, j = jt0 + u / per;
+        const bool isv = per == 2 && (u & 1);
         if (!mbar_wait(kv_empty + st, (n & 1) ^ 1, abort_flag, p.status, a.wait_ns)) break;
         mbar_expect_tx(kv_full + st, C::KV_BYTES);
         if (!p.block_table) {
           for (int kb = 0; kb < HD / 64; ++kb)
-            tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, (u & 1) ? &tmV : &tmK, kv_full + st,
+            tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128, isv ? &tmV : &tmK, kv_full + st,
                         kb * 64, kvh, j * BN, b);
         } else {
           // one box per page of the tile
@@ -207,7 +232,7 @@ __global__ void __launch_bounds__(THREADS, 2)
             const int ti = (j - jt0) * ppt + i;
             const int page = ti < C::MAX_TAB ? tab[ti] : p.num_pages;
             for (int kb = 0; kb < HD / 64; ++kb)
-              tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128 + i * p.page_size * 128, (u & 1) ? &tmV : &tmK,
+              tma_load_4d(sKV + st * C::KV_BYTES + kb * BN * 128 + i * p.page_size * 128, isv ? &tmV : &tmK,
                           kv_full + st, kb * 64, kvh, 0, page);
           }
         }
@@ -217,7 +242,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       for (int w = (u > NS ? u - NS : 0); w < u; ++w)
         mbar_wait_drain(kv_full + w % NS, (w / NS) & 1, DRAIN_LIMIT_NS);
     }
-  } else if (warp == 2) {
+  } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       const uint64_t dQ = smem_desc_sw128(smem_u32(sQ), 16, 1024);
@@ -226,7 +251,8 @@ __global__ void __launch_bounds__(THREADS, 2)
       int u = 0, c = 0;
       if (a.test_stall && !mbar_wait(never, 0, abort_flag, p.status, a.wait_ns)) goto mma_drain;
       for (int j = jt0; j <= jt1; ++j, ++c) {
-        const int stK = u % NS, stV = (u + 1) % NS;
+        // keys at ring use u; values at u + 1, or (one cache) the same use
+        const int stK = u % NS, uV = a.kv_same ? u : u + 1, stV = uV % NS;
         if (!mbar_wait(kv_full + stK, (u / NS) & 1, abort_flag, p.status, a.wait_ns)) goto mma_drain;
         tc_fence_after();
         const uint64_t bk = dK + (uint64_t)((stK * C::KV_BYTES) >> 4);
@@ -236,9 +262,8 @@ __global__ void __launch_bounds__(THREADS, 2)
           umma_ss(tmem, dQ + off, bk + off, C::IDESC_QK, kk > 0);
         }
         umma_commit(s_full);
-        umma_commit(kv_empty + stK);
-        ++u;
-        if (!mbar_wait(kv_full + stV, (u / NS) & 1, abort_flag, p.status, a.wait_ns)) goto mma_drain;
+        if (!a.kv_same) umma_commit(kv_empty + stK);
+        if (!mbar_wait(kv_full + stV, (uV / NS) & 1, abort_flag, p.status, a.wait_ns)) goto mma_drain;
         if (!mbar_wait(p_full, c & 1, abort_flag, p.status, a.wait_ns)) goto mma_drain;
         tc_fence_after();
         const uint64_t bv = dV + (uint64_t)((stV * C::KV_BYTES) >> 4);
@@ -248,125 +273,132 @@ __global__ void __launch_bounds__(THREADS, 2)
                   (kk > 0 || c > 0) ? 1u : 0u);
         umma_commit(o_done);
         umma_commit(kv_empty + stV);
-        ++u;
+        u = uV + 1;
       }
     mma_drain:
       // every MMA issued above completes before tensor memory is released
       umma_commit(drain);
       mbar_wait_drain(drain, 0, DRAIN_LIMIT_NS);
     }
-  } else if (warp == 0) {
-    // ------------------------------------------------------------ softmax (lane = head)
+  } else {
+    // ------------------------------------------------ softmax (warp = lane quarter, lane = head)
+    const int k = warp;
+    const uint32_t lq = (uint32_t)(32 * k) << 16;  // this warp's TMEM lanes
     const int h = kvh * G + lane;
-    const float slope = (p.alibi.on && lane < G) ? p.alibi.slope[h] * LOG2E : 0.f;
+    const bool real = lane < G;
+    const float slope = (p.alibi.on && real) ? p.alibi.slope[h] * LOG2E : 0.f;
     const float sc = a.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     int c = 0;
     for (int j = jt0; j <= jt1; ++j, ++c) {
       if (!mbar_wait(s_full, c & 1, abort_flag, p.status, a.wait_ns)) goto done;
       tc_fence_after();
-      const int key0 = j * BN;
-      const bool need_mask = key0 < j0 || key0 + BN > j1;
-      float m_exp = m_ref, rs = 0.f;
-#pragma unroll 1
-      for (int h2 = 0; h2 < BN / 64; ++h2) {
-        float xa[32], xb[32];
-        tmem_ld32(tmem + h2 * 64, xa);
-        tmem_ld32(tmem + h2 * 64 + 32, xb);
-        tmem_wait_ld();
-        float hx = -INFINITY;
+      const int key0 = j * BN + 32 * k;  // this warp's 32 keys of the tile
+      const bool need_mask = key0 < j0 || key0 + 32 > j1;
+      float x[32];
+      tmem_ld32(tmem + lq + 32 * k, x);
+      tmem_wait_ld();
+      float hx = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const int ja = key0 + h2 * 64 + k, jb = ja + 32;
-          float va = p.alibi.on ? fmaf(xa[k], sc, -slope * fabsf((float)(qp - ja))) : xa[k] * sc;
-          float vb = p.alibi.on ? fmaf(xb[k], sc, -slope * fabsf((float)(qp - jb))) : xb[k] * sc;
-          if (need_mask) {
-            va = (ja >= j0 && ja < j1) ? va : -INFINITY;
-            vb = (jb >= j0 && jb < j1) ? vb : -INFINITY;
-          }
-          xa[k] = va;
-          xb[k] = vb;
-          hx = max3(hx, va, vb);
-        }
-        // same lazy reference as the prefill: move it only by more than 8 (log2 units)
-        const float m_cand = (hx > m_exp + 8.f) ? hx : m_exp;
-        if (__any_sync(0xffffffffu, m_cand != m_exp)) {
-          if (h2 > 0) {
-            const float f = (m_cand == m_exp) ? 1.f : ex2(m_exp - m_cand);
-            float pp[32];
-            tmem_wait_st();
-            tmem_ld32(tmem, pp);
-            tmem_wait_ld();
-            uint32_t pq[32];
+      for (int i = 0; i < 32; ++i) {
+        const int key = key0 + i;
+        float v = p.alibi.on ? fmaf(x[i], sc, -slope * fabsf((float)(qp - key))) : x[i] * sc;
+        if (need_mask) v = (key >= j0 && key < j1) ? v : -INFINITY;
+        x[i] = v;
+        hx = fmaxf(hx, v);
+      }
+      // the head's maximum over the whole tile, from the four quarters
+      float* rt = red + (c & 1) * 128;
+      rt[k * 32 + lane] = hx;
+      mbar_arrive(red_bar + (c & 1));
+      if (!mbar_wait(red_bar + (c & 1), (c >> 1) & 1, abort_flag, p.status, a.wait_ns)) goto done;
+      hx = fmaxf(fmaxf(rt[lane], rt[32 + lane]), fmaxf(rt[64 + lane], rt[96 + lane]));
+      // same lazy reference as the prefill: move it only by more than 8 (log2 units)
+      const float m_exp = (hx > m_ref + 8.f) ? hx : m_ref;
+      const float mu = (m_exp == -INFINITY) ? 0.f : m_exp;
+      uint32_t pk[16];
+      float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const float2 v = bf2_to_f2(__float_as_uint(pp[k]));
-              pq[k] = f2_to_bf2(v.x * f, v.y * f);
-            }
-            tmem_st32u(tmem, pq);
-            rs *= f;
-          }
-          m_exp = m_cand;
-        }
-        const float mu = (m_exp == -INFINITY) ? 0.f : m_exp;
-        uint32_t pk[32];
-        float rs0 = 0.f, rs1 = 0.f;
+      for (int i = 0; i < 16; i += 2) {
+        const float e0 = ex2(x[2 * i] - mu), e1 = ex2(x[2 * i + 1] - mu);
+        const float e2 = ex2(x[2 * i + 2] - mu), e3 = ex2(x[2 * i + 3] - mu);
+        rs0 += e0 + e1;
+        rs1 += e2 + e3;
+        pk[i] = f2_to_bf2(e0, e1);
+        pk[i + 1] = f2_to_bf2(e2, e3);
+      }
+      // P over the S columns of this warp's lanes: its keys' weights, zeros for the others
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float e0 = ex2(xa[2 * k] - mu), e1 = ex2(xa[2 * k + 1] - mu);
-          const float e2 = ex2(xb[2 * k] - mu), e3 = ex2(xb[2 * k + 1] - mu);
-          rs0 += e0 + e1;
-          rs1 += e2 + e3;
-          pk[k] = f2_to_bf2(e0, e1);
-          pk[16 + k] = f2_to_bf2(e2, e3);
-        }
-        rs += rs0 + rs1;
-        tmem_st32u(tmem + h2 * 32, pk);
+      for (int qq = 0; qq < 4; ++qq) {
+        uint32_t v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = qq == k ? pk[i] : 0u;
+        tmem_st16u(tmem + lq + 16 * qq, v);
       }
       const float alpha = (m_exp == m_ref) ? 1.f : ex2(m_ref - m_exp);
       m_ref = m_exp;
-      // rescale O (its previous PV finished before this tile's QK, which this tile waited for)
+      // rescale this quarter's part of O (the previous PV finished before this tile's QK,
+      // which this tile waited for)
       if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
         for (int q4 = 0; q4 < HD / 32; ++q4) {
           float o[32];
-          tmem_ld32(tmem + 128 + q4 * 32, o);
+          tmem_ld32(tmem + lq + 128 + q4 * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(tmem + 128 + q4 * 32, o);
+          tmem_st32(tmem + lq + 128 + q4 * 32, o);
         }
       }
-      l = l * alpha + rs;
+      l = l * alpha + (rs0 + rs1);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    // write this split's partial state
+    // add the four parts of O and of the row sum, and write this split's partial state
     if (!mbar_wait(o_done, (c - 1) & 1, abort_flag, p.status, a.wait_ns)) goto done;
     tc_fence_after();
-    const size_t pi = ((size_t)b * p.H + h) * a.nsplit + split;
+    {
+      // every copy into the ring was consumed by an MMA that o_done covers: the ring is idle
+      float* part = reinterpret_cast<float*>(sKV);  // [4][HD][32]
 #pragma unroll 1
-    for (int q4 = 0; q4 < HD / 32; ++q4) {
-      float o[32];
-      tmem_ld32(tmem + 128 + q4 * 32, o);
-      tmem_wait_ld();
-      if (lane < G) {
-        float4* dst = reinterpret_cast<float4*>(wsO + pi * HD + q4 * 32);
+      for (int q4 = 0; q4 < HD / 32; ++q4) {
+        float o[32];
+        tmem_ld32(tmem + lq + 128 + q4 * 32, o);
+        tmem_wait_ld();
 #pragma unroll
-        for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_float4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
+        for (int e = 0; e < 32; ++e) part[(k * HD + q4 * 32 + e) * 32 + lane] = o[e];
       }
-    }
-    if (lane < G) {
-      // the merge kernel works in natural-log units
-      wsM[pi] = m_ref == -INFINITY ? -INFINITY : m_ref * 0.6931471805599453f;
-      wsL[pi] = l;
+      lpart[k * 32 + lane] = l;
+      mbar_arrive(fin_bar);
+      if (!mbar_wait(fin_bar, 0, abort_flag, p.status, a.wait_ns)) goto done;
+      if (real) {
+        const size_t pi = ((size_t)b * p.H + h) * a.nsplit + split;
+        constexpr int DQ = HD / 4;  // features of O this warp adds up and writes
+        float4* dst = reinterpret_cast<float4*>(wsO + pi * HD + k * DQ);
+#pragma unroll 1
+        for (int v4 = 0; v4 < DQ / 4; ++v4) {
+          float r[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int d = k * DQ + v4 * 4 + e;
+            r[e] = part[d * 32 + lane] + part[(HD + d) * 32 + lane] + part[(2 * HD + d) * 32 + lane] +
+                   part[(3 * HD + d) * 32 + lane];
+          }
+          dst[v4] = make_float4(r[0], r[1], r[2], r[3]);
+        }
+        if (k == 0) {
+          // the merge kernel works in natural-log units
+          wsM[pi] = m_ref == -INFINITY ? -INFINITY : m_ref * 0.6931471805599453f;
+          wsL[pi] = lpart[lane] + lpart[32 + lane] + lpart[64 + lane] + lpart[96 + lane];
+        }
+      }
     }
   }
 done:
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
@@ -434,6 +466,7 @@ cudaError_t launch_hd(const DecodeParams& p, int chunk, int nsplit, void* ws, cu
   // records ATTN_ERR_TIMEOUT in the device status word, drains its own copies and exits.
   a.wait_ns = WAIT_LIMIT_NS;
   a.test_stall = 0;
+  a.kv_same = p.kcache == p.vcache;
   if (const char* e = std::getenv("ATTN_TEST_DECODE_STALL_NS")) {
     const long long ns = std::atoll(e);
     if (ns > 0) {

@@ -62,6 +62,10 @@ struct DecodeParams {
   // block_table[b * max_blocks + j / page_size]; Lmax = max_blocks * page_size.
   const int* block_table;
   int page_size, num_pages, max_blocks;
+  // Latent attention: the merge multiplies each head's merged output (hd numbers, the latent
+  // width) by W_out[h] ([H][hd][hd_out], bf16) and writes out [B,H,hd_out]. Otherwise nullptr.
+  const void* W_out;
+  int hd_out;
 };
 
 // Split-KV geometry: keys per split and number of splits for these sizes.
@@ -88,10 +92,10 @@ struct AppendParams {
 };
 cudaError_t launch_kv_append(const AppendParams& p, int dtype, cudaStream_t s);
 
-// Latent attention's per-head projections (bf16): fold: y[b,h,:] = W[h] x[b,h,:] (hd -> dc);
-// otherwise y[b,h,:] = x[b,h,:] W[h] (dc -> hd). W is [H][dc][hd].
-cudaError_t launch_head_proj(bool fold, const void* x, const void* W, void* y, int B, int H, int dc, int hd,
-                             cudaStream_t s);
+// Latent attention's key up-projection folded into the query (bf16): y[b,h,:] = W[h] x[b,h,:]
+// (hd -> dc), W [H][dc][hd].
+cudaError_t launch_latent_fold(const void* x, const void* W, void* y, int B, int H, int dc, int hd,
+                               cudaStream_t s);
 
 // C[M,N] = A[M,K] @ W[K,N], row-major, fp32 accumulation, output in the input dtype.
 cudaError_t launch_gemm_simt(const void* A, const void* W, void* C, int M, int N, int K, int dtype,

@@ -217,8 +217,10 @@ int attn_decode_paged(const void* q, const void* kpages, const void* vpages, con
  * between c and W_uk does not fold into the query); window and ALiBi as attn_decode.
  * q: [B,H,hd]; ccache: [B,Lmax,dc] (device); out: [B,H,hd]; lse: [B,H] or NULL.
  * workspace: attn_decode_latent_workspace_size(B,H,hd,dc,Lmax) bytes (device, caller-owned).
- * bf16 with dc in {64, 128} and H <= 32; anything else returns ATTN_ERR_UNSUPPORTED.
- * Four launches: the fold, the split pass, the merge, the value up-projection.
+ * bf16 with dc in {64, 128}, H <= 32 and hd a multiple of 8; anything else returns
+ * ATTN_ERR_UNSUPPORTED. Three launches: the fold, the split pass over the latent cache (one
+ * fetch of each latent tile serves as both key and value), and the merge of the splits with
+ * the value up-projection.
  */
 size_t attn_decode_latent_workspace_size(int B, int H, int hd, int dc, int Lmax);
 int attn_decode_latent(const void* q, const void* ccache, const void* W_uk, const void* W_uv,
