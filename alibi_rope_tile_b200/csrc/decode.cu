@@ -3,8 +3,8 @@
 // the keys and merged with the log-sum-exp rule of the FlashAttention section's online
 // softmax (m = max m_c, l = sum exp(m_c - m) l_c, O = sum exp(m_c - m) O_c / l).
 //
-// Pass 1 runs on the tensor cores for bf16 with hd 64 or 128 (decode_tc.cu). Otherwise it
-// is the CUDA-core kernel below, one CTA per (split, key/value head, sequence): the CTA
+// bf16 with hd 64 or 128 runs on the tensor cores (decode_tc.cu: its own work split and
+// merge). Otherwise pass 1 is the CUDA-core kernel below, one CTA per (split, key/value head, sequence): the CTA
 // reads its chunk of cache rows once, 16 bytes per lane per load, and serves every query
 // head of the group from those rows. Each warp owns a stream of keys; a key row of hd bf16 is covered by
 // hd/8 lanes, so one warp load instruction covers 32*8/hd rows. Per key the group's
@@ -14,6 +14,7 @@
 // chunk and written to the workspace as (O unnormalised, m, l).
 // Pass 2 merges the splits of each (sequence, head) and writes out and lse.
 #include "kernels.h"
+#include "merge.cuh"
 
 namespace attn {
 namespace {
@@ -219,42 +220,6 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeP
   }
 }
 
-// Merges the splits c < used of one (sequence, head) in one warp with the log-sum-exp rule:
-// the lanes read the splits' maxima and sums in parallel, then each lane adds up output
-// features lane, lane + 32, ... over the splits, several splits' loads in flight at once.
-// Returns the unnormalised sums in acc, the maximum in M and the denominator in den (all
-// lanes). A split that saw no key (maximum -inf) wrote no O and is given weight 0.
-template <int NI>
-__device__ __forceinline__ void warp_merge(const Partials& P, size_t pi0, int used, int hd, int lane,
-                                           float (&acc)[NI], float& M, float& den) {
-  M = -INFINITY;
-  for (int c = lane; c < used; c += 32) M = fmaxf(M, P.m[pi0 + c]);
-  M = warp_max(M);
-  den = 0.f;
-#pragma unroll
-  for (int i = 0; i < NI; ++i) acc[i] = 0.f;
-  if (M == -INFINITY) return;
-  for (int c0 = 0; c0 < used; c0 += 32) {
-    const int c = c0 + lane;
-    const float mc = c < used ? P.m[pi0 + c] : -INFINITY;
-    const float wc = mc == -INFINITY ? 0.f : expf(mc - M);
-    if (wc != 0.f) den += wc * P.l[pi0 + c];
-    const int n = min(32, used - c0);
-#pragma unroll 4
-    for (int k = 0; k < n; ++k) {
-      const float w = __shfl_sync(0xffffffffu, wc, k);
-      const float* Oc = P.O + (pi0 + c0 + k) * hd;
-#pragma unroll
-      for (int i = 0; i < NI; ++i) {
-        const int d = lane + 32 * i;
-        const float o = d < hd ? Oc[d] : 0.f;
-        acc[i] = fmaf(w, w != 0.f ? o : 0.f, acc[i]);
-      }
-    }
-  }
-  den = warp_sum(den);
-}
-
 // One warp per (sequence, head): four heads of one sequence per CTA.
 template <typename T>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p, int chunk, int nsplit, const void* ws) {
@@ -268,79 +233,13 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p,
   const int used = min(nsplit, (L + chunk - 1) / chunk);
   const size_t pi0 = ((size_t)b * p.H + h) * nsplit;
   float acc[ATTN_MAX_HD / 32], M, den;
-  warp_merge(P, pi0, used, hd, lane, acc, M, den);
+  warp_merge(P.m + pi0, P.l + pi0, P.O + pi0 * hd, 1, hd, used, hd, lane, acc, M, den);
   const float inv = den > 0.f ? 1.f / den : 0.f;
   T* out = static_cast<T*>(p.out) + ((size_t)b * p.H + h) * hd;
 #pragma unroll
   for (int i = 0; i < ATTN_MAX_HD / 32; ++i)
     if (lane + 32 * i < hd) Elem<T>::store(out + lane + 32 * i, acc[i] * inv);
   if (p.lse && lane == 0) p.lse[(size_t)b * p.H + h] = den > 0.f ? M + logf(den) : -INFINITY;
-}
-
-// Latent attention's merge: one CTA per (head, group of MERGE_SEQ sequences). Warp w merges
-// the splits of sequence b0 + w into its latent output (dc numbers, in shared memory): the
-// lanes take the splits' maxima and sums in parallel, then every lane adds up its dc / 32
-// features over the splits. The value up-projection W_out[h] ([dc][hd_out] bf16, staged once
-// per CTA by 16-byte copies) follows: thread e writes out[b, h, e] = sum_m olat[m] W_out[h][m][e]
-// for every sequence of the group.
-constexpr int MERGE_SEQ = 4;
-constexpr int MAX_DC = 128;  // latent widths: 64 or 128
-__global__ void __launch_bounds__(128)
-    decode_merge_up_kernel(const DecodeParams p, int chunk, int nsplit, const void* ws) {
-  extern __shared__ uint4 msh[];
-  const int h = blockIdx.x, b0 = blockIdx.y * MERGE_SEQ;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int dc = p.hd, ho = p.hd_out;
-  __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(msh);           // [dc][ho]
-  float* olat = reinterpret_cast<float*>(Ws + (size_t)dc * ho);         // [MERGE_SEQ][dc]
-  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.W_out) +
-                                                    (size_t)h * dc * ho);
-  const int nchunk = dc * ho / 8;
-  for (int c0 = threadIdx.x; c0 < nchunk; c0 += 8 * 128) {  // eight loads in flight per thread
-    uint4 u[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (c0 + r * 128 < nchunk) u[r] = __ldg(src + c0 + r * 128);
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (c0 + r * 128 < nchunk) msh[c0 + r * 128] = u[r];
-  }
-  const Partials P = partials(const_cast<void*>(ws), p.B, p.H, dc, nsplit);
-  const int b = b0 + warp;
-  if (b < p.B) {
-    int L = p.seqlens[b];
-    if (L < 0 || L > p.Lmax || p.qpos[b] < 0 || p.qpos[b] >= (1 << 24)) L = 0;
-    const int used = min(nsplit, (L + chunk - 1) / chunk);
-    float acc[MAX_DC / 32], M, den;
-    warp_merge(P, ((size_t)b * p.H + h) * nsplit, used, dc, lane, acc, M, den);
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-#pragma unroll
-    for (int i = 0; i < MAX_DC / 32; ++i)
-      if (lane + 32 * i < dc) olat[warp * dc + lane + 32 * i] = acc[i] * inv;
-    if (p.lse && lane == 0) p.lse[(size_t)b * p.H + h] = den > 0.f ? M + logf(den) : -INFINITY;
-  }
-  __syncthreads();
-  const int nb = min(MERGE_SEQ, p.B - b0);
-  for (int e = threadIdx.x; e < ho; e += blockDim.x) {
-    float acc[MERGE_SEQ];
-#pragma unroll
-    for (int sq = 0; sq < MERGE_SEQ; ++sq) acc[sq] = 0.f;
-#pragma unroll 2
-    for (int m = 0; m < dc; m += 4) {
-      const float w0 = __bfloat162float(Ws[(size_t)m * ho + e]), w1 = __bfloat162float(Ws[(size_t)(m + 1) * ho + e]);
-      const float w2 = __bfloat162float(Ws[(size_t)(m + 2) * ho + e]), w3 = __bfloat162float(Ws[(size_t)(m + 3) * ho + e]);
-#pragma unroll
-      for (int sq = 0; sq < MERGE_SEQ; ++sq) {
-        if (sq >= nb) break;
-        const float4 o = *reinterpret_cast<const float4*>(olat + sq * dc + m);
-        acc[sq] = fmaf(o.x, w0, fmaf(o.y, w1, fmaf(o.z, w2, fmaf(o.w, w3, acc[sq]))));
-      }
-    }
-#pragma unroll
-    for (int sq = 0; sq < MERGE_SEQ; ++sq)
-      if (sq < nb)
-        static_cast<__nv_bfloat16*>(p.out)[((size_t)(b0 + sq) * p.H + h) * ho + e] = __float2bfloat16_rn(acc[sq]);
-  }
 }
 
 template <typename T, int G>
@@ -359,21 +258,10 @@ cudaError_t launch_g(const DecodeParams& p, int chunk, int nsplit, void* ws, cud
 
 template <typename T>
 cudaError_t launch_t(const DecodeParams& p, void* ws, cudaStream_t s) {
+  if (decode_tc_supported(p, sizeof(T) == 2 ? 1 : 0)) return launch_decode_tc(p, ws, s);
+  if (p.W_out) return cudaErrorInvalidValue;  // the up-projection is on the tensor-core path only
   const int chunk = decode_chunk(p.B, p.KV, p.Lmax);
   const int nsplit = (p.Lmax + chunk - 1) / chunk;
-  if (decode_tc_supported(p, sizeof(T) == 2 ? 1 : 0)) {
-    cudaError_t e = launch_decode_tc(p, chunk, nsplit, ws, s);
-    if (e != cudaSuccess) return e;
-    if (p.W_out) {
-      const size_t smem = (size_t)p.hd * p.hd_out * 2 + (size_t)MERGE_SEQ * p.hd * sizeof(float);
-      e = cudaFuncSetAttribute(decode_merge_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      decode_merge_up_kernel<<<dim3(p.H, (p.B + MERGE_SEQ - 1) / MERGE_SEQ), 128, smem, s>>>(p, chunk, nsplit, ws);
-    } else {
-      decode_merge_kernel<T><<<dim3((p.H + 3) / 4, p.B), 128, 0, s>>>(p, chunk, nsplit, ws);
-    }
-    return cudaGetLastError();
-  }
   switch (p.H / p.KV) {
     case 1: return launch_g<T, 1>(p, chunk, nsplit, ws, s);
     case 2: return launch_g<T, 2>(p, chunk, nsplit, ws, s);
@@ -437,7 +325,9 @@ int decode_chunk(int B, int KV, int Lmax) {
 size_t decode_workspace_bytes(int B, int H, int KV, int hd, int Lmax) {
   const int chunk = decode_chunk(B, KV, Lmax);
   const size_t nsplit = ((size_t)Lmax + chunk - 1) / chunk;
-  return sizeof(float) * (size_t)B * H * nsplit * (hd + 2);
+  const size_t split = sizeof(float) * (size_t)B * H * nsplit * (hd + 2);
+  const size_t tc = (hd == 64 || hd == 128) ? decode_tc_workspace_bytes(B, H, KV, hd) : 0;
+  return split > tc ? split : tc;
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int dtype, void* ws, cudaStream_t s) {

@@ -68,14 +68,16 @@ struct DecodeParams {
   int hd_out;
 };
 
-// Split-KV geometry: keys per split and number of splits for these sizes.
+// Split-KV geometry of the CUDA-core path: keys per split for these sizes.
 int decode_chunk(int B, int KV, int Lmax);
+// Workspace of either decode path (the larger of the two).
 size_t decode_workspace_bytes(int B, int H, int KV, int hd, int Lmax);
 cudaError_t launch_decode(const DecodeParams& p, int dtype, void* workspace, cudaStream_t s);
-// Tensor-core split pass (bf16, hd in {64, 128}, H/KV <= 32); writes the same partials as
-// the CUDA-core split pass, which the log-sum-exp merge then combines.
+// Tensor-core decode (bf16, hd in {64, 128}, H/KV <= 32): plan, stream-K pass over all key
+// tiles, merge (with the up-projection when W_out is set). Its own partial layout.
 bool decode_tc_supported(const DecodeParams& p, int dtype);
-cudaError_t launch_decode_tc(const DecodeParams& p, int chunk, int nsplit, void* ws, cudaStream_t s);
+size_t decode_tc_workspace_bytes(int B, int H, int KV, int hd);
+cudaError_t launch_decode_tc(const DecodeParams& p, void* ws, cudaStream_t s);
 
 struct AppendParams {
   const void* k_new;

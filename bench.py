@@ -350,7 +350,7 @@ def build_families(art, only):
             hout.copy_(d["out"], non_blocking=True)
 
         return Family(key, dw.name + (f"_paged{PAGE_SIZE}" if paged else ""), "GB/s", "hbm",
-                      decode_bytes(hsl, dw), 2, "decode_tc_kernel<128>", run,
+                      decode_bytes(hsl, dw), DECODE_LAUNCHES, "decode_tc_kernel<128>", run,
                       e2e=(tnb(hq), tnb(hq), e2e_step))
 
     if want("decode_kv8"):
@@ -472,9 +472,10 @@ def block_families(art, want):
 
 
 # kernel launches of one run of the multi-launch families
-LATENT_LAUNCHES = 4       # the fold, the split pass, the merge, the value up-projection
-BLOCK_LAUNCHES = 5        # three projection GEMMs, the prefill, the output GEMM
-FUSED_LAUNCHES = 5        # RoPE table, RMSNorm, QKV GEMM (+ rotation, cache write), prefill, Wo GEMM (+ residual)
+DECODE_LAUNCHES = 3       # the plan (tiles per unit), the stream-K pass, the merge
+LATENT_LAUNCHES = 4       # the fold, the plan, the stream-K pass, the merge with the value up-projection
+BLOCK_LAUNCHES = 4        # RoPE table, QKV GEMM (+ key rotation), the prefill, the output GEMM
+FUSED_LAUNCHES = 6        # RoPE table, 1/rms, gamma folding, QKV GEMM (+ rotation, cache write), prefill, Wo GEMM (+ residual)
 
 
 def run_ours(args, rank, world):

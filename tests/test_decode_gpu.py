@@ -114,3 +114,23 @@ def test_append_position_error(art):
     with pytest.raises(art.AttnError):
         art.attn_sync_status()
     assert torch.all(kc[0, 3] == 1) and torch.all(kc[1] == 0)
+
+
+@pytest.mark.parametrize("nctas", ["1", "3"])
+@pytest.mark.parametrize("KV,hd,variant", [(1, 128, "rope"), (8, 128, "window"), (2, 64, "alibi"), (1, 64, "rope")])
+def test_few_ctas_long_pieces(art, monkeypatch, nctas, KV, hd, variant):
+    """The tensor-core decode gives every CTA an equal run of key tiles; a fixed small grid
+    (a test hook) makes each CTA run many tiles of a sequence and cross sequence boundaries
+    on small inputs, as the full-size workloads do."""
+    monkeypatch.setenv("ATTN_TEST_DECODE_CTAS", nctas)
+    B, H, Lmax = 3, 32 if KV <= 2 else 8, 900
+    lens = [900, 1, 517]
+    q, kc, vc, sl, qp = small_case(B, H, KV, hd, Lmax, 300 + KV + hd + int(nctas), torch.bfloat16, lens)
+    base = 10000.0 if variant == "rope" else 0.0
+    window = 300 if variant == "window" else 0
+    out, lse = run_decode(art, q, kc, vc, sl, qp, base, window=window, alibi=variant == "alibi")
+    assert art.attn_sync_status() == 0
+    slopes = A.alibi_slopes(H) if variant == "alibi" else None
+    ro, rl = A.decode(q, kc, vc, lens, lens, rope_base=base, window=window, slopes=slopes)
+    assert_close(out, ro, torch.bfloat16, f"decode {nctas} CTAs KV={KV} hd={hd} {variant}")
+    assert_lse_close(lse, rl, torch.bfloat16, "lse")
