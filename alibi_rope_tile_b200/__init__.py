@@ -43,6 +43,7 @@ SIGNATURES = {
     "attn_kv_write_paged": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "attn_decode_latent_workspace_size": (_S, [_I, _I, _I, _I, _I]),
     "attn_block_fused_workspace_size": (_S, [_I, _I, _I, _I, _I, _I]),
+    "attn_fold_rmsnorm_gamma": (_I, [_P, _P, _P, _I, _I, _P]),
     "attn_block_fused": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _L, _F, _I, _I,
                               _FP, _F, _I, _P, _S, _P]),
     "attn_decode_latent": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _FP, _I, _P, _S,
@@ -392,14 +393,16 @@ def attn_block_fused(x, gamma, Wqkv, Wo, out=None, kcache=None, vcache=None, wor
                      H: int, KV: int, pos0: int = 0, rope_base: float = 0.0, causal: bool = True,
                      window: int = 0, alibi_slopes=None, eps: float = 1e-6, stream=None):
     """x [B,T,d] -> x + attention(RMSNorm(x) Wqkv) Wo (Wqkv [d,(H+2KV)hd] = [q|k|v] heads);
-    with caches [B,Lmax,KV,hd], the turned keys and the values go to slots pos0 .. pos0+T-1."""
+    with caches [B,Lmax,KV,hd], the turned keys and the values go to slots pos0 .. pos0+T-1.
+    gamma=None: Wqkv already carries gamma (fold_rmsnorm_gamma), so it is not folded again."""
     B, T, d = x.shape
     if H < 1 or KV < 1 or Wqkv.dim() != 2 or Wqkv.shape[1] % (H + 2 * KV):
         raise ValueError(f"Wqkv must be [d, (H+2KV)*hd] with H={H}, KV={KV}, got {tuple(Wqkv.shape)}")
     hd = Wqkv.shape[1] // (H + 2 * KV)
     _shape(Wqkv, (d, (H + 2 * KV) * hd), "Wqkv")
     _shape(Wo, (H * hd, d), "Wo")
-    _shape(gamma, (d,), "gamma")
+    if gamma is not None:
+        _shape(gamma, (d,), "gamma")
     _shape(out, x.shape, "out")
     if (kcache is None) != (vcache is None):
         raise ValueError("give both kcache and vcache, or neither")
@@ -415,13 +418,27 @@ def attn_block_fused(x, gamma, Wqkv, Wo, out=None, kcache=None, vcache=None, wor
     need = int(lib().attn_block_fused_workspace_size(B, T, d, H, KV, hd))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
-    st = lib().attn_block_fused(_dev(x, "x"), _dev(gamma, "gamma", dt), _dev(Wqkv, "Wqkv", dt),
+    st = lib().attn_block_fused(_dev(x, "x"), None if gamma is None else _dev(gamma, "gamma", dt),
+                                _dev(Wqkv, "Wqkv", dt),
                                 _dev(Wo, "Wo", dt), _dev(out, "out", dt), _dev(kcache, "kcache", dt),
                                 _dev(vcache, "vcache", dt), Lmax, B, T, d, H, KV, hd, int(pos0),
                                 float(rope_base), int(bool(causal)), int(window),
                                 _slopes(alibi_slopes, H), float(eps), _dtype(x),
                                 _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                                 _stream(stream))
+    _check(st)
+    return out
+
+
+def fold_rmsnorm_gamma(gamma, W, out=None, stream=None):
+    """diag(gamma) W for W [d, N] (bf16): weights for attn_block_fused(..., gamma=None, ...)."""
+    d, N = W.shape
+    _shape(gamma, (d,), "gamma")
+    if out is None:
+        out = torch.empty_like(W)
+    _shape(out, W.shape, "out")
+    st = lib().attn_fold_rmsnorm_gamma(_dev(gamma, "gamma", W.dtype), _dev(W, "W", W.dtype),
+                                       _dev(out, "out", W.dtype), d, N, _stream(stream))
     _check(st)
     return out
 

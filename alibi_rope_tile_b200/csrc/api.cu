@@ -553,10 +553,9 @@ int attn_block_fused(const void* x, const void* gamma, const void* Wqkv, const v
                      float eps, int dtype, void* workspace, size_t ws_bytes, void* stream) {
   int st = check_common(H, KV, hd, dtype, rope_base);
   if (st) return st;
-  if (!x || !gamma || !Wqkv || !Wo || !out)
-    return fail(ATTN_ERR_ARG, "x, gamma, Wqkv, Wo and out must not be NULL");
+  if (!x || !Wqkv || !Wo || !out) return fail(ATTN_ERR_ARG, "x, Wqkv, Wo and out must not be NULL");
   if ((kcache == nullptr) != (vcache == nullptr)) return fail(ATTN_ERR_ARG, "give both caches or neither");
-  if (!aligned16(x) || !aligned16(gamma) || !aligned16(Wqkv) || !aligned16(Wo) || !aligned16(out) ||
+  if (!aligned16(x) || (gamma && !aligned16(gamma)) || !aligned16(Wqkv) || !aligned16(Wo) || !aligned16(out) ||
       (kcache && (!aligned16(kcache) || !aligned16(vcache))) || (workspace && !aligned16(workspace)))
     return fail(ATTN_ERR_ALIGN, "tensors and workspace must be 16-byte aligned");
   if (B < 1 || T < 1 || d < 8 || d % 8) return fail(ATTN_ERR_ARG, "B, T >= 1 and d a multiple of 8");
@@ -588,11 +587,12 @@ int attn_block_fused(const void* x, const void* gamma, const void* Wqkv, const v
   const RopeFreqs rope = make_rope(hd, rope_base);
   float2* cs = reinterpret_cast<float2*>(ws + L.cs);
   float* rinv = reinterpret_cast<float*>(ws + L.rinv);
-  // RMSNorm folded into the projection: 1 / rms per row, gamma into the weights' rows
+  // RMSNorm folded into the projection: 1 / rms per row, gamma into the weights' rows (here,
+  // or once by the caller through attn_fold_rmsnorm_gamma, then gamma is NULL)
   cudaError_t e = cudaSuccess;
   if (rope.on) e = launch_rope_table(cs, T, (int)pos0, rope, hd, s);
   if (e == cudaSuccess) e = launch_rms_inverse(x, rinv, M, d, eps, s);
-  if (e == cudaSuccess) e = launch_fold_gamma(Wqkv, gamma, ws + L.wg, d, Nqkv, s);
+  if (e == cudaSuccess && gamma) e = launch_fold_gamma(Wqkv, gamma, ws + L.wg, d, Nqkv, s);
   if (e != cudaSuccess) return cuda_fail(e, "fused block norm");
   // (x @ [Wq | Wk | Wv] with gamma folded) / rms, the keys turned, k and v also into the cache
   GemmEpilogue qkv;
@@ -606,7 +606,7 @@ int attn_block_fused(const void* x, const void* gamma, const void* Wqkv, const v
   qkv.cache[2] = vcache;
   qkv.Lmax = Lmax;
   qkv.pos0 = (int)pos0;
-  const char* wg = ws + L.wg;
+  const char* wg = gamma ? ws + L.wg : static_cast<const char*>(Wqkv);
   const void* Ws[3] = {wg, wg + (size_t)H * hd * 2, wg + (size_t)(H + KV) * hd * 2};
   void* Cs[3] = {ws + L.q, ws + L.k, ws + L.v};
   if ((e = launch_gemm_tc_multi(x, 3, Ws, Cs, Ns, M, d, status, s, &qkv, Nqkv)) != cudaSuccess)
@@ -622,6 +622,16 @@ int attn_block_fused(const void* x, const void* gamma, const void* Wqkv, const v
   res.residual = x;
   if ((e = launch_gemm_tc(ws + L.ctx, Wo, out, M, d, H * hd, status, s, &res)) != cudaSuccess)
     return cuda_fail(e, "fused block Wo GEMM");
+  return ok();
+}
+
+int attn_fold_rmsnorm_gamma(const void* gamma, const void* W, void* Wg, int d, int N, void* stream) {
+  if (!gamma || !W || !Wg) return fail(ATTN_ERR_ARG, "gamma, W and Wg must not be NULL");
+  if (!aligned16(gamma) || !aligned16(W) || !aligned16(Wg)) return fail(ATTN_ERR_ALIGN, "16-byte alignment");
+  if (d < 1 || N < 8 || N % 8 || (long long)d * N >= (1LL << 40))
+    return fail(ATTN_ERR_ARG, "d >= 1 and N a positive multiple of 8 (d=%d, N=%d)", d, N);
+  cudaError_t e = launch_fold_gamma(W, gamma, Wg, d, N, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fold_rmsnorm_gamma launch");
   return ok();
 }
 

@@ -61,7 +61,7 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
-  static constexpr int NBAR = 3 * NS + 18;
+  static constexpr int NBAR = 3 * NS + 19;
   // the MMA thread waits for tile j+1's keys before issuing tile j's PV: the ring must hold
   // more than two tiles so that those keys never wait for a stage only that PV frees
   static_assert(NS >= 5, "ring depth");
@@ -104,11 +104,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* q_rot = q_full + 2;     // the query tile is in tensor memory
   uint64_t* s_full = q_full + 3;    // [S buffer]: a QK completed
   uint64_t* p_full = q_full + 5;    // [S buffer]: P written (and O rescaled)
-  uint64_t* o_done = q_full + 7;    // a PV completed
-  uint64_t* red_bar = q_full + 8;   // [parity of the tile count][lane quarter]: the four warps of
+  // [S buffer]: the PV of a tile in that buffer (and every MMA before it) completed. One per
+  // buffer: with QK a tile ahead of PV, a single barrier can be two phases behind its waiter
+  // at the last tile, where a parity wait would pass early.
+  uint64_t* o_done = q_full + 7;
+  uint64_t* red_bar = q_full + 9;   // [parity of the tile count][lane quarter]: the four warps of
                                     // those rows wrote their maxima
-  uint64_t* lsum_bar = q_full + 16; // all warps' row sums written
-  uint64_t* drain = q_full + 17;    // the MMA thread's final commit
+  uint64_t* lsum_bar = q_full + 17; // all warps' row sums written
+  uint64_t* drain = q_full + 18;    // the MMA thread's final commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -157,6 +160,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int qq = 0; qq < 4; ++qq) mbar_init(red_bar + 4 * s + qq, 4);
     }
     mbar_init(o_done, 1);
+    mbar_init(o_done + 1, 1);
     mbar_init(lsum_bar, 16);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -299,7 +303,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(p_full + (i & 1), (i >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
         tc_fence_after();
         issue_pv(i & 1, uV % C::NS, i > 0);
-        umma_commit(o_done);
+        umma_commit(o_done + (i & 1));
         umma_commit(kv_empty + uV % C::NS);
       }
     mma_drain:
@@ -392,7 +396,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // O is rescaled before this tile's PV is issued, once the previous PV has completed
         // (the tile before the previous one completed before this tile's QK)
         if (c > 0 && kq * 32 < HD && __any_sync(0xffffffffu, alpha != 1.f)) {
-          if (!mbar_wait(o_done, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+          if (!mbar_wait(o_done + ((c - 1) & 1), ((c - 1) >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS))
+            goto done;
           tc_fence_after();
           const uint32_t tO = tmem + lane_off + C::COL_O + kq * 32;
           float o[32];
@@ -432,7 +437,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive(lsum_bar);
       if (!mbar_wait(lsum_bar, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
       const float lt = (lsum[r] + lsum[128 + r]) + (lsum[256 + r] + lsum[384 + r]);
-      if (!mbar_wait(o_done, (c - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
+      if (!mbar_wait(o_done + ((c - 1) & 1), ((c - 1) >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
       tc_fence_after();
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       if (kq * 32 < HD) {

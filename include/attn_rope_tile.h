@@ -260,6 +260,15 @@ int attn_block(const void* x, const void* Wq, const void* Wk, const void* Wv, co
                void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * attn_fold_rmsnorm_gamma -- Wg[k][n] = gamma[k] W[k][n] (bf16, rounded to nearest even): the
+ * weights of a projection that follows RMSNorm with gamma folded in, since
+ * (x / r * gamma) @ W = (x @ diag(gamma) W) / r ([XF5] "RMSNorm and Pre-LN residuals").
+ * gamma: [d]; W, Wg: [d, N] (device, bf16; Wg caller-owned, may not alias W). N a multiple of
+ * 8. One launch on stream; errors as the other entry points.
+ */
+int attn_fold_rmsnorm_gamma(const void* gamma, const void* W, void* Wg, int d, int N, void* stream);
+
+/*
  * attn_block_fused -- the attention sub-layer of a pre-norm decoder block ([XF5] "RMSNorm and
  * Pre-LN residuals": x + attn(norm(x))), fused around the attention core:
  *   xn = x / sqrt(mean(x^2) + eps) * gamma                      (RMSNorm per row)
@@ -267,11 +276,14 @@ int attn_block(const void* x, const void* Wq, const void* Wk, const void* Wv, co
  *                 v heads); q and k are turned at positions pos0 + t in the GEMM's epilogue,
  *                 which also writes k (turned) and v to kcache, vcache slots pos0 + t
  *   out = x + attention(q, k, v) @ Wo                           (the residual in the epilogue)
- * x, out: [B,T,d]; gamma: [d]; Wo: [H*hd, d]; all bf16 (device). kcache, vcache: [B,Lmax,KV,hd]
+ * x, out: [B,T,d]; gamma: [d]; Wo: [H*hd, d]; all bf16 (device). gamma may be NULL: Wqkv is then
+ * taken as already carrying gamma in its rows (diag(gamma) Wqkv, from attn_fold_rmsnorm_gamma),
+ * which saves re-folding static weights on every call. kcache, vcache: [B,Lmax,KV,hd]
  * or both NULL (no cache write); with caches, pos0 + T <= Lmax. Causal, window and ALiBi as
  * attn_prefill. workspace: attn_block_fused_workspace_size(...) bytes (device, caller-owned).
  * bf16, hd in {64, 128}, d and (H + 2 KV) hd multiples of 8; anything else returns
- * ATTN_ERR_UNSUPPORTED. Launches: RoPE table, RMSNorm, QKV GEMM, attention, Wo GEMM.
+ * ATTN_ERR_UNSUPPORTED. Launches: RoPE table, 1/rms per row, gamma folding (with gamma only),
+ * QKV GEMM (rows scaled by 1/rms in its epilogue), attention, Wo GEMM (+ residual).
  */
 size_t attn_block_fused_workspace_size(int B, int T, int d, int H, int KV, int hd);
 int attn_block_fused(const void* x, const void* gamma, const void* Wqkv, const void* Wo, void* out,

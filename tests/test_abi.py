@@ -190,13 +190,16 @@ def test_fused_block_argument_errors(lib):
         return lib.attn_block_fused(P, a["gamma"], P, P, P, a["kc"], a["vc"], a["Lmax"], 2, a["T"], a["d"],
                                     a["H"], a["KV"], a["hd"], a["pos0"], 10000.0, 1, 0, None, 1e-6,
                                     a["dtype"], P, 1 << 30, None)
-    assert fused(gamma=None) == -1
     assert fused(kc=P) == -1                          # one cache without the other
     assert fused(kc=P, vc=P, Lmax=20, pos0=8) == -1   # slots pos0..pos0+T-1 exceed the cache
     assert fused(d=500) == -1                         # d not a multiple of 8
     assert fused(hd=32, d=256) == -3                  # head size without a tensor-core path
     assert fused(dtype=0) == -3
     assert lib.attn_block_fused_workspace_size(2, 16, 512, 8, 2, 64) > 0
+    # gamma = NULL means "already folded into Wqkv"; the folding entry point checks its own
+    assert lib.attn_fold_rmsnorm_gamma(None, P, P, 512, 768, None) == -1
+    assert lib.attn_fold_rmsnorm_gamma(P, P, P, 512, 770, None) == -1   # N not a multiple of 8
+    assert lib.attn_fold_rmsnorm_gamma(P + 4, P, P, 512, 768, None) == -2  # misaligned
 
 
 def test_binding_requires_cuda_tensors(lib):

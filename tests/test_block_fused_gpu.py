@@ -101,3 +101,24 @@ def test_fused_block_rows_near_eps(art):
     assert_close(out, ref, BF, "fused block, rows near eps")
     wrong, _, _ = A.block_fused(x, gamma, Wqkv, Wo, H=H, KV=KV, rope_base=1e4, eps=0.0)
     assert np.abs(wrong - ref).max() > 0.05   # the case does tell the readings apart
+
+
+def test_prefolded_weights_give_the_same_output(art):
+    """gamma folded into Wqkv once by the caller (fold_rmsnorm_gamma, then gamma=None) gives the
+    same bits as folding on every call; the folded weights equal gamma[k] W[k][n] rounded to bf16."""
+    B, T, d, H, KV = 2, 256, 512, 8, 2
+    hd = d // H
+    g = torch.Generator().manual_seed(11)
+    x = (0.25 * torch.randn(B, T, d, generator=g)).to(BF).cuda()
+    gamma = (1.0 + 0.1 * torch.randn(d, generator=g)).to(BF).cuda()
+    Wqkv = (torch.randn(d, (H + 2 * KV) * hd, generator=g) / np.sqrt(d)).to(BF).cuda()
+    Wo = (torch.randn(H * hd, d, generator=g) / (2 * np.sqrt(H * hd))).to(BF).cuda()
+    Wg = art.fold_rmsnorm_gamma(gamma, Wqkv)
+    torch.cuda.synchronize()
+    expect = (gamma.double().cpu()[:, None] * Wqkv.double().cpu()).to(BF)
+    assert torch.equal(Wg.cpu(), expect)
+    a = art.attn_block_fused(x, gamma, Wqkv, Wo, H=H, KV=KV, rope_base=1e4)
+    b = art.attn_block_fused(x, None, Wg, Wo, H=H, KV=KV, rope_base=1e4)
+    torch.cuda.synchronize()
+    assert art.attn_sync_status() == 0
+    assert torch.equal(a, b)
