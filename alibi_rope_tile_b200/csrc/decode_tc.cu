@@ -4,11 +4,12 @@
 // FlashAttention equations (merge.cuh).
 //
 // Work split (stream-K). A unit is one (sequence, key/value head); its keys are the 128-key
-// tiles that hold slots [j0, seqlens) (j0 = qpos - window + 1 with a window, else 0). A plan
-// kernel counts every unit's tiles and writes their running sum; the decode kernel runs
-// two CTAs per SM and gives CTA i the tiles [i T / n, (i+1) T / n) of the concatenated units
-// (T tiles in all, n = min(grid, T) working CTAs), so every CTA streams the same amount of
-// cache whatever the mix of lengths. A CTA's range covers pieces of one or more units; each piece
+// tiles that hold slots [j0, seqlens) (j0 = qpos - window + 1 with a window, else 0). Every
+// unit's tile count and their running sum come first (each CTA computes them for up to
+// PLAN_MAX units; beyond that a plan kernel writes them once). The decode kernel runs two
+// CTAs per SM and gives CTA i the tiles [i T / n, (i+1) T / n) of the concatenated units (T
+// tiles in all, n = min(grid, T) working CTAs), so every CTA streams the same amount of cache
+// whatever the mix of lengths. A CTA's range covers pieces of one or more units; each piece
 // leaves a partial state in slot (unit + CTA index), which is unique because both numbers
 // only grow along the concatenation. The merge kernel finds the CTAs that cover a unit from
 // the same running sum and combines their partials.
@@ -51,6 +52,7 @@ constexpr int NS = 2;                 // ring stages (K, V alternate)
 constexpr int THREADS = 192;          // 4 softmax warps, the TMA warp, the MMA warp
 constexpr int TMA_WARP = 4, MMA_WARP = 5;
 constexpr int CTAS_PER_SM = 2;
+constexpr int PLAN_MAX = 1024;        // units up to which each CTA counts the tiles itself
 constexpr uint64_t WAIT_LIMIT_NS = 4000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;  // own copies/MMAs finish in microseconds
 constexpr float LOG2E = 1.4426950408889634f;
@@ -67,7 +69,9 @@ struct Cfg {
   // the softmax warps' exchange: running maxima red[2][4][32], row-sum parts lpart[4][32]
   static constexpr int OFF_RED = (OFF_MISC + 16 + 15) / 16 * 16;
   static constexpr int RED_BYTES = (2 * 4 * 32 + 4 * 32) * 4;
-  static constexpr int SMEM = OFF_RED + RED_BYTES + 1024;  // (two CTAs per SM stay within 200 KB)
+  // the running tile counts of up to PLAN_MAX units, when every CTA plans for itself (int)
+  static constexpr int OFF_PREF = OFF_RED + RED_BYTES;
+  static constexpr int SMEM = OFF_PREF + (PLAN_MAX + 1) * 4 + 1024;  // (two CTAs per SM: < 210 KB)
   // a piece's four O parts are added through the query tile's memory in rounds of RC columns:
   // [4 warps][RC][32 lanes] fp32
   static constexpr int RC = Q_BYTES / (4 * 32 * 4);
@@ -82,7 +86,9 @@ struct DecArgs {
   float* partO;              // [slots][G][hd]
   float* partM;              // [slots][G] (natural-log units)
   float* partL;              // [slots][G]
-  const long long* prefix;   // [U + 1]: tiles of the units before u; prefix[U] = all tiles
+  long long* prefix;         // [U + 1]: tiles of the units before u; prefix[U] = all tiles
+  int plan_in_cta;           // U <= PLAN_MAX: each CTA computes the counts (CTA 0 also writes
+                             // prefix for the merge); otherwise the plan kernel wrote prefix
   int U;                     // units: B * KV
   int nctas;                 // grid size
   unsigned long long wait_ns;  // bound of every wait (4 s unless a test lowers it)
@@ -191,9 +197,49 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
   const DecodeParams& p = a.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.H / p.KV;
+  int* spref = reinterpret_cast<int*>(smem + C::OFF_PREF);
+  if (a.plan_in_cta) {
+    // Tiles of every unit and their running sum, as the plan kernel computes them: thread tid
+    // counts a run of up to PER consecutive units, one block scan adds the runs up.
+    constexpr int PER = (PLAN_MAX + THREADS - 1) / THREADS;
+    __shared__ int wsum[THREADS / 32];
+    const int per = (a.U + THREADS - 1) / THREADS, u0 = tid * per;
+    int n[PER], run = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      n[i] = 0;
+      const int u = u0 + i;
+      if (i < per && u < a.U) {
+        const Unit x = unit_of(p, u);
+        n[i] = unit_tiles(x);
+        if (blockIdx.x == 0 && x.kvh == 0 && bad_sequence(p, p.seqlens[x.b], x.qp)) flag_error(p.status, DEV_BAD_ARG);
+      }
+      run += n[i];
+    }
+    int v = run;  // inclusive scan within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane == 31) wsum[warp] = v;
+    __syncthreads();
+    int before = v - run;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      if (i < per && u0 + i < a.U) spref[u0 + i] = before;
+      before += n[i];
+    }
+    if (tid == THREADS - 1) spref[a.U] = before;
+    __syncthreads();
+    if (blockIdx.x == 0)
+      for (int u = tid; u <= a.U; u += THREADS) a.prefix[u] = spref[u];  // for the merge
+  }
+  auto pref = [&](int u) -> long long { return a.plan_in_cta ? (long long)spref[u] : a.prefix[u]; };
   // With fewer tiles than CTAs only the first T CTAs work, so that every working CTA has at
   // least one tile (the merge relies on it).
-  const long long T = a.prefix[a.U];
+  const long long T = pref(a.U);
   const int nw = (int)(T < a.nctas ? T : a.nctas);
   if ((int)blockIdx.x >= nw) return;
   const long long t0 = T * blockIdx.x / nw, t1 = T * (blockIdx.x + 1) / nw;
@@ -204,7 +250,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
     while (hi - lo > 1) {
       const int step = (hi - lo + 31) / 32;
       const int idx = lo + lane * step;
-      const unsigned le = __ballot_sync(0xffffffffu, idx < hi && a.prefix[idx] <= t0);
+      const unsigned le = __ballot_sync(0xffffffffu, idx < hi && pref(idx) <= t0);
       const int nlo = lo + (31 - __clz(le)) * step;  // lane 0 always qualifies
       hi = min(hi, nlo + step);
       lo = nlo;
@@ -245,7 +291,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
   long long t = t0;                                                           \
   for (int pc = 0; t < t1; ++pc)
 #define PIECE_BOUNDS                                                          \
-  const long long ub = a.prefix[u], ue = a.prefix[u + 1];                     \
+  const long long ub = pref(u), ue = pref(u + 1);                             \
   const long long pe = ue < t1 ? ue : t1;                                     \
   const Unit x = unit_of(p, u);                                               \
   const int jb = x.jt0 + (int)(t - ub);                                       \
@@ -253,7 +299,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
 #define NEXT_PIECE                                                            \
   t = pe;                                                                     \
   ++u;                                                                        \
-  while (t < t1 && a.prefix[u + 1] <= t) ++u;
+  while (t < t1 && pref(u + 1) <= t) ++u;
 
   if (warp == TMA_WARP) {
     // ------------------------------------------------------------ TMA producer (whole warp;
@@ -720,7 +766,7 @@ cudaError_t launch_hd(const DecodeParams& p, void* ws, cudaStream_t s) {
   const int U = p.B * p.KV;
   const Layout lay = layout(ws, p.B, p.H, p.KV, HD);
 
-  decode_plan_kernel<<<1, 1024, 0, s>>>(p, lay.prefix, U);
+  if (U > PLAN_MAX) decode_plan_kernel<<<1, 1024, 0, s>>>(p, lay.prefix, U);
 
   DecArgs a;
   a.p = p;
@@ -729,6 +775,7 @@ cudaError_t launch_hd(const DecodeParams& p, void* ws, cudaStream_t s) {
   a.partM = lay.M;
   a.partL = lay.L;
   a.prefix = lay.prefix;
+  a.plan_in_cta = U <= PLAN_MAX;
   a.U = U;
   a.nctas = nctas;
   // Test hook (failure detection without a GPU fault): with ATTN_TEST_DECODE_STALL_NS set

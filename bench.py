@@ -474,8 +474,8 @@ def block_families(art, want):
 
 
 # kernel launches of one run of the multi-launch families
-DECODE_LAUNCHES = 3       # the plan (tiles per unit), the stream-K pass, the merge
-LATENT_LAUNCHES = 4       # the fold, the plan, the stream-K pass, the merge with the value up-projection
+DECODE_LAUNCHES = 2       # the stream-K pass (each CTA counts the tiles per unit), the merge
+LATENT_LAUNCHES = 3       # the fold, the stream-K pass, the merge with the value up-projection
 BLOCK_LAUNCHES = 4        # RoPE table, QKV GEMM (+ key rotation), the prefill, the output GEMM
 FUSED_LAUNCHES = 5        # RoPE table, 1/rms, QKV GEMM (+ 1/rms, rotation, cache write), prefill, Wo GEMM (+ residual)
 
