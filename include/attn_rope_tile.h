@@ -114,8 +114,8 @@ int attn_prefill_chunk(const void* q, const void* kcache, const void* vcache, co
 
 /*
  * attn_decode_workspace_size -- bytes of device scratch attn_decode needs for these
- * sizes (split-KV partial outputs and their softmax statistics). Returns 0 on invalid
- * sizes.
+ * sizes (partial outputs of runs of key tiles, their softmax statistics, the tile counts of
+ * the (sequence, key/value head) units). Returns 0 on invalid sizes.
  */
 size_t attn_decode_workspace_size(int B, int H, int KV, int hd, int Lmax);
 
@@ -133,8 +133,12 @@ size_t attn_decode_workspace_size(int B, int H, int KV, int hd, int Lmax);
  * bytes, owned by the caller; its contents on entry do not matter.
  * seqlens[b] > Lmax or qpos[b] < 0 is recorded as ATTN_ERR_DEVICE_ARG (read it with
  * attn_sync_status) and that sequence's output is zeroed.
- * Two kernels run on stream: split-KV partials (each CTA reads its cache rows once with
- * 16-byte loads for all H/KV query heads of a key/value head), then a log-sum-exp merge.
+ * Two kernels run on stream (bf16, hd 64 or 128, H/KV <= 32): the tensor-core pass, whose
+ * CTAs (two per SM) take equal runs of all sequences' 128-key tiles and serve every query
+ * head of a key/value head from each tile they read once, then a log-sum-exp merge of the
+ * runs; with more than 1024 (sequence, key/value head) units a one-CTA kernel counts their
+ * tiles first. Other types and head sizes: a CUDA-core split pass (16-byte loads, fixed
+ * splits of 2048 keys) and the same merge rule.
  */
 int attn_decode(const void* q, const void* kcache, const void* vcache, const int* seqlens,
                 const int* qpos, void* out, float* lse, int B, int H, int KV, int hd, int Lmax,
@@ -150,7 +154,7 @@ int attn_decode(const void* q, const void* kcache, const void* vcache, const int
  * plugin inside another framework's memory pool), or a latency-critical step where an
  * allocation, which may synchronise the device, is not allowed.
  *
- * Arguments and results are those of attn_decode without workspace/ws_bytes. The split
+ * Arguments and results are those of attn_decode without workspace/ws_bytes. The
  * partials live in a fixed scratch array of ATTN_DECODE_NOALLOC_MAX_SCRATCH bytes that is
  * part of the library's device image: every GPU that loads the library holds it until the
  * process exits. Sizes whose attn_decode_workspace_size() exceeds that maximum are
@@ -198,8 +202,8 @@ int attn_kv_write(const void* k_new, const void* v_new, void* kcache, void* vcac
  * the sequence does not reach are not read. A table entry outside [0, num_pages) is
  * recorded as ATTN_ERR_DEVICE_ARG and its page reads as zeros. Everything else (q rotated
  * at qpos[b], window, ALiBi, outputs, workspace = attn_decode_workspace_size(B, H, KV, hd,
- * max_blocks * page_size)) is as attn_decode. Runs the tensor-core split pass: bf16, hd 64
- * or 128, H/KV <= 32; anything else returns ATTN_ERR_UNSUPPORTED.
+ * max_blocks * page_size)) is as attn_decode. Runs the tensor-core pass: bf16, hd 64 or 128,
+ * H/KV <= 32; anything else returns ATTN_ERR_UNSUPPORTED.
  */
 int attn_decode_paged(const void* q, const void* kpages, const void* vpages, const int* block_table,
                       const int* seqlens, const int* qpos, void* out, float* lse, int B, int H, int KV,
@@ -218,8 +222,8 @@ int attn_decode_paged(const void* q, const void* kpages, const void* vpages, con
  * q: [B,H,hd]; ccache: [B,Lmax,dc] (device); out: [B,H,hd]; lse: [B,H] or NULL.
  * workspace: attn_decode_latent_workspace_size(B,H,hd,dc,Lmax) bytes (device, caller-owned).
  * bf16 with dc in {64, 128}, H <= 32 and hd a multiple of 8; anything else returns
- * ATTN_ERR_UNSUPPORTED. Three launches: the fold, the split pass over the latent cache (one
- * fetch of each latent tile serves as both key and value), and the merge of the splits with
+ * ATTN_ERR_UNSUPPORTED. Three launches: the fold, the tensor-core pass over the latent cache
+ * (one fetch of each latent tile serves as both key and value), and the merge of its runs with
  * the value up-projection.
  */
 size_t attn_decode_latent_workspace_size(int B, int H, int hd, int dc, int Lmax);
