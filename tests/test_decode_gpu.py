@@ -134,3 +134,18 @@ def test_few_ctas_long_pieces(art, monkeypatch, nctas, KV, hd, variant):
     ro, rl = A.decode(q, kc, vc, lens, lens, rope_base=base, window=window, slopes=slopes)
     assert_close(out, ro, torch.bfloat16, f"decode {nctas} CTAs KV={KV} hd={hd} {variant}")
     assert_lse_close(lse, rl, torch.bfloat16, "lse")
+
+
+def test_many_units_use_the_plan_kernel(art):
+    """More than 1024 (sequence, key/value head) units: a one-CTA kernel counts the tiles
+    before the decode instead of every CTA counting them itself."""
+    B, H, KV, hd, Lmax = 130, 8, 8, 64, 300
+    rng = np.random.default_rng(5)
+    lens = [int(x) for x in rng.integers(0, Lmax + 1, size=B)]
+    lens[3] = 0
+    q, kc, vc, sl, qp = small_case(B, H, KV, hd, Lmax, 77, torch.bfloat16, lens)
+    out, lse = run_decode(art, q, kc, vc, sl, qp, 10000.0)
+    assert art.attn_sync_status() == 0
+    ro, rl = A.decode(q, kc, vc, lens, lens, rope_base=10000.0)
+    assert_close(out, ro, torch.bfloat16, "decode, 1040 units")
+    assert_lse_close(lse, rl, torch.bfloat16, "lse")

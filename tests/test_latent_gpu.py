@@ -46,3 +46,26 @@ def test_latent_decode_matches_unfolded_oracle(art, dc, flags):
     assert_close(out, ref, BF, f"latent dc{dc} {flags}")
     assert_lse_close(lse, ref_lse, BF, "latent lse")
     assert torch.count_nonzero(out[4]) == 0  # empty cache
+
+
+def test_latent_decode_few_ctas(art, monkeypatch):
+    """A fixed grid of 3 CTAs (a test hook): each CTA's run of latent tiles crosses sequences."""
+    monkeypatch.setenv("ATTN_TEST_DECODE_CTAS", "3")
+    B, H, hd, dc, Lmax = 4, 32, 128, 128, 1500
+    g = torch.Generator().manual_seed(41)
+    q = workloads.normal((B, H, hd), 0, BF, g)
+    c = workloads.normal((B, Lmax, dc), 0, BF, g)
+    W_uk = (torch.randn(H, dc, hd, generator=g) / np.sqrt(dc)).to(BF)
+    W_uv = (torch.randn(H, dc, hd, generator=g) / np.sqrt(dc)).to(BF)
+    lens = [1500, 3, 0, 901]
+    sl = torch.tensor(lens, dtype=torch.int32)
+    for b, L in enumerate(lens):
+        c[b, L:] = 0
+    lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
+    out = art.attn_decode_latent(q.cuda(), c.cuda(), W_uk.cuda(), W_uv.cuda(), sl.cuda(), sl.cuda(), lse=lse)
+    torch.cuda.synchronize()
+    assert art.attn_sync_status() == 0
+    ref, ref_lse = A.latent_decode(q, c, W_uk, W_uv, sl.numpy(), sl.numpy())
+    assert_close(out, ref, BF, "latent, 3 CTAs")
+    assert_lse_close(lse, ref_lse, BF, "latent lse")
+    assert torch.count_nonzero(out[2]) == 0  # empty cache

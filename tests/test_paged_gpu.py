@@ -101,3 +101,25 @@ def test_paged_writes_then_decode_equal_the_contiguous_cache(art):
     assert torch.equal(paged, flat), "same rows, same tiles: the two layouts decode identically"
     ref, _ = A.decode(q.cpu(), kc.cpu(), vc.cpu(), sl.cpu().numpy(), sl.cpu().numpy(), rope_base=base)
     assert_close(paged, ref, BF, "paged decode after paged writes")
+
+
+@pytest.mark.parametrize("page_size,KV,flags", [(16, 2, dict(alibi=True)), (128, 1, dict(window=300))])
+def test_paged_decode_few_ctas(art, monkeypatch, page_size, KV, flags):
+    """A fixed grid of 2 CTAs (a test hook): each CTA walks many paged tiles across sequences."""
+    monkeypatch.setenv("ATTN_TEST_DECODE_CTAS", "2")
+    B, H, hd, max_blocks = 5, 32, 128, 4096 // page_size
+    lens = [1, 130, 2047, 4096, 777]
+    q, kp, vp, table, sl = paged_case(B, H, KV, hd, page_size, max_blocks, lens, seed=7 + page_size + KV)
+    base = 0.0 if flags.get("alibi") else 10000.0
+    window = flags.get("window", 0)
+    slopes = art.alibi_slopes(H) if flags.get("alibi") else None
+    lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
+    out = art.attn_decode_paged(q.cuda(), kp.cuda(), vp.cuda(), table.cuda(), sl.cuda(), sl.cuda(), lse=lse,
+                                rope_base=base, window=window, alibi_slopes=slopes)
+    torch.cuda.synchronize()
+    assert art.attn_sync_status() == 0
+    ref, ref_lse = A.decode_paged(q, kp, vp, table.numpy(), sl.numpy(), sl.numpy(), page_size=page_size,
+                                  rope_base=base, window=window,
+                                  slopes=None if slopes is None else np.array(slopes))
+    assert_close(out, ref, BF, f"paged decode, 2 CTAs, ps{page_size} KV{KV} {flags}")
+    assert_lse_close(lse, ref_lse, BF, "paged decode lse")
