@@ -349,14 +349,14 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
               for (int kb = 0; kb < HD / 64; ++kb)
                 tma_load_4d(dst + kb * BN * 128, m, kv_full + st, kb * 64, x.kvh, j * BN, x.b);
           } else {
+            // one box per page, each lane issuing its own page's boxes (the expected bytes
+            // were posted by lane 0 first)
+            __syncwarp();
             const int ppt = BN / p.page_size;
-            for (int i = 0; i < ppt; ++i) {
-              const int pg = __shfl_sync(0xffffffffu, page, i);
-              if (lane == 0)
-                for (int kb = 0; kb < HD / 64; ++kb)
-                  tma_load_4d(dst + kb * BN * 128 + i * p.page_size * 128, m, kv_full + st, kb * 64, x.kvh, 0,
-                              pg);
-            }
+            if (lane < ppt)
+              for (int kb = 0; kb < HD / 64; ++kb)
+                tma_load_4d(dst + kb * BN * 128 + lane * p.page_size * 128, m, kv_full + st, kb * 64, x.kvh, 0,
+                            page);
           }
           ++use;
         }
