@@ -469,14 +469,26 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
         float xs[32];
         tmem_ld32(tmem + lq + 32 * k4, xs);
         tmem_wait_ld();
+        // plain tiles (no bias, no mask) keep the raw scores: the maximum is taken first and
+        // scaled once (a positive scale keeps the order), the scale goes into the ex2 FMA
+        const bool plain = !p.alibi.on && !need_mask;
         float hx = -INFINITY;
+        if (plain) {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = key0 + i;
-          float v = p.alibi.on ? fmaf(xs[i], sc, -slope * fabsf((float)(x.qp - key))) : xs[i] * sc;
-          if (need_mask) v = (key >= x.j0 && key < x.j1) ? v : -INFINITY;
-          xs[i] = v;
-          hx = fmaxf(hx, v);
+          for (int i = 0; i < 32; i += 4)
+#pragma unroll
+            for (int t = 0; t < 4; ++t) m4[t] = fmaxf(m4[t], xs[i + t]);
+          hx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int key = key0 + i;
+            float v = p.alibi.on ? fmaf(xs[i], sc, -slope * fabsf((float)(x.qp - key))) : xs[i] * sc;
+            if (need_mask) v = (key >= x.j0 && key < x.j1) ? v : -INFINITY;
+            xs[i] = v;
+            hx = fmaxf(hx, v);
+          }
         }
         // the head's maximum over the whole tile, from the four quarters
         float* rt = red + (c & 1) * 128;
@@ -488,16 +500,21 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
         const float m_exp = (hx > m_ref + 8.f) ? hx : m_ref;
         const float mu = (m_exp == -INFINITY) ? 0.f : m_exp;
         uint32_t pk[16];
-        float rs0 = 0.f, rs1 = 0.f;
+        // ex2 arguments by packed FMA: x * s - mu with s = the scale (plain tiles) or 1
+        const f2x SC = plain ? pk2(sc, sc) : pk2(1.f, 1.f), NM = pk2(-mu, -mu);
+        f2x RS = pk2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          const float e0 = ex2(xs[2 * i] - mu), e1 = ex2(xs[2 * i + 1] - mu);
-          const float e2 = ex2(xs[2 * i + 2] - mu), e3 = ex2(xs[2 * i + 3] - mu);
-          rs0 += e0 + e1;
-          rs1 += e2 + e3;
+          float a0, a1, b0, b1;
+          up2(fma2(pk2(xs[2 * i], xs[2 * i + 1]), SC, NM), a0, a1);
+          up2(fma2(pk2(xs[2 * i + 2], xs[2 * i + 3]), SC, NM), b0, b1);
+          const float e0 = ex2(a0), e1 = ex2(a1), e2 = ex2(b0), e3 = ex2(b1);
+          RS = add2(RS, add2(pk2(e0, e1), pk2(e2, e3)));
           pk[i] = f2_to_bf2(e0, e1);
           pk[i + 1] = f2_to_bf2(e2, e3);
         }
+        float rs0, rs1;
+        up2(RS, rs0, rs1);
         // P over the S columns of this warp's lanes: its keys' weights, zeros for the others
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
