@@ -641,10 +641,11 @@ __global__ void __launch_bounds__(128) sk_merge_kernel(const DecodeParams p, con
 // Latent attention's merge (one key/value unit per sequence): one CTA per (head, group of
 // MERGE_SEQ sequences). Warp w merges the partials of sequence b0 + w into its latent output
 // (dc = hd numbers, in shared memory); the value up-projection W_out[h] ([dc][hd_out] bf16,
-// staged once per CTA by 16-byte copies) follows: thread e writes
-// out[b, h, e] = sum_m olat[m] W_out[h][m][e] for every sequence of the group.
-constexpr int MERGE_SEQ = 4;
-__global__ void __launch_bounds__(128) sk_merge_up_kernel(const DecodeParams p, const float* partO,
+// staged once per CTA by 16-byte copies) follows: thread (e, half) writes
+// out[b, h, e] = sum_m olat[m] W_out[h][m][e] for the sequences of its half of the group.
+constexpr int MERGE_SEQ = 8;
+constexpr int MERGE_THREADS = 32 * MERGE_SEQ;
+__global__ void __launch_bounds__(MERGE_THREADS) sk_merge_up_kernel(const DecodeParams p, const float* partO,
                                                           const float* partM, const float* partL,
                                                           const long long* prefix, int nctas) {
   extern __shared__ uint4 msh[];
@@ -655,14 +656,14 @@ __global__ void __launch_bounds__(128) sk_merge_up_kernel(const DecodeParams p, 
   float* olat = reinterpret_cast<float*>(Ws + (size_t)dc * ho);  // [MERGE_SEQ][dc]
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.W_out) + (size_t)h * dc * ho);
   const int nchunk = dc * ho / 8;
-  for (int c0 = threadIdx.x; c0 < nchunk; c0 += 8 * 128) {  // eight loads in flight per thread
+  for (int c0 = threadIdx.x; c0 < nchunk; c0 += 8 * MERGE_THREADS) {  // eight loads in flight per thread
     uint4 v[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r)
-      if (c0 + r * 128 < nchunk) v[r] = __ldg(src + c0 + r * 128);
+      if (c0 + r * MERGE_THREADS < nchunk) v[r] = __ldg(src + c0 + r * MERGE_THREADS);
 #pragma unroll
     for (int r = 0; r < 8; ++r)
-      if (c0 + r * 128 < nchunk) msh[c0 + r * 128] = v[r];
+      if (c0 + r * MERGE_THREADS < nchunk) msh[c0 + r * MERGE_THREADS] = v[r];
   }
   const int b = b0 + warp;
   if (b < p.B) {
@@ -678,25 +679,27 @@ __global__ void __launch_bounds__(128) sk_merge_up_kernel(const DecodeParams p, 
   }
   __syncthreads();
   const int nb = min(MERGE_SEQ, p.B - b0);
-  for (int e = threadIdx.x; e < ho; e += blockDim.x) {
-    float acc[MERGE_SEQ];
+  constexpr int HALF = MERGE_SEQ / 2;
+  for (int idx = threadIdx.x; idx < 2 * ho; idx += blockDim.x) {
+    const int e = idx % ho, s0 = (idx / ho) * HALF;  // output feature, first sequence of the half
+    float acc[HALF];
 #pragma unroll
-    for (int sq = 0; sq < MERGE_SEQ; ++sq) acc[sq] = 0.f;
+    for (int sq = 0; sq < HALF; ++sq) acc[sq] = 0.f;
 #pragma unroll 2
     for (int m = 0; m < dc; m += 4) {
       const float w0 = __bfloat162float(Ws[(size_t)m * ho + e]), w1 = __bfloat162float(Ws[(size_t)(m + 1) * ho + e]);
       const float w2 = __bfloat162float(Ws[(size_t)(m + 2) * ho + e]), w3 = __bfloat162float(Ws[(size_t)(m + 3) * ho + e]);
 #pragma unroll
-      for (int sq = 0; sq < MERGE_SEQ; ++sq) {
-        if (sq >= nb) break;
-        const float4 o = *reinterpret_cast<const float4*>(olat + sq * dc + m);
+      for (int sq = 0; sq < HALF; ++sq) {
+        if (s0 + sq >= nb) break;
+        const float4 o = *reinterpret_cast<const float4*>(olat + (s0 + sq) * dc + m);
         acc[sq] = fmaf(o.x, w0, fmaf(o.y, w1, fmaf(o.z, w2, fmaf(o.w, w3, acc[sq]))));
       }
     }
 #pragma unroll
-    for (int sq = 0; sq < MERGE_SEQ; ++sq)
-      if (sq < nb)
-        static_cast<__nv_bfloat16*>(p.out)[((size_t)(b0 + sq) * p.H + h) * ho + e] = __float2bfloat16_rn(acc[sq]);
+    for (int sq = 0; sq < HALF; ++sq)
+      if (s0 + sq < nb)
+        static_cast<__nv_bfloat16*>(p.out)[((size_t)(b0 + s0 + sq) * p.H + h) * ho + e] = __float2bfloat16_rn(acc[sq]);
   }
 }
 
@@ -817,7 +820,7 @@ cudaError_t launch_hd(const DecodeParams& p, void* ws, cudaStream_t s) {
     const size_t smem = (size_t)p.hd * p.hd_out * 2 + (size_t)MERGE_SEQ * p.hd * sizeof(float);
     e = cudaFuncSetAttribute(sk_merge_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    sk_merge_up_kernel<<<dim3(p.H, (p.B + MERGE_SEQ - 1) / MERGE_SEQ), 128, smem, s>>>(p, lay.O, lay.M, lay.L,
+    sk_merge_up_kernel<<<dim3(p.H, (p.B + MERGE_SEQ - 1) / MERGE_SEQ), MERGE_THREADS, smem, s>>>(p, lay.O, lay.M, lay.L,
                                                                                        lay.prefix, nctas);
   } else {
     sk_merge_kernel<<<dim3((p.H + 3) / 4, p.B), 128, 0, s>>>(p, lay.O, lay.M, lay.L, lay.prefix, nctas);
