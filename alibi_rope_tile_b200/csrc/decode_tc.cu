@@ -197,6 +197,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
   const DecodeParams& p = a.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.H / p.KV;
+  launch_dependents();  // the merge may start its independent set-up
   int* spref = reinterpret_cast<int*>(smem + C::OFF_PREF);
   if (a.plan_in_cta) {
     // Tiles of every unit and their running sum, as the plan kernel computes them: thread tid
@@ -419,6 +420,8 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
     // ---------------------------------- softmax and query set-up (warp = lane quarter, lane = head)
     const int k4 = warp;
     const uint32_t lq = (uint32_t)(32 * k4) << 16;  // this warp's TMEM lanes
+    // q may be the previous kernel's output (the latent fold, launched ahead of this one)
+    grid_dependency_wait();
     const float sc = a.scale_log2;
     float* part = reinterpret_cast<float*>(sQ);  // [4][RC][32] while no query tile is needed
     int c = 0, fc = 0;
@@ -624,6 +627,7 @@ __global__ void __launch_bounds__(128) sk_merge_kernel(const DecodeParams p, con
                                                        const float* partL, const long long* prefix, int nctas) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x * 4 + warp, b = blockIdx.y;
+  grid_dependency_wait();  // the decode's partials and counts
   if (h >= p.H) return;
   const int G = p.H / p.KV, hd = p.hd;
   const UnitParts up = unit_parts(prefix, p.B * p.KV, nctas, b * p.KV + h / G, G, h % G);
@@ -665,6 +669,7 @@ __global__ void __launch_bounds__(MERGE_THREADS) sk_merge_up_kernel(const Decode
     for (int r = 0; r < 8; ++r)
       if (c0 + r * MERGE_THREADS < nchunk) msh[c0 + r * MERGE_THREADS] = v[r];
   }
+  grid_dependency_wait();  // the decode's partials and counts (the weights did not depend on it)
   const int b = b0 + warp;
   if (b < p.B) {
     const UnitParts up = unit_parts(prefix, p.B, nctas, b, G, h);
@@ -814,16 +819,41 @@ cudaError_t launch_hd(const DecodeParams& p, void* ws, cudaStream_t s) {
   }
   e = cudaFuncSetAttribute(decode_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<HD>::SMEM);
   if (e != cudaSuccess) return e;
-  decode_tc_kernel<HD><<<nctas, THREADS, Cfg<HD>::SMEM, s>>>(mk, mv, a);
+  // Programmatic dependent launches: the latent decode follows its fold, which writes only q'
+  // (this kernel waits for it before reading q); the merges follow this kernel and wait for it
+  // before reading the partials. The plain decode is launched normally: the kernel before it
+  // may be writing the cache.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nctas);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = Cfg<HD>::SMEM;
+  cfg.stream = s;
+  cfg.attrs = pdl;
+  cfg.numAttrs = (p.W_out && U <= PLAN_MAX) ? 1 : 0;  // (a plan kernel writes what every role reads)
+  if ((e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<HD>, mk, mv, a)) != cudaSuccess) return e;
 
   if (p.W_out) {
     const size_t smem = (size_t)p.hd * p.hd_out * 2 + (size_t)MERGE_SEQ * p.hd * sizeof(float);
     e = cudaFuncSetAttribute(sk_merge_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    sk_merge_up_kernel<<<dim3(p.H, (p.B + MERGE_SEQ - 1) / MERGE_SEQ), MERGE_THREADS, smem, s>>>(p, lay.O, lay.M, lay.L,
-                                                                                       lay.prefix, nctas);
+    cfg.gridDim = dim3(p.H, (p.B + MERGE_SEQ - 1) / MERGE_SEQ);
+    cfg.blockDim = dim3(MERGE_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, sk_merge_up_kernel, p, (const float*)lay.O, (const float*)lay.M, (const float*)lay.L,
+                           (const long long*)lay.prefix, nctas);
+    if (e != cudaSuccess) return e;
   } else {
-    sk_merge_kernel<<<dim3((p.H + 3) / 4, p.B), 128, 0, s>>>(p, lay.O, lay.M, lay.L, lay.prefix, nctas);
+    cfg.gridDim = dim3((p.H + 3) / 4, p.B);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, sk_merge_kernel, p, (const float*)lay.O, (const float*)lay.M, (const float*)lay.L,
+                           (const long long*)lay.prefix, nctas);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

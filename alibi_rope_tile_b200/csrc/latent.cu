@@ -19,6 +19,8 @@ __global__ void __launch_bounds__(THREADS)
     latent_fold_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ W,
                        __nv_bfloat16* __restrict__ y, int B, int H, int dc, int hd) {
   extern __shared__ float sh[];
+  // the decode that follows may start its independent set-up now (it waits for q')
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int h = blockIdx.x, b0 = blockIdx.y * SEQ;
   const int nb = min(SEQ, B - b0);
   const int ld = dc + 1;

@@ -119,6 +119,13 @@ __device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, v
   return mbar_wait_slow(bar, parity, abort, status, limit_ns);
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may
+// start while the previous kernel in the stream still runs. launch_dependents lets this
+// kernel's own dependents start early; grid_dependency_wait blocks the calling thread until
+// the previous kernel has completed and its writes are visible (a no-op without a dependency).
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
