@@ -29,6 +29,9 @@ _FP = ctypes.POINTER(ctypes.c_float)
 # (name, restype, argtypes) of every exported entry point
 SIGNATURES = {
     "attn_prefill": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _F, _I, _I, _FP, _I, _P]),
+    "attn_prefill_workspace_size": (_S, [_I, _I, _I, _I, _F, _I]),
+    "attn_prefill_ws": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _F, _I, _I, _FP, _I, _P, _S,
+                             _P]),
     "attn_decode_workspace_size": (_S, [_I, _I, _I, _I, _I]),
     "attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _FP, _I, _P, _S,
                          _P]),
@@ -140,10 +143,23 @@ def alibi_slopes(H: int) -> list:
     return list(buf)
 
 
+def attn_prefill_workspace_size(B: int, T: int, KV: int, hd: int, rope_base: float,
+                                dtype=torch.bfloat16) -> int:
+    """Bytes of scratch the key rotation pass of attn_prefill uses (0: the keys are turned
+    inside the attention kernel)."""
+    dt = ATTN_BF16 if dtype == torch.bfloat16 else ATTN_F32
+    return int(lib().attn_prefill_workspace_size(B, T, KV, hd, float(rope_base), dt))
+
+
 def attn_prefill(q, k, v, out=None, lse=None, *, pos0: int = 0, rope_base: float = 0.0,
                  causal: bool = True, window: int = 0, alibi_slopes: Optional[Sequence] = None,
-                 stream=None):
-    """q [B,T,H,hd], k/v [B,T,KV,hd] (CUDA, fp32 or bf16) -> out [B,T,H,hd] (and lse [B,H,T])."""
+                 workspace=None, turn_keys_first: bool = True, stream=None):
+    """q [B,T,H,hd], k/v [B,T,KV,hd] (CUDA, fp32 or bf16) -> out [B,T,H,hd] (and lse [B,H,T]).
+
+    Where a separate key rotation pass applies (bf16, hd 128, RoPE on) the keys are turned
+    once into ``workspace`` (a device byte tensor of attn_prefill_workspace_size bytes;
+    allocated here when not given) before the attention kernel; ``turn_keys_first=False``
+    turns them inside the attention kernel instead (no workspace)."""
     B, T, H, hd = q.shape
     KV = k.shape[2]
     if k.shape != (B, T, KV, hd) or v.shape != k.shape:
@@ -153,10 +169,18 @@ def attn_prefill(q, k, v, out=None, lse=None, *, pos0: int = 0, rope_base: float
     dt = q.dtype
     if out is None:
         out = torch.empty_like(q)
-    st = lib().attn_prefill(_dev(q, "q"), _dev(k, "k", dt), _dev(v, "v", dt), _dev(out, "out", dt),
-                            _dev(lse, "lse", torch.float32), B, T, H, KV, hd, int(pos0),
-                            float(rope_base), int(bool(causal)), int(window),
-                            _slopes(alibi_slopes, H), _dtype(q), _stream(stream))
+    ws_ptr, ws_bytes = 0, 0
+    if turn_keys_first:
+        need = attn_prefill_workspace_size(B, T, KV, hd, rope_base, dt)
+        if need > 0:
+            if workspace is None:
+                workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+            ws_ptr = _dev(workspace, "workspace")
+            ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib().attn_prefill_ws(_dev(q, "q"), _dev(k, "k", dt), _dev(v, "v", dt), _dev(out, "out", dt),
+                               _dev(lse, "lse", torch.float32), B, T, H, KV, hd, int(pos0),
+                               float(rope_base), int(bool(causal)), int(window),
+                               _slopes(alibi_slopes, H), _dtype(q), ws_ptr, ws_bytes, _stream(stream))
     _check(st)
     return out
 

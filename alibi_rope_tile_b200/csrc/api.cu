@@ -118,9 +118,14 @@ int check_common(int H, int KV, int hd, int dtype, float rope_base) {
 
 extern "C" {
 
-int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int T,
-                 int H, int KV, int hd, long long pos0, float rope_base, int causal, int window,
-                 const float* alibi_slopes, int dtype, void* stream) {
+size_t attn_prefill_workspace_size(int B, int T, int KV, int hd, float rope_base, int dtype) {
+  if (B < 1 || T < 1 || KV < 1 || dtype != ATTN_BF16 || hd != 128 || !(rope_base > 0.f)) return 0;
+  return (size_t)B * T * KV * hd * 2;
+}
+
+int attn_prefill_ws(const void* q, const void* k, const void* v, void* out, float* lse, int B, int T,
+                    int H, int KV, int hd, long long pos0, float rope_base, int causal, int window,
+                    const float* alibi_slopes, int dtype, void* workspace, size_t ws_bytes, void* stream) {
   int st = check_common(H, KV, hd, dtype, rope_base);
   if (st) return st;
   if (!q || !k || !v || !out) return fail(ATTN_ERR_ARG, "q, k, v and out must not be NULL");
@@ -133,6 +138,14 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
   if (pos0 < 0 || pos0 + (long long)T >= (1LL << 24))
     return fail(ATTN_ERR_ARG, "positions pos0..pos0+T-1 must lie in [0, 2^24)");
   if ((long long)B * T * H * hd >= (1LL << 40)) return fail(ATTN_ERR_ARG, "tensor too large");
+  // the key rotation pass runs when it applies and the caller gave its scratch
+  const size_t need = attn_prefill_workspace_size(B, T, KV, hd, rope_base, dtype);
+  if (workspace) {
+    if (!aligned16(workspace)) return fail(ATTN_ERR_ALIGN, "workspace must be 16-byte aligned");
+    if (ws_bytes < need)
+      return fail(ATTN_ERR_WORKSPACE, "prefill needs %zu bytes of workspace (got %zu)", need, ws_bytes);
+  }
+  const bool turn_first = workspace && need > 0;
 
   PrefillParams p;
   std::memset(&p, 0, sizeof(p));
@@ -146,10 +159,23 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
   p.status = device_status(&err);
   if (!p.status) return err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (turn_first) {
+    cudaError_t e = launch_rope_keys(k, workspace, B, T, KV, hd, p.pos0, p.rope, s);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_prefill_ws key rotation launch");
+    p.k = workspace;
+    p.k_rotated = 1;
+  }
   cudaError_t e = prefill_tc_supported(p, dtype) ? launch_prefill_tc(p, s)
                                                  : launch_prefill_simt(p, dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "attn_prefill launch");
   return ok();
+}
+
+int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int T,
+                 int H, int KV, int hd, long long pos0, float rope_base, int causal, int window,
+                 const float* alibi_slopes, int dtype, void* stream) {
+  return attn_prefill_ws(q, k, v, out, lse, B, T, H, KV, hd, pos0, rope_base, causal, window,
+                         alibi_slopes, dtype, nullptr, 0, stream);
 }
 
 int attn_prefill_chunk(const void* q, const void* kcache, const void* vcache, const int* seqlens,

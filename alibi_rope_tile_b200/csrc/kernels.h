@@ -136,6 +136,11 @@ cudaError_t launch_rms_inverse(const void* x, float* rinv, int M, int d, float e
 cudaError_t launch_fold_gamma(const void* W, const void* gamma, void* Wg, int d, int N, cudaStream_t s);
 cudaError_t launch_rope_table(float2* cs, int T, int pos0, const RopeFreqs& rope, int hd, cudaStream_t s);
 
+// Key rotation pass (bf16, hd % 8 == 0): kr [B,T,KV,hd] = k turned at positions pos0 + t.
+// The prefill then runs with k_rotated set on kr.
+cudaError_t launch_rope_keys(const void* k, void* kr, int B, int T, int KV, int hd, int pos0,
+                             const RopeFreqs& rope, cudaStream_t s);
+
 // Records a failure for attn_last_error() and returns ``code`` (used by entry points
 // defined outside api.cu).
 int record_error(int code, const char* message);

@@ -233,13 +233,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // hd = 128: key-tile start angles by recurrence; hd = 64 (half the rotation work per
     // tile, and registers are tighter) computes each accurately
     if constexpr (HD == 128)
-      if (p.rope.on && !CHUNK) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
+      if (p.rope.on && !CHUNK && !p.k_rotated) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
     int u = 0;
     for (int j = jt0; j <= jt1; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++u) {
         const int st = u % C::NS, n = u / C::NS;
         if (!mbar_wait(kv_full + st, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        if (kv == 0 && p.rope.on && !CHUNK) {  // cached keys are already rotated
+        if (kv == 0 && p.rope.on && !CHUNK && !p.k_rotated) {  // cached or pre-turned keys
           if constexpr (HD == 128)
             krot.rotate_next(sKV + st * C::KV_BYTES);
           else

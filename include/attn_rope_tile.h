@@ -85,10 +85,38 @@ typedef enum {
  * causal: 0 or 1. window: <= 0 none, else W >= 1 (requires causal).
  * bf16 with hd in {64, 128} runs the tensor-core (tcgen05/TMEM) kernel; other shapes
  * and fp32 run the CUDA-core kernel. Returns ATTN_OK or an attn_status.
+ * The keys are turned inside the attention kernel as its tiles land (every CTA that reads
+ * a key tile turns it); attn_prefill_ws turns them once in a pass of their own instead.
  */
 int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse,
                  int B, int T, int H, int KV, int hd, long long pos0, float rope_base,
                  int causal, int window, const float* alibi_slopes, int dtype, void* stream);
+
+/*
+ * attn_prefill_workspace_size -- bytes of device scratch attn_prefill_ws uses to hold the
+ * turned keys: B*T*KV*hd*2 for bf16 with hd = 128 and rope_base > 0 (where a separate key
+ * rotation pass is faster than turning each key tile in every CTA that reads it), else 0.
+ * Returns 0 on invalid sizes.
+ */
+size_t attn_prefill_workspace_size(int B, int T, int KV, int hd, float rope_base, int dtype);
+
+/*
+ * attn_prefill_ws -- attn_prefill with caller-owned scratch ([LAB] rope: turning a key
+ * depends only on its own position, so it may be done once, before the attention).
+ *
+ * Arguments and results are those of attn_prefill, plus workspace: NULL (ws_bytes 0), or
+ * 16-byte aligned device memory of at least attn_prefill_workspace_size(B,T,KV,hd,
+ * rope_base,dtype) bytes, owned by the caller, contents on entry irrelevant. When that
+ * size is non-zero and the workspace is given, two kernels run on stream: the rotation pass
+ * writes k turned at positions pos0+j into the workspace (fp32 arithmetic, rounded once to
+ * bf16), then the attention kernel reads the keys from there. Otherwise (size 0 or
+ * workspace NULL) this is attn_prefill. A non-NULL workspace smaller than the size query
+ * returns ATTN_ERR_WORKSPACE; a misaligned one ATTN_ERR_ALIGN.
+ */
+int attn_prefill_ws(const void* q, const void* k, const void* v, void* out, float* lse,
+                    int B, int T, int H, int KV, int hd, long long pos0, float rope_base,
+                    int causal, int window, const float* alibi_slopes, int dtype, void* workspace,
+                    size_t ws_bytes, void* stream);
 
 /*
  * attn_prefill_chunk -- a chunk of Tq query rows that continues sequences held in a KV

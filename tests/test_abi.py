@@ -34,6 +34,7 @@ def test_header_declares_entry_points():
                  "attn_prefill_chunk", "attn_kv_write", "attn_decode_paged", "attn_kv_write_paged",
                  "attn_decode_latent", "attn_block_fused",
                  "attn_decode_workspace_size", "attn_block_workspace_size", "attn_alibi_slopes",
+                 "attn_prefill_ws", "attn_prefill_workspace_size",
                  "attn_sync_status", "attn_last_error", "attn_version"):
         assert must in names
 
@@ -111,6 +112,29 @@ def test_decode_workspace_error(lib):
     st = lib.attn_decode(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, 2, 4, 2, 48, 128,
                          10000.0, 0, None, 1, 0x1000, 1 << 30, None)
     assert st == -3      # hd = 48 is not a decode head size
+
+
+def test_prefill_workspace_size_and_errors(lib):
+    import alibi_rope_tile_b200 as art
+    # the key rotation pass applies to bf16, hd 128, RoPE on: one turned copy of k
+    assert lib.attn_prefill_workspace_size(2, 4096, 8, 128, 5e5, 1) == 2 * 4096 * 8 * 128 * 2
+    assert lib.attn_prefill_workspace_size(2, 100, 3, 128, 1e4, 1) == 2 * 100 * 3 * 128 * 2
+    assert lib.attn_prefill_workspace_size(2, 4096, 8, 128, 0.0, 1) == 0    # no rotation
+    assert lib.attn_prefill_workspace_size(4, 1024, 16, 64, 1e4, 1) == 0    # hd 64: in the kernel
+    assert lib.attn_prefill_workspace_size(2, 64, 8, 128, 1e4, 0) == 0      # fp32
+    assert lib.attn_prefill_workspace_size(0, 64, 8, 128, 1e4, 1) == 0      # invalid size
+    assert art.attn_prefill_workspace_size(1, 10, 2, 128, 1e4) == 10 * 2 * 128 * 2
+    need = lib.attn_prefill_workspace_size(1, 8, 2, 128, 1e4, 1)
+
+    def call(ws, n, **kw):
+        a = dict(B=1, T=8, H=4, KV=2, hd=128, base=1e4, window=0)
+        a.update(kw)
+        return lib.attn_prefill_ws(0x1000, 0x1000, 0x1000, 0x1000, None, a["B"], a["T"], a["H"],
+                                   a["KV"], a["hd"], 0, a["base"], 1, a["window"], None, 1, ws, n, None)
+    assert call(0x1000, need - 1) == -6          # workspace smaller than the size query
+    assert call(0x1008, need) == -2              # misaligned workspace
+    assert call(0x1000, need, H=6, KV=4) == -1   # argument errors come first
+    assert call(0x1000, need, T=0) == -1
 
 
 def test_block_workspace_error(lib):

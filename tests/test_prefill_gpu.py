@@ -26,13 +26,14 @@ def art():
     return m
 
 
-def run(art, q, k, v, w, with_lse=True):
+def run(art, q, k, v, w, with_lse=True, turn_keys_first=True):
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
     B, T, H, hd = q.shape
     lse = torch.empty(B, H, T, dtype=torch.float32, device="cuda") if with_lse else None
     slopes = art.alibi_slopes(H) if w.alibi else None
     out = art.attn_prefill(dq, dk, dv, lse=lse, pos0=w.pos0, rope_base=w.rope_base,
-                           causal=w.causal, window=w.window, alibi_slopes=slopes)
+                           causal=w.causal, window=w.window, alibi_slopes=slopes,
+                           turn_keys_first=turn_keys_first)
     torch.cuda.synchronize()
     art.attn_sync_status()
     return out, lse
@@ -79,6 +80,59 @@ def test_named_workload_full(art, wname):
     ro, rl = oracle(q, k, v, w)
     assert_close(out, ro, torch.bfloat16, w.name)
     assert_lse_close(lse, rl, torch.bfloat16, w.name)
+
+
+# hd = 128 with RoPE runs two ways: a key rotation pass into the workspace, then the
+# attention kernel on turned keys (the default), or the keys turned inside the attention
+# kernel as its tiles land (no workspace). Both must match the oracle.
+ROPE_FLAGS = sorted(f for f in FLAGS if FLAGS[f].get("rope_base", 0) > 0)
+SHAPES_128 = [s for s in SHAPES if s[4] == 128]
+
+
+@pytest.mark.parametrize("flags", ROPE_FLAGS)
+@pytest.mark.parametrize("shape", SHAPES_128, ids=lambda s: "B{}T{}H{}KV{}hd{}".format(*s))
+def test_small_keys_turned_in_kernel(art, shape, flags):
+    B, T, H, KV, hd = shape
+    w = workloads.small_prefill(B, T, H, KV, hd, seed=zlib.crc32(repr((shape, flags)).encode()) % 1000, **FLAGS[flags])
+    q, k, v = workloads.prefill_inputs(w, torch.bfloat16)
+    out, lse = run(art, q, k, v, w, turn_keys_first=False)
+    ro, rl = oracle(q, k, v, w)
+    assert_close(out, ro, torch.bfloat16, f"out {w.name} {flags} (keys turned in the kernel)")
+    assert_lse_close(lse, rl, torch.bfloat16, f"lse {w.name} {flags} (keys turned in the kernel)")
+
+
+def test_gqa_workload_keys_turned_in_kernel(art):
+    w = workloads.GQA
+    q, k, v = workloads.prefill_inputs(w)
+    out, lse = run(art, q, k, v, w, turn_keys_first=False)
+    ro, rl = oracle(q, k, v, w)
+    assert_close(out, ro, torch.bfloat16, w.name + " (keys turned in the kernel)")
+    assert_lse_close(lse, rl, torch.bfloat16, w.name + " (keys turned in the kernel)")
+
+
+def test_rotation_pass_workspace(art):
+    """The rotation pass writes exactly B*T*KV*hd bf16 values into a caller's workspace and
+    leaves the bytes after them alone; a larger, reused workspace gives the same output."""
+    w = workloads.small_prefill(2, 333, 8, 2, 128, seed=21, rope_base=10000.0, pos0=7)
+    q, k, v = workloads.prefill_inputs(w)
+    need = art.attn_prefill_workspace_size(2, 333, 2, 128, 10000.0)
+    assert need == 2 * 333 * 2 * 128 * 2
+    ws = torch.full((need + 4096,), 0x5A, dtype=torch.uint8, device="cuda")
+    dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
+    o1 = art.attn_prefill(dq, dk, dv, pos0=7, rope_base=10000.0, workspace=ws)
+    o2 = art.attn_prefill(dq, dk, dv, pos0=7, rope_base=10000.0, workspace=ws)
+    torch.cuda.synchronize()
+    art.attn_sync_status()
+    assert torch.equal(o1, o2)
+    assert bool((ws[need:] == 0x5A).all())
+    # the workspace holds the keys turned at positions pos0 + t: compare with the oracle's turn
+    # (fp32 arithmetic, about 1e-6 of the pair's size, then one rounding to bf16 within
+    # 2^-9 of the value)
+    kr = ws[:need].view(torch.bfloat16).view(2, 333, 2, 128).cpu().double().numpy()
+    ref = A.rope(k.permute(0, 2, 1, 3), np.arange(7, 7 + 333), 10000.0).transpose(0, 2, 1, 3)
+    assert np.all(np.abs(kr - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4)
+    ro, _ = oracle(q, k, v, w)
+    assert_close(o1, ro, torch.bfloat16, "out with a reused workspace")
 
 
 def long_rows(T=16384, W=4096, seed=3):
