@@ -42,6 +42,10 @@ cudaError_t launch_prefill_simt(const PrefillParams& p, int dtype, cudaStream_t 
 bool prefill_tc_supported(const PrefillParams& p, int dtype);
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t s);
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t s);
+// Persistent form of the single-slot kernel (one CTA per SM over all work units) for a
+// prefill without chunk mode whose keys need no turn in the kernel (k_rotated, or no RoPE).
+bool prefill_ps_supported(const PrefillParams& p);
+cudaError_t launch_prefill_ps(const PrefillParams& p, cudaStream_t s);
 
 struct DecodeParams {
   const void* q;        // [B,H,hd]

@@ -497,6 +497,9 @@ bool prefill_tc_supported(const PrefillParams& p, int dtype) {
 }
 
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t s) {
+  // no key to turn in the kernel (and no chunk): the persistent form, whose units' set-up and
+  // epilogues overlap their neighbours' key tiles
+  if (prefill_ps_supported(p)) return launch_prefill_ps(p, s);
   // hd = 128 with the keys turned in the kernel: the two-slot kernel turns each key tile
   // once per 256 query rows instead of once per 128
   if (p.hd == 128 && p.rope.on && !p.seqlens && !p.k_rotated) return launch_prefill_pair(p, s);
