@@ -156,7 +156,7 @@ def attn_prefill(q, k, v, out=None, lse=None, *, pos0: int = 0, rope_base: float
                  workspace=None, turn_keys_first: bool = True, stream=None):
     """q [B,T,H,hd], k/v [B,T,KV,hd] (CUDA, fp32 or bf16) -> out [B,T,H,hd] (and lse [B,H,T]).
 
-    Where a separate key rotation pass applies (bf16, hd 128, RoPE on) the keys are turned
+    Where a separate key rotation pass applies (bf16, hd 64 or 128, RoPE on) the keys are turned
     once into ``workspace`` (a device byte tensor of attn_prefill_workspace_size bytes;
     allocated here when not given) before the attention kernel; ``turn_keys_first=False``
     turns them inside the attention kernel instead (no workspace)."""

@@ -119,7 +119,7 @@ int check_common(int H, int KV, int hd, int dtype, float rope_base) {
 extern "C" {
 
 size_t attn_prefill_workspace_size(int B, int T, int KV, int hd, float rope_base, int dtype) {
-  if (B < 1 || T < 1 || KV < 1 || dtype != ATTN_BF16 || hd != 128 || !(rope_base > 0.f)) return 0;
+  if (B < 1 || T < 1 || KV < 1 || dtype != ATTN_BF16 || (hd != 64 && hd != 128) || !(rope_base > 0.f)) return 0;
   return (size_t)B * T * KV * hd * 2;
 }
 
@@ -164,6 +164,7 @@ int attn_prefill_ws(const void* q, const void* k, const void* v, void* out, floa
     if (e != cudaSuccess) return cuda_fail(e, "attn_prefill_ws key rotation launch");
     p.k = workspace;
     p.k_rotated = 1;
+    p.after_key_pass = 1;
   }
   cudaError_t e = prefill_tc_supported(p, dtype) ? launch_prefill_tc(p, s)
                                                  : launch_prefill_simt(p, dtype, s);

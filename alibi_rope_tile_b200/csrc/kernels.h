@@ -32,6 +32,10 @@ struct PrefillParams {
   // Keys arrive turned at positions pos0 + j (a block's key projection turned them in its
   // epilogue): only the queries are turned here.
   int k_rotated;
+  // The launch directly follows the key rotation pass, whose only output is k: the kernel may
+  // start while the pass finishes (programmatic dependent launch) and waits for it only
+  // before its first key/value load.
+  int after_key_pass;
 };
 
 // CUDA-core flash prefill: fp32 or bf16 elements, any even hd <= 256.

@@ -203,6 +203,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       bool ok = true;
       if (has_unit(0)) issue_q(0);
+      // after the key rotation pass (programmatic dependent launch), keys are read only once
+      // that grid has completed; without a dependency this returns at once
+      grid_dependency_wait();
       for (int n = 0; ok && has_unit(n); ++n) {
         const Unit x = unit(n);
         // The next unit's query tile goes into the one query buffer as soon as this unit's
@@ -533,8 +536,17 @@ cudaError_t launch_ps(const PrefillParams& p, cudaStream_t s) {
   auto kern = prefill_ps_kernel<HD>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<HD>::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)grid, NUM_THREADS, Cfg<HD>::SMEM, s>>>(mq, mk, mv, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = Cfg<HD>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.after_key_pass ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, a);
 }
 
 }  // namespace

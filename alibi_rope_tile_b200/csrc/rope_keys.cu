@@ -35,6 +35,9 @@ __global__ void __launch_bounds__(RK_THREADS) rope_keys_kernel(const uint4* __re
                                                               int B, int T, int KV, int chunks, int pos0,
                                                               const RopeFreqs rope) {
   __shared__ float2 cs[RK_POS][ATTN_MAX_PAIRS];
+  // the attention kernel that follows may be scheduled now; it waits for this grid's
+  // completion before it reads a key
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int t0 = blockIdx.x * RK_POS;
   const int np = min(RK_POS, T - t0);  // positions of this CTA
   const int half = chunks * 4;         // pairs per key

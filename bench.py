@@ -282,7 +282,7 @@ def build_families(art, only):
         slopes = art.alibi_slopes(w.H) if w.alibi else None
         ins = [(q.to(dev), k.to(dev), v.to(dev)) for _ in range(copies)]
         outs = [torch.empty(q.shape, dtype=q.dtype, device=dev) for _ in range(copies)]
-        # hd = 128 with RoPE: a key rotation pass into this workspace, then the attention
+        # bf16 with hd 64 or 128 and RoPE: a key rotation pass into this workspace, then the attention
         need = art.attn_prefill_workspace_size(w.B, w.T, w.KV, w.hd, w.rope_base)
         ws = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
 
@@ -302,7 +302,8 @@ def build_families(art, only):
             run(0)
             hout.copy_(outs[0], non_blocking=True)
 
-        kern = f"prefill_tc_kernel<{w.hd}, false>"
+        # keys turned by the pass, or no RoPE: the persistent kernel
+        kern = f"prefill_ps_kernel<{w.hd}>"
         note = ("two launches: the key rotation pass, then the attention kernel on turned keys; "
                 "the roofline's time is the whole step's") if need else None
         return Family(key, w.name, "TFLOP/s", "tensor", w.flops, 2 if need else 1, kern, run, reps=copies,

@@ -94,9 +94,9 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
 
 /*
  * attn_prefill_workspace_size -- bytes of device scratch attn_prefill_ws uses to hold the
- * turned keys: B*T*KV*hd*2 for bf16 with hd = 128 and rope_base > 0 (where a separate key
- * rotation pass is faster than turning each key tile in every CTA that reads it), else 0.
- * Returns 0 on invalid sizes.
+ * turned keys: B*T*KV*hd*2 for bf16 with hd in {64, 128} and rope_base > 0 (where a
+ * separate key rotation pass is faster than turning each key tile in every CTA that reads
+ * it), else 0. Returns 0 on invalid sizes.
  */
 size_t attn_prefill_workspace_size(int B, int T, int KV, int hd, float rope_base, int dtype);
 
@@ -109,7 +109,8 @@ size_t attn_prefill_workspace_size(int B, int T, int KV, int hd, float rope_base
  * rope_base,dtype) bytes, owned by the caller, contents on entry irrelevant. When that
  * size is non-zero and the workspace is given, two kernels run on stream: the rotation pass
  * writes k turned at positions pos0+j into the workspace (fp32 arithmetic, rounded once to
- * bf16), then the attention kernel reads the keys from there. Otherwise (size 0 or
+ * bf16), then the persistent attention kernel reads the keys from there (it may start while
+ * the pass finishes, and reads no key before the pass has completed). Otherwise (size 0 or
  * workspace NULL) this is attn_prefill. A non-NULL workspace smaller than the size query
  * returns ATTN_ERR_WORKSPACE; a misaligned one ATTN_ERR_ALIGN.
  */

@@ -116,11 +116,12 @@ def test_decode_workspace_error(lib):
 
 def test_prefill_workspace_size_and_errors(lib):
     import alibi_rope_tile_b200 as art
-    # the key rotation pass applies to bf16, hd 128, RoPE on: one turned copy of k
+    # the key rotation pass applies to bf16, hd 64 or 128, RoPE on: one turned copy of k
     assert lib.attn_prefill_workspace_size(2, 4096, 8, 128, 5e5, 1) == 2 * 4096 * 8 * 128 * 2
     assert lib.attn_prefill_workspace_size(2, 100, 3, 128, 1e4, 1) == 2 * 100 * 3 * 128 * 2
     assert lib.attn_prefill_workspace_size(2, 4096, 8, 128, 0.0, 1) == 0    # no rotation
-    assert lib.attn_prefill_workspace_size(4, 1024, 16, 64, 1e4, 1) == 0    # hd 64: in the kernel
+    assert lib.attn_prefill_workspace_size(4, 1024, 16, 64, 1e4, 1) == 4 * 1024 * 16 * 64 * 2
+    assert lib.attn_prefill_workspace_size(1, 64, 2, 32, 1e4, 1) == 0       # hd 32: in the kernel
     assert lib.attn_prefill_workspace_size(2, 64, 8, 128, 1e4, 0) == 0      # fp32
     assert lib.attn_prefill_workspace_size(0, 64, 8, 128, 1e4, 1) == 0      # invalid size
     assert art.attn_prefill_workspace_size(1, 10, 2, 128, 1e4) == 10 * 2 * 128 * 2

@@ -82,11 +82,11 @@ def test_named_workload_full(art, wname):
     assert_lse_close(lse, rl, torch.bfloat16, w.name)
 
 
-# hd = 128 with RoPE runs two ways: a key rotation pass into the workspace, then the
-# attention kernel on turned keys (the default), or the keys turned inside the attention
-# kernel as its tiles land (no workspace). Both must match the oracle.
+# bf16 with hd 64 or 128 and RoPE runs two ways: a key rotation pass into the workspace, then
+# the persistent attention kernel on turned keys (the default), or the keys turned inside the
+# attention kernel as its tiles land (no workspace). Both must match the oracle.
 ROPE_FLAGS = sorted(f for f in FLAGS if FLAGS[f].get("rope_base", 0) > 0)
-SHAPES_128 = [s for s in SHAPES if s[4] == 128]
+SHAPES_128 = [s for s in SHAPES if s[4] in (64, 128)]
 
 
 @pytest.mark.parametrize("flags", ROPE_FLAGS)
