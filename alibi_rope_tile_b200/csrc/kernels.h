@@ -47,7 +47,7 @@ bool prefill_tc_supported(const PrefillParams& p, int dtype);
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t s);
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t s);
 // Persistent form of the single-slot kernel (one CTA per SM over all work units) for a
-// prefill without chunk mode whose keys need no turn in the kernel (k_rotated, or no RoPE).
+// prefill whose keys need no turn in the kernel (k_rotated, a chunk over a cache, or no RoPE).
 bool prefill_ps_supported(const PrefillParams& p);
 cudaError_t launch_prefill_ps(const PrefillParams& p, cudaStream_t s);
 

@@ -1,6 +1,6 @@
 // Persistent tensor-core flash prefill for sm_100a, the form for keys that need no turn inside
-// the kernel (turned by the key rotation pass or a block's key projection, or no rotary
-// embedding at all). One CTA per SM walks a list of work units; its roles run on from one
+// the kernel (turned by the key rotation pass or a block's key projection, read from a cache
+// that holds them turned, or no rotary embedding at all). One CTA per SM walks a list of work units; its roles run on from one
 // unit to the next, so a unit's set-up (the query tile's load, turn and move into tensor
 // memory) and its epilogue (normalising and storing the output rows) overlap the key tiles
 // of its neighbours instead of idling the tensor core between CTAs.
@@ -22,8 +22,8 @@
 // from, S double-buffered. Tensor memory (512 columns): O (hd) | Q0, Q1 (hd/2 each, bf16
 // pairs, alternate units) | S0 (128) | S1 (128) from column 256.
 // Issue order over the CTA's tiles t (all units in sequence): QK(0); then per tile t:
-// QK(t+1) (the next unit's first tile after a unit's last), PV(t). The first PV of a unit
-// waits until the previous unit's output has been read out of O.
+// QK(t+1) (after a unit's last tile: the next unit's first, if it has keys), PV(t). The
+// first PV of a unit waits until the previous unit's output has been read out of O.
 //
 // Warp roles (22 warps):
 //   warps 0-15  softmax: warp w owns TMEM lanes 32*(w%4).. (32 query rows) and keys
@@ -39,7 +39,9 @@
 // only where the waiter is at most one unit behind.
 //
 // Masking: a pair outside the causal/window/length limits gets -inf before the row max, so
-// its weight is exactly 0; tiles outside a unit's key range are skipped entirely.
+// its weight is exactly 0; tiles outside a unit's key range are skipped entirely. In chunk
+// mode (queries that continue sequences held in a cache) a unit may attend no key at all:
+// it has no tiles and writes zero rows with lse = -inf.
 #include <algorithm>
 
 #include "prefill_common.cuh"
@@ -92,8 +94,12 @@ struct PsArgs {
   float scale_log2;
 };
 
+// A unit's rows and key range. Keys are indexed by position in k/v (a prefill: key j is row
+// j) or by cache slot (chunk mode); qoff is the key index of query row 0, Tk the number of
+// keys, qrope0 the position of row 0; the nt tiles from jt0 on hold the unit's keys.
 struct Unit {
-  int b, h, g, qs, jt0, jt1;
+  int b, h, g, qs, qoff, Tk, qrope0, jt0, nt;
+  bool bad;  // chunk mode: the sequence's cache position or length is out of range
 };
 
 // Rank of the n-th unit of this CTA (>= nunits: none; ranks grow with n).
@@ -103,6 +109,7 @@ __device__ __forceinline__ int unit_rank(int n) {
 }
 
 // The unit of a rank: longest rows first, heads of one key/value group adjacent.
+template <bool CHUNK>
 __device__ __forceinline__ Unit unit_at(const PrefillParams& p, int nqb, int rank) {
   Unit x;
   const int per_qb = p.B * p.H;
@@ -112,17 +119,31 @@ __device__ __forceinline__ Unit unit_at(const PrefillParams& p, int nqb, int ran
   x.b = rest / p.H;
   x.g = x.h / (p.H / p.KV);
   x.qs = qb * BM;
-  // keys lo..hi (a prefill's key j is row j); lo <= qs <= hi, so every unit has a tile
-  const int lo = p.window > 0 ? max(0, x.qs - p.window + 1) : 0;
-  const int hi = p.causal ? min(p.T - 1, x.qs + BM - 1) : p.T - 1;
-  x.jt0 = lo / BN;
-  x.jt1 = hi / BN;
+  x.qoff = 0;
+  x.Tk = p.T;
+  x.qrope0 = p.pos0;
+  x.bad = false;
+  if constexpr (CHUNK) {
+    x.qoff = p.qpos0[x.b];
+    x.Tk = p.seqlens[x.b];
+    x.qrope0 = x.qoff;
+    if (x.qoff < 0 || x.qoff > (1 << 24) - p.T || x.Tk < 0 || x.Tk > p.Lk) {
+      x.bad = true;
+      x.qoff = 0;
+      x.Tk = 0;  // nothing is attended: zero rows
+    }
+  }
+  // keys lo..hi (in a prefill lo <= qs <= hi: every unit has a tile)
+  const int lo = p.window > 0 ? max(0, x.qoff + x.qs - p.window + 1) : 0;
+  const int hi = p.causal ? min(x.Tk - 1, x.qoff + x.qs + BM - 1) : x.Tk - 1;
+  x.jt0 = lo <= hi ? lo / BN : 0;
+  x.nt = lo <= hi ? hi / BN - x.jt0 + 1 : 0;
   return x;
 }
 
 __device__ __forceinline__ void qe_sync() { asm volatile("bar.sync %0, 128;" ::"n"(QE_BARRIER) : "memory"); }
 
-template <int HD>
+template <int HD, bool CHUNK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_ps_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ PsArgs a) {
@@ -154,7 +175,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const PrefillParams& p = a.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   auto has_unit = [&](int n) { return unit_rank(n) < a.nunits; };
-  auto unit = [&](int n) { return unit_at(p, a.nqb, unit_rank(n)); };
+  auto unit = [&](int n) { return unit_at<CHUNK>(p, a.nqb, unit_rank(n)); };
 
   // ---- set-up: barriers, tensor memory
   if (tid == 0) {
@@ -208,11 +229,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       grid_dependency_wait();
       for (int n = 0; ok && has_unit(n); ++n) {
         const Unit x = unit(n);
+        if (x.bad) flag_error(p.status, DEV_BAD_ARG);
         // The next unit's query tile goes into the one query buffer as soon as this unit's
         // tile has moved into tensor memory (q_rot of unit n; it cannot be a phase ahead,
         // as unit n+2's tile needs the load issued here).
         bool q_next = !has_unit(n + 1);
-        const int total = 2 * (x.jt1 - x.jt0 + 1);  // K and V of every tile
+        const int total = 2 * x.nt;  // K and V of every tile
         for (int k = 0; k < total; ++k, ++u) {
           if (!q_next && mbar_test_wait(q_rot + (n & 1), (n >> 1) & 1)) {
             issue_q(n + 1);
@@ -252,7 +274,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     auto prep = [&](int n) -> bool {
       const Unit x = unit(n);
       if (!mbar_wait(q_full, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) return false;
-      if (p.rope.on) krot.rotate(sQ, p.pos0 + x.qs, p.rope);
+      if (p.rope.on) krot.rotate(sQ, x.qrope0 + x.qs, p.rope);
       qe_sync();
       const uint32_t base = smem_u32(sQ);
       const uint32_t colq = C::COL_Q + (uint32_t)(n & 1) * (HD / 2);
@@ -290,6 +312,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
                                             (((size_t)x.b * p.T + i) * p.H + x.h) * HD);
+      if (x.nt == 0) {
+        // no key attended (chunk mode): zero rows; O belongs to another unit and is not read
+        if (i < p.T)
+          for (int v4 = 0; v4 < HD / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+      } else {
 #pragma unroll
       for (int hb = 0; hb < HD / 32; ++hb) {
         float o[32];
@@ -303,6 +330,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                           f2_to_bf2(o[8 * v4 + 4] * inv, o[8 * v4 + 5] * inv),
                                           f2_to_bf2(o[8 * v4 + 6] * inv, o[8 * v4 + 7] * inv));
         }
+      }
       }
       tc_fence_before();
       mbar_arrive(o_free);
@@ -346,25 +374,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         return mbar_wait(kv_full + u % C::NS, (u / C::NS) & 1, abort_flag, p.status, WAIT_LIMIT_NS);
       };
       int t = 0;
-      if (!has_unit(0)) goto mma_drain;
-      if (!mbar_wait(q_rot, 0, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
-      if (!wait_kv(0)) goto mma_drain;
-      tc_fence_after();
-      issue_qk(0, 0, 0);
-      umma_commit(s_full);
-      umma_commit(kv_empty);
+      // QK of a unit's first tile: issued ahead, during the previous unit's last tile, when
+      // that unit had tiles; otherwise (the CTA's first unit, or one after a unit without
+      // keys) at the unit's start. Its query buffer's q_rot cannot be a phase ahead: unit
+      // n+2's query waits for the epilogue of unit n, which waits for unit n's MMAs.
+      bool first_qk_issued = false;
       for (int n = 0; has_unit(n); ++n) {
         const Unit x = unit(n);
-        const int nt = x.jt1 - x.jt0 + 1;
-        const bool more = has_unit(n + 1);
+        const int nt = x.nt;
+        if (nt > 0 && !first_qk_issued) {
+          if (!mbar_wait(q_rot + (n & 1), (n >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto mma_drain;
+          if (!wait_kv(2 * t)) goto mma_drain;
+          tc_fence_after();
+          issue_qk(t & 1, (2 * t) % C::NS, n & 1);
+          umma_commit(s_full + (t & 1));
+          umma_commit(kv_empty + (2 * t) % C::NS);
+        }
+        first_qk_issued = false;
+        const bool next_has_tiles = has_unit(n + 1) && unit(n + 1).nt > 0;
         for (int i = 0; i < nt; ++i, ++t) {
-          // QK of the CTA's next tile: this unit's next one, or the next unit's first (its
-          // query buffer's q_rot cannot be a phase ahead: unit n+3's query waits for the
-          // epilogue of unit n, which waits for this unit's MMAs)
-          if (i + 1 < nt || more) {
+          // QK of the CTA's next tile: this unit's next one, or the next unit's first
+          if (i + 1 < nt || next_has_tiles) {
             const int nq = i + 1 < nt ? n : n + 1;
-            if (nq != n && !mbar_wait(q_rot + (nq & 1), (nq >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS))
-              goto mma_drain;
+            if (nq != n) {
+              if (!mbar_wait(q_rot + (nq & 1), (nq >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS))
+                goto mma_drain;
+              first_qk_issued = true;
+            }
             const int uK = 2 * (t + 1);
             if (!wait_kv(uK)) goto mma_drain;
             tc_fence_after();
@@ -382,8 +418,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           issue_pv(t & 1, uV % C::NS, i > 0);
           umma_commit(o_done + (t & 1));
           umma_commit(kv_empty + uV % C::NS);
-          if (i + 1 == nt) umma_commit(unit_done);
         }
+        // Every MMA of the unit completed. A unit without keys has no PV to wait for the
+        // previous unit's epilogue; it waits here, so that unit_done never runs two phases
+        // ahead of the epilogue warps that wait on it.
+        if (nt == 0 && n > 0 && !mbar_wait(o_free, (n - 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS))
+          goto mma_drain;
+        umma_commit(unit_done);
       }
     mma_drain:
       // every MMA issued above completes before tensor memory is released
@@ -402,11 +443,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float sc = a.scale_log2;
-    const int Tk = p.T;
     int t = 0;  // tile count over the CTA's units
     for (int n = 0; has_unit(n); ++n) {
       const Unit x = unit(n);
-      const int ip = x.qs + r;  // the query's key index (a prefill: its row)
+      const int Tk = x.Tk;
+      const int q0 = x.qoff + x.qs;  // key index of the unit's first query row
+      const int ip = q0 + r;         // the query's key index
       const float slope = p.alibi.on ? p.alibi.slope[x.h] * LOG2E : 0.f;
       // Row state in the log2 domain: m_ref is the reference the weights are taken against
       // (-inf until the row has seen an allowed key), l the running sum of this warp's share
@@ -414,15 +456,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // 8 (a factor 256), so O is rescaled rarely; weights stay below 2^8.
       float m_ref = -INFINITY, l = 0.f;
 #pragma unroll 1
-      for (int j = x.jt0; j <= x.jt1; ++j, ++t) {
+      for (int j = x.jt0; j < x.jt0 + x.nt; ++j, ++t) {
         const int buf = t & 1;
         if (!mbar_wait(s_full + buf, (t >> 1) & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
         tc_fence_after();
         const uint32_t tS = tmem + lane_off + C::COL_S + buf * BN;
         const int key0 = j * BN + kq * 32;  // first of my 32 keys
         // does any row of this tile need per-element masking in my keys? (uniform per warp)
-        const bool need_mask = (key0 + 32 > Tk) || (p.causal && key0 + 31 > x.qs) ||
-                               (p.window > 0 && x.qs + BM - 1 - key0 >= p.window);
+        const bool need_mask = (key0 + 32 > Tk) || (p.causal && key0 + 31 > q0) ||
+                               (p.window > 0 && q0 + BM - 1 - key0 >= p.window);
         float xv[32];
         tmem_ld32(tS + kq * 32, xv);
         tmem_wait_ld();
@@ -517,8 +559,9 @@ done:
 template <int HD>
 cudaError_t launch_ps(const PrefillParams& p, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, p.q, p.B, p.T, p.H, HD) || !make_map(&mk, p.k, p.B, p.T, p.KV, HD) ||
-      !make_map(&mv, p.v, p.B, p.T, p.KV, HD))
+  const int Lk = p.seqlens ? p.Lk : p.T;  // rows of k and v
+  if (!make_map(&mq, p.q, p.B, p.T, p.H, HD) || !make_map(&mk, p.k, p.B, Lk, p.KV, HD) ||
+      !make_map(&mv, p.v, p.B, Lk, p.KV, HD))
     return cudaErrorInvalidValue;
   PsArgs a;
   a.p = p;
@@ -533,7 +576,7 @@ cudaError_t launch_ps(const PrefillParams& p, cudaStream_t s) {
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const int grid = (int)std::min<long long>(units, (long long)sms);
-  auto kern = prefill_ps_kernel<HD>;
+  auto kern = p.seqlens ? prefill_ps_kernel<HD, true> : prefill_ps_kernel<HD, false>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<HD>::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -553,7 +596,8 @@ cudaError_t launch_ps(const PrefillParams& p, cudaStream_t s) {
 }  // namespace tc
 
 bool prefill_ps_supported(const PrefillParams& p) {
-  return !p.seqlens && (p.k_rotated || !p.rope.on) && (p.hd == 64 || p.hd == 128);
+  // chunk mode reads keys turned in the cache
+  return (p.seqlens || p.k_rotated || !p.rope.on) && (p.hd == 64 || p.hd == 128);
 }
 
 cudaError_t launch_prefill_ps(const PrefillParams& p, cudaStream_t s) {

@@ -303,7 +303,7 @@ def build_families(art, only):
             hout.copy_(outs[0], non_blocking=True)
 
         # keys turned by the pass, or no RoPE: the persistent kernel
-        kern = f"prefill_ps_kernel<{w.hd}>"
+        kern = f"prefill_ps_kernel<{w.hd}, false>"
         note = ("two launches: the key rotation pass, then the attention kernel on turned keys; "
                 "the roofline's time is the whole step's") if need else None
         return Family(key, w.name, "TFLOP/s", "tensor", w.flops, 2 if need else 1, kern, run, reps=copies,
@@ -420,7 +420,7 @@ def chunk_family(art):
         C["q"].copy_(hq, non_blocking=True)
         run(0)
         ho.copy_(C["out"], non_blocking=True)
-    return Family("chunk", cw.name, "TFLOP/s", "tensor", cw.flops, 1, "prefill_tc_kernel<128, true>", run,
+    return Family("chunk", cw.name, "TFLOP/s", "tensor", cw.flops, 1, "prefill_ps_kernel<128, true>", run,
                   e2e=(tnb(hcq), tnb(hcq), e2e_step))
 
 

@@ -94,6 +94,44 @@ def test_chunk_over_empty_cache_is_zero(art):
 
 
 @pytest.mark.parametrize("hd", [64, 128])
+def test_chunk_units_without_keys_between_units_with_keys(art, hd):
+    """More units than SMs, every other sequence with an empty cache: CTAs of the persistent
+    kernel take units with and without keys in turn (zero rows, lse -inf for the empty ones)."""
+    B, Tq, H, KV, Lmax = 6, 300, 16, 4, 800
+    qpos0 = [0, 120, 7, 400, 0, 33]
+    seqlens = [0, 120 + Tq, 0, 400 + Tq, 0, 33 + Tq]
+    q, kc, vc, sl, qp = _cache_case(B, Tq, H, KV, hd, Lmax, qpos0, seqlens, seed=31 + hd)
+    lse = torch.empty(B, H, Tq, dtype=torch.float32, device="cuda")
+    out = art.attn_prefill_chunk(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), qp.cuda(), lse=lse,
+                                 rope_base=1e4, window=200)
+    torch.cuda.synchronize()
+    assert art.attn_sync_status() == 0
+    ref, ref_lse = A.chunk(q, kc, vc, sl.numpy(), qp.numpy(), rope_base=1e4, causal=True, window=200)
+    assert_close(out, ref, BF, f"mixed empty chunk hd{hd}")
+    assert_lse_close(lse, ref_lse, BF, f"mixed empty chunk lse hd{hd}")
+    for b in (0, 2, 4):
+        assert torch.count_nonzero(out[b]) == 0 and torch.all(torch.isneginf(lse[b]))
+
+
+def test_chunk_device_argument_error(art):
+    """A query position below 0 or a length beyond the cache is reported through
+    attn_sync_status; that sequence's rows are zero, the others are unaffected."""
+    B, Tq, H, KV, hd, Lmax = 3, 150, 8, 2, 128, 400
+    q, kc, vc, sl, qp = _cache_case(B, Tq, H, KV, hd, Lmax, [10, 20, 30], None, seed=41)
+    qp_bad = torch.tensor([10, -5, 30], dtype=torch.int32)
+    sl_bad = torch.tensor([10 + Tq, 20 + Tq, Lmax + 1], dtype=torch.int32)
+    out = art.attn_prefill_chunk(q.cuda(), kc.cuda(), vc.cuda(), sl_bad.cuda(), qp_bad.cuda(), rope_base=1e4)
+    torch.cuda.synchronize()
+    with pytest.raises(art.AttnError) as e:
+        art.attn_sync_status()
+    assert e.value.status == -7
+    art.attn_sync_status()  # cleared
+    assert torch.count_nonzero(out[1]) == 0 and torch.count_nonzero(out[2]) == 0
+    ref, _ = A.chunk(q[:1], kc[:1], vc[:1], sl[:1].numpy(), qp[:1].numpy(), rope_base=1e4)
+    assert_close(out[:1], ref, BF, "the valid sequence beside the bad ones")
+
+
+@pytest.mark.parametrize("hd", [64, 128])
 def test_chunks_on_the_gpu_equal_the_one_pass_prefill(art, hd):
     """Write each chunk's keys into the cache, run the chunk's queries, compare with the oracle's
     one-pass prefill, and with the GPU's own one-pass prefill."""
