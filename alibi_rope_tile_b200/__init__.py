@@ -32,6 +32,9 @@ SIGNATURES = {
     "attn_prefill_workspace_size": (_S, [_I, _I, _I, _I, _F, _I]),
     "attn_prefill_ws": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _F, _I, _I, _FP, _I, _P, _S,
                              _P]),
+    "attn_prefill_host_workspace_size": (_S, [_I, _I, _I, _I, _I, _F, _I]),
+    "attn_prefill_host": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _F, _I, _I, _FP, _I, _P, _S,
+                               _P]),
     "attn_decode_workspace_size": (_S, [_I, _I, _I, _I, _I]),
     "attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _FP, _I, _P, _S,
                          _P]),
@@ -181,6 +184,52 @@ def attn_prefill(q, k, v, out=None, lse=None, *, pos0: int = 0, rope_base: float
                                _dev(lse, "lse", torch.float32), B, T, H, KV, hd, int(pos0),
                                float(rope_base), int(bool(causal)), int(window),
                                _slopes(alibi_slopes, H), _dtype(q), ws_ptr, ws_bytes, _stream(stream))
+    _check(st)
+    return out
+
+
+def _host(t: Optional[torch.Tensor], name: str, dtype=None) -> int:
+    if t is None:
+        return 0
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return t.data_ptr()
+
+
+def attn_prefill_host_workspace_size(B: int, T: int, H: int, KV: int, hd: int, rope_base: float,
+                                     dtype=torch.bfloat16) -> int:
+    dt = ATTN_BF16 if dtype == torch.bfloat16 else ATTN_F32
+    return int(lib().attn_prefill_host_workspace_size(B, T, H, KV, hd, float(rope_base), dt))
+
+
+def attn_prefill_host(q, k, v, out=None, lse=None, *, pos0: int = 0, rope_base: float = 0.0,
+                      causal: bool = True, window: int = 0, alibi_slopes: Optional[Sequence] = None,
+                      workspace=None, stream=None):
+    """attn_prefill on HOST tensors (pinned memory lets the copies overlap the attention):
+    q [B,T,H,hd], k/v [B,T,KV,hd] -> out [B,T,H,hd] (and lse [B,H,T]) in host memory, written
+    once the stream reaches the end of the call. ``workspace``: a device byte tensor of
+    attn_prefill_host_workspace_size bytes (allocated here when not given)."""
+    B, T, H, hd = q.shape
+    KV = k.shape[2]
+    if k.shape != (B, T, KV, hd) or v.shape != k.shape:
+        raise ValueError(f"k and v must be [B,T,KV,hd] matching q {tuple(q.shape)}")
+    _shape(out, q.shape, "out")
+    _shape(lse, (B, H, T), "lse")
+    dt = q.dtype
+    if out is None:
+        out = torch.empty(q.shape, dtype=dt, pin_memory=True)
+    need = attn_prefill_host_workspace_size(B, T, H, KV, hd, rope_base, dt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+    st = lib().attn_prefill_host(_host(q, "q"), _host(k, "k", dt), _host(v, "v", dt), _host(out, "out", dt),
+                                 _host(lse, "lse", torch.float32), B, T, H, KV, hd, int(pos0),
+                                 float(rope_base), int(bool(causal)), int(window), _slopes(alibi_slopes, H),
+                                 _dtype(q), _dev(workspace, "workspace"),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st)
     return out
 

@@ -20,8 +20,8 @@
  *
  * Conventions shared by every entry point
  *   - Tensors are dense, row-major, contiguous, caller-owned DEVICE buffers unless a
- *     parameter says "host". The library never allocates, frees or keeps a pointer
- *     after a call returns.
+ *     parameter says "host". The library never allocates device memory, frees or keeps a
+ *     pointer after a call returns (attn_prefill_host keeps two copy streams per device).
  *   - Layouts: q and out [B, T, H, hd]; k and v [B, T, KV, hd]; decode q/out [B, H, hd];
  *     caches [B, Lmax, KV, hd]; lse (log-sum-exp of each softmax row, natural log, fp32)
  *     [B, H, T] for prefill and [B, H] for decode.
@@ -118,6 +118,40 @@ int attn_prefill_ws(const void* q, const void* k, const void* v, void* out, floa
                     int B, int T, int H, int KV, int hd, long long pos0, float rope_base,
                     int causal, int window, const float* alibi_slopes, int dtype, void* workspace,
                     size_t ws_bytes, void* stream);
+
+/*
+ * attn_prefill_host_workspace_size -- bytes of device scratch attn_prefill_host needs: dense
+ * device copies of q, k, v, out (and lse) cut into its slices, and the rotation pass's
+ * scratch for one slice. Returns 0 on invalid sizes.
+ */
+size_t attn_prefill_host_workspace_size(int B, int T, int H, int KV, int hd, float rope_base, int dtype);
+
+/*
+ * attn_prefill_host -- attn_prefill_ws on q, k, v and results in HOST memory ([LAB]
+ * attention(): every (sequence, query head) reads only its own key/value head, so the problem
+ * splits into independent slices).
+ *
+ * q, k, v: [B,T,H,hd] / [B,T,KV,hd] host buffers (read); out: [B,T,H,hd] host buffer
+ * (written); lse: [B,H,T] fp32 host buffer or NULL. Page-locked (pinned) host memory lets the
+ * copies run asynchronously and overlap; pageable memory gives the same results without the
+ * overlap. workspace: 256-byte aligned device memory of at least
+ * attn_prefill_host_workspace_size(...) bytes, owned by the caller; it must not be in use by
+ * work that the call does not follow on `stream`. The other arguments are attn_prefill's.
+ * The call cuts the problem into slices: runs of whole sequences when B >= 4, else one
+ * sequence and a group of key/value heads with their query heads. It copies each slice's rows
+ * into the workspace on a copy stream of its own, runs the prefill of attn_prefill_ws on
+ * `stream` as soon as the slice has landed, and copies the slice's results back on a second
+ * copy stream, so copies in, attention and copies out of different slices overlap; every
+ * output row is computed exactly as by attn_prefill_ws over the whole tensors on the device.
+ * Asynchronous: work issued on `stream` after the call (a synchronisation included) sees out
+ * and lse in host memory. The copy streams and their events are created on the first call on a
+ * device and kept for the process. Returns ATTN_OK or an attn_status (ATTN_ERR_WORKSPACE for
+ * a missing or short workspace, ATTN_ERR_ALIGN for a misaligned one).
+ */
+int attn_prefill_host(const void* q, const void* k, const void* v, void* out, float* lse,
+                      int B, int T, int H, int KV, int hd, long long pos0, float rope_base,
+                      int causal, int window, const float* alibi_slopes, int dtype, void* workspace,
+                      size_t ws_bytes, void* stream);
 
 /*
  * attn_prefill_chunk -- a chunk of Tq query rows that continues sequences held in a KV

@@ -34,7 +34,8 @@ def test_header_declares_entry_points():
                  "attn_prefill_chunk", "attn_kv_write", "attn_decode_paged", "attn_kv_write_paged",
                  "attn_decode_latent", "attn_block_fused",
                  "attn_decode_workspace_size", "attn_block_workspace_size", "attn_alibi_slopes",
-                 "attn_prefill_ws", "attn_prefill_workspace_size",
+                 "attn_prefill_ws", "attn_prefill_workspace_size", "attn_prefill_host",
+                 "attn_prefill_host_workspace_size",
                  "attn_sync_status", "attn_last_error", "attn_version"):
         assert must in names
 
@@ -136,6 +137,28 @@ def test_prefill_workspace_size_and_errors(lib):
     assert call(0x1008, need) == -2              # misaligned workspace
     assert call(0x1000, need, H=6, KV=4) == -1   # argument errors come first
     assert call(0x1000, need, T=0) == -1
+
+
+def test_prefill_host_workspace_and_errors(lib):
+    import alibi_rope_tile_b200 as art
+    n = lib.attn_prefill_host_workspace_size(2, 4096, 32, 8, 128, 5e5, 1)
+    # dense device copies of q, k, v, out and lse, plus one slice's rotation scratch
+    assert n >= 2 * 4096 * (2 * 32 + 2 * 8) * 128 * 2 + 2 * 32 * 4096 * 4
+    assert lib.attn_prefill_host_workspace_size(2, 4096, 30, 8, 128, 5e5, 1) == 0   # H % KV
+    assert lib.attn_prefill_host_workspace_size(0, 4096, 32, 8, 128, 5e5, 1) == 0   # B
+    assert art.attn_prefill_host_workspace_size(5, 100, 8, 2, 64, 1e4) > 0
+    need = lib.attn_prefill_host_workspace_size(1, 8, 4, 2, 128, 1e4, 1)
+
+    def call(ws, nbytes, **kw):
+        a = dict(B=1, T=8, H=4, KV=2, hd=128)
+        a.update(kw)
+        return lib.attn_prefill_host(0x1000, 0x1000, 0x1000, 0x1000, None, a["B"], a["T"], a["H"], a["KV"],
+                                     a["hd"], 0, 1e4, 1, 0, None, 1, ws, nbytes, None)
+    assert call(None, 0) == -6              # no workspace
+    assert call(0x1000, need - 1) == -6     # too small
+    assert call(0x1010, need) == -2         # not 256-byte aligned
+    assert call(0x1000, need, H=6, KV=4) == -1
+    assert call(0x1000, need, hd=7) == -1
 
 
 def test_block_workspace_error(lib):
