@@ -87,8 +87,7 @@ struct TcArgs {
   float scale_log2;
 };
 
-// CHUNK: the queries continue sequences held in a cache (PrefillParams::seqlens != nullptr).
-template <int HD, bool CHUNK>
+template <int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ TcArgs a) {
@@ -134,19 +133,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     qs[0] = qb * 2 * BM;
     qs[1] = qs[0] + BM;
   }
-  // Keys are indexed by position in k/v (a prefill: key j = row j) or by cache slot (chunk
-  // mode); qoff is the key index of query row 0 and Tk the number of keys there are.
-  int qoff = 0, Tk = p.T, qrope0 = p.pos0;
-  if constexpr (CHUNK) {
-    qoff = p.qpos0[b];
-    Tk = p.seqlens[b];
-    qrope0 = qoff;
-    if (qoff < 0 || qoff > (1 << 24) - p.T || Tk < 0 || Tk > p.Lk) {
-      if (tid == 0) flag_error(p.status, DEV_BAD_ARG);
-      qoff = 0;
-      Tk = 0;  // nothing is attended: zero rows
-    }
-  }
+  // Key j is row j of k/v: qoff is the key index of query row 0, Tk the number of keys.
+  const int qoff = 0, Tk = p.T, qrope0 = p.pos0;
   int t0[2], t1[2];
   bool valid[2], has[2];
 #pragma unroll
@@ -233,13 +221,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // hd = 128: key-tile start angles by recurrence; hd = 64 (half the rotation work per
     // tile, and registers are tighter) computes each accurately
     if constexpr (HD == 128)
-      if (p.rope.on && !CHUNK && !p.k_rotated) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
+      if (p.rope.on && !p.k_rotated) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
     int u = 0;
     for (int j = jt0; j <= jt1; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++u) {
         const int st = u % C::NS, n = u / C::NS;
         if (!mbar_wait(kv_full + st, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        if (kv == 0 && p.rope.on && !CHUNK && !p.k_rotated) {  // cached or pre-turned keys
+        if (kv == 0 && p.rope.on && !p.k_rotated) {  // keys that arrive turned are not turned again
           if constexpr (HD == 128)
             krot.rotate_next(sKV + st * C::KV_BYTES);
           else
@@ -458,7 +446,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < 2; ++s) {
       const int c = s ? cs1 : cs0;
       if (c == 0) {
-        // a slot that attends no key at all (a chunk over an empty range): zero rows, lse -inf
+        // a slot that attends no key at all (not a prefill's rows, which see their own key):
+        // zero rows, lse -inf
         const int i = qs[s] + r;
         if (valid[s] && i < p.T) {
           if (kq * 32 < HD) {
@@ -516,9 +505,8 @@ done:
 template <int HD>
 cudaError_t launch_hd(const PrefillParams& p, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
-  const int Lk = p.seqlens ? p.Lk : p.T;  // rows of k and v
-  if (!make_map(&mq, p.q, p.B, p.T, p.H, HD) || !make_map(&mk, p.k, p.B, Lk, p.KV, HD) ||
-      !make_map(&mv, p.v, p.B, Lk, p.KV, HD))
+  if (!make_map(&mq, p.q, p.B, p.T, p.H, HD) || !make_map(&mk, p.k, p.B, p.T, p.KV, HD) ||
+      !make_map(&mv, p.v, p.B, p.T, p.KV, HD))
     return cudaErrorInvalidValue;
   TcArgs a;
   a.p = p;
@@ -530,7 +518,7 @@ cudaError_t launch_hd(const PrefillParams& p, cudaStream_t s) {
   a.scale_log2 = p.scale * LOG2E;
   const long long units = (long long)p.B * p.KV * a.npairs * a.nqb;
   if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
-  auto kern = prefill_pair_kernel<HD, false>;
+  auto kern = prefill_pair_kernel<HD>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<HD>::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)units, NUM_THREADS, Cfg<HD>::SMEM, s>>>(mq, mk, mv, a);

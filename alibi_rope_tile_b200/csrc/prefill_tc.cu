@@ -1,5 +1,9 @@
 // Tensor-core flash prefill for sm_100a: TMA-staged tiles, tcgen05 MMAs accumulating in
-// TMEM, warp-specialised online softmax, rotary embedding applied as tiles land.
+// TMEM, warp-specialised online softmax, rotary embedding applied as tiles land. One CTA per
+// 128-row unit; it serves attn_prefill without a workspace for hd = 64 with RoPE, where the keys
+// are turned inside the kernel (hd = 128 takes the two-slot kernel of prefill_pair.cu; every
+// prefill whose keys need no turn here, and every chunk, takes the persistent kernel of
+// prefill_persist.cu).
 //
 // What it computes is the attention core of "Write attention from scratch" (worked
 // example): per query row i, softmax over allowed keys j of
@@ -85,8 +89,7 @@ struct TcArgs {
   float scale_log2;
 };
 
-// CHUNK: the queries continue sequences held in a cache (PrefillParams::seqlens != nullptr).
-template <int HD, bool CHUNK>
+template <int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ TcArgs a) {
@@ -126,19 +129,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int b = rest / p.H;
   const int g = h / (p.H / p.KV);
   const int qs = qb * BM;
-  // Keys are indexed by position in k/v (a prefill: key j = row j) or by cache slot (chunk
-  // mode); qoff is the key index of query row 0 and Tk the number of keys there are.
-  int qoff = 0, Tk = p.T, qrope0 = p.pos0;
-  if constexpr (CHUNK) {
-    qoff = p.qpos0[b];
-    Tk = p.seqlens[b];
-    qrope0 = qoff;
-    if (qoff < 0 || qoff > (1 << 24) - p.T || Tk < 0 || Tk > p.Lk) {
-      if (tid == 0) flag_error(p.status, DEV_BAD_ARG);
-      qoff = 0;
-      Tk = 0;  // nothing is attended: zero rows
-    }
-  }
+  // Key j is row j of k/v: qoff is the key index of query row 0, Tk the number of keys.
+  const int qoff = 0, Tk = p.T, qrope0 = p.pos0;
   const int lo = p.window > 0 ? max(0, qoff + qs - p.window + 1) : 0;
   const int hi = p.causal ? min(Tk - 1, qoff + qs + BM - 1) : Tk - 1;
   const bool has = lo <= hi;  // the tile attends at least one key
@@ -236,13 +228,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // hd = 128: key-tile start angles by recurrence; hd = 64 (half the rotation work per
     // tile) computes each accurately
     if constexpr (HD == 128)
-      if (p.rope.on && !CHUNK && !p.k_rotated) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
+      if (p.rope.on && !p.k_rotated) krot.start_keys(p.pos0 + jt0 * BN, p.rope);
     int u = 0;
     for (int j = jt0; j <= jt1; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++u) {
         const int st = u % C::NS, n = u / C::NS;
         if (!mbar_wait(kv_full + st, n & 1, abort_flag, p.status, WAIT_LIMIT_NS)) goto done;
-        if (kv == 0 && p.rope.on && !CHUNK && !p.k_rotated) {  // cached keys are already rotated
+        if (kv == 0 && p.rope.on && !p.k_rotated) {  // keys that arrive turned are not turned again
           if constexpr (HD == 128)
             krot.rotate_next(sKV + st * C::KV_BYTES);
           else
@@ -420,7 +412,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     // ---- epilogue: out = O / l (bf16), lse = (m + log2 l) ln 2
     if (c == 0) {
-      // a tile that attends no key at all (a chunk over an empty range): zero rows, lse -inf
+      // a tile that attends no key at all (not a prefill's rows, which see their own key):
+      // zero rows, lse -inf
       if (i < p.T) {
         if (kq * 32 < HD) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
@@ -472,9 +465,9 @@ done:
 template <int HD>
 cudaError_t launch_hd(const PrefillParams& p, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
-  const int Lk = p.seqlens ? p.Lk : p.T;  // rows of k and v
-  if (!make_map(&mq, p.q, p.B, p.T, p.H, HD) || !make_map(&mk, p.k, p.B, Lk, p.KV, HD) ||
-      !make_map(&mv, p.v, p.B, Lk, p.KV, HD))
+  if (p.seqlens) return cudaErrorInvalidValue;  // chunks run on the persistent kernel
+  if (!make_map(&mq, p.q, p.B, p.T, p.H, HD) || !make_map(&mk, p.k, p.B, p.T, p.KV, HD) ||
+      !make_map(&mv, p.v, p.B, p.T, p.KV, HD))
     return cudaErrorInvalidValue;
   TcArgs a;
   a.p = p;
@@ -482,7 +475,7 @@ cudaError_t launch_hd(const PrefillParams& p, cudaStream_t s) {
   a.scale_log2 = p.scale * LOG2E;
   const long long units = (long long)p.B * p.H * a.nqb;
   if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
-  auto kern = p.seqlens ? prefill_tc_kernel<HD, true> : prefill_tc_kernel<HD, false>;
+  auto kern = prefill_tc_kernel<HD>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<HD>::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)units, NUM_THREADS, Cfg<HD>::SMEM, s>>>(mq, mk, mv, a);
@@ -497,8 +490,8 @@ bool prefill_tc_supported(const PrefillParams& p, int dtype) {
 }
 
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t s) {
-  // no key to turn in the kernel (and no chunk): the persistent form, whose units' set-up and
-  // epilogues overlap their neighbours' key tiles
+  // no key to turn in the kernel (keys turned before, no RoPE, or a chunk over the cache): the
+  // persistent form, whose units' set-up and epilogues overlap their neighbours' key tiles
   if (prefill_ps_supported(p)) return launch_prefill_ps(p, s);
   // hd = 128 with the keys turned in the kernel: the two-slot kernel turns each key tile
   // once per 256 query rows instead of once per 128

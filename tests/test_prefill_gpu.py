@@ -101,6 +101,28 @@ def test_small_keys_turned_in_kernel(art, shape, flags):
     assert_lse_close(lse, rl, torch.bfloat16, f"lse {w.name} {flags} (keys turned in the kernel)")
 
 
+# More units (128 query rows of one head) than SMs, with a ragged last block: every CTA of the
+# persistent kernel walks several units (the snake order, the query-buffer and statistics
+# hand-overs), with windows that cut the key range of later units.
+MULTI_UNIT = [
+    ((3, 1000, 16, 4, 128), dict(rope_base=1e4)),
+    ((2, 1100, 16, 2, 128), dict(rope_base=5e5, pos0=9, window=300, alibi=True)),
+    ((4, 777, 16, 16, 64), dict(rope_base=1e4, alibi=True)),
+    ((2, 650, 32, 8, 64), dict(rope_base=0.0, causal=False)),
+]
+
+
+@pytest.mark.parametrize("shape,flags", MULTI_UNIT, ids=lambda c: str(c) if isinstance(c, tuple) else "")
+def test_multi_unit_ragged(art, shape, flags):
+    B, T, H, KV, hd = shape
+    w = workloads.small_prefill(B, T, H, KV, hd, seed=zlib.crc32(repr(shape).encode()) % 1000, **flags)
+    q, k, v = workloads.prefill_inputs(w)
+    out, lse = run(art, q, k, v, w)
+    ro, rl = oracle(q, k, v, w)
+    assert_close(out, ro, torch.bfloat16, f"out {w.name}")
+    assert_lse_close(lse, rl, torch.bfloat16, f"lse {w.name}")
+
+
 def test_gqa_workload_keys_turned_in_kernel(art):
     w = workloads.GQA
     q, k, v = workloads.prefill_inputs(w)
