@@ -1,14 +1,16 @@
 // Persistent tensor-core flash prefill for sm_100a, the form for keys that need no turn inside
 // the kernel (turned by the key rotation pass or a block's key projection, read from a cache
-// that holds them turned, or no rotary embedding at all). One CTA per SM walks a list of work units; its roles run on from one
-// unit to the next, so a unit's set-up (the query tile's load, turn and move into tensor
-// memory) and its epilogue (normalising and storing the output rows) overlap the key tiles
-// of its neighbours instead of idling the tensor core between CTAs.
+// that holds them turned, or no rotary embedding at all). One CTA per SM walks a list of work
+// units; its roles run on from one unit to the next, so a unit's set-up (the query tile's
+// load, turn and move into tensor memory) and its epilogue (normalising and storing the
+// output rows) overlap the key tiles of its neighbours instead of idling the tensor core
+// between CTAs.
 //
 // What it computes is the attention core of "Write attention from scratch" (worked
 // example): per query row i, softmax over allowed keys j of
-//   (R(pos0+i) q_i . k'_j) / sqrt(hd) - slope_h |i - j|,  k'_j = R(pos0+j) k_j (turned already)
-// weighting the value rows, reached through the key-block recurrences of "Building
+//   (R(P_i) q_i . k'_j) / sqrt(hd) - slope_h |P_i - j|,  k'_j = R(j) k_j (turned already)
+// with P_i = pos0 + i (key j at position pos0 + j) or, in chunk mode, P_i = qpos0[b] + i over
+// cache slots j, weighting the value rows, reached through the key-block recurrences of "Building
 // grouped-query attention with RoPE and Flash Attention from scratch" (Step 3): a running
 // maximum, a running denominator and a rescaled output accumulator.
 //
