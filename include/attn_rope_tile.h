@@ -138,7 +138,9 @@ size_t attn_prefill_host_workspace_size(int B, int T, int H, int KV, int hd, flo
  * attn_prefill_host_workspace_size(...) bytes, owned by the caller; it must not be in use by
  * work that the call does not follow on `stream`. The other arguments are attn_prefill's.
  * The call cuts the problem into slices: runs of whole sequences when B >= 4, else one
- * sequence and a group of key/value heads with their query heads. It copies each slice's rows
+ * sequence and a group of key/value heads with their query heads; the last slice is cut
+ * finer (halving groups of key/value heads), as its attention and copy back are what remains
+ * once every slice's rows have landed. It copies each slice's rows
  * into the workspace on a copy stream of its own, runs the prefill of attn_prefill_ws on
  * `stream` as soon as the slice has landed, and copies the slice's results back on a second
  * copy stream, so copies in, attention and copies out of different slices overlap; every
