@@ -100,3 +100,44 @@ def test_host_prefill_back_to_back_calls_share_a_workspace(art):
     torch.cuda.synchronize()
     assert torch.equal(o1, device_run(art, q1, k1, v1, w1)[0])
     assert torch.equal(o2, device_run(art, q2, k2, v2, w2)[0])
+
+
+def test_host_prefill_from_two_threads(art):
+    """Two host threads, each with its own stream and workspace, call attn_prefill_host at
+    once (the calls share the device's copy streams; their enqueueing is serialised): every
+    result equals the device prefill's."""
+    import threading
+    shapes = [(2, 260, 8, 2, 128, 1e4), (1, 300, 16, 4, 64, 5e5)]
+    cases = []
+    for i, (B, T, H, KV, hd, base) in enumerate(shapes):
+        w = workloads.small_prefill(B, T, H, KV, hd, seed=50 + i, rope_base=base)
+        q, k, v = workloads.prefill_inputs(w)
+        cases.append((w, q.pin_memory(), k.pin_memory(), v.pin_memory()))
+    results = [[None] * 3 for _ in cases]
+    errors = []
+
+    def worker(i):
+        try:
+            w, q, k, v = cases[i]
+            s = torch.cuda.Stream()
+            ws = torch.empty(art.attn_prefill_host_workspace_size(w.B, w.T, w.H, w.KV, w.hd, w.rope_base),
+                             dtype=torch.uint8, device="cuda")
+            for r in range(3):
+                out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+                art.attn_prefill_host(q, k, v, out, rope_base=w.rope_base, workspace=ws, stream=s)
+                s.synchronize()
+                results[i][r] = out
+        except Exception as e:  # surfaced below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(len(cases))]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    assert not errors, errors
+    art.attn_sync_status()
+    for i, (w, q, k, v) in enumerate(cases):
+        ref, _ = device_run(art, q, k, v, w)
+        for r in range(3):
+            assert torch.equal(results[i][r], ref)
