@@ -441,12 +441,21 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
 #pragma unroll
           for (int e = 0; e < 4; ++e) rope_cos_sin(x.qp, p.rope.hi[cc * 4 + e], p.rope.lo[cc * 4 + e], cs[e], sn[e]);
         const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q);
-#pragma unroll 1
-        for (int row = tid / CH; row < 32; row += 128 / CH) {
+        // the thread's rows tid/CH, +RSTEP, ...: all their loads are issued before any is used
+        constexpr int RSTEP = 128 / CH, NROW = 32 / RSTEP;
+        uint4 u4[NROW];
+#pragma unroll
+        for (int k = 0; k < NROW; ++k) {
+          const int row = tid / CH + k * RSTEP;
+          u4[k] = row < G ? *reinterpret_cast<const uint4*>(q + ((size_t)x.b * p.H + x.kvh * G + row) * HD + cc * 8)
+                          : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < NROW; ++k) {
+          const int row = tid / CH + k * RSTEP;
           uint32_t w[4] = {0u, 0u, 0u, 0u};
           if (row < G) {
-            const uint4 u4 = *reinterpret_cast<const uint4*>(q + ((size_t)x.b * p.H + x.kvh * G + row) * HD + cc * 8);
-            const uint32_t in[4] = {u4.x, u4.y, u4.z, u4.w};
+            const uint32_t in[4] = {u4[k].x, u4[k].y, u4[k].z, u4[k].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               float2 f = bf2_to_f2(in[e]);
@@ -456,7 +465,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
           }
           const uint4 v = make_uint4(w[0], w[1], w[2], w[3]);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) sts128(smem_u32(sQ) + sw128_offset(32 * k + row, cc * 8, BM), v);
+          for (int kk = 0; kk < 4; ++kk) sts128(smem_u32(sQ) + sw128_offset(32 * kk + row, cc * 8, BM), v);
         }
         fence_proxy_async();
         tc_fence_before();  // the previous piece's O reads are complete before this arrive
