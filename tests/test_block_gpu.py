@@ -50,7 +50,7 @@ def test_tiny_block_lab_properties_on_gpu(art):
 
 
 @pytest.mark.parametrize("shape", [(2, 256, 512, 8, 2), (1, 300, 256, 4, 4), (1, 1024, 2048, 16, 4),
-                                   (1, 200, 1040, 8, 8)])
+                                   (1, 200, 1040, 8, 8), (1, 300, 320, 5, 5)])
 def test_bf16_block(art, shape):
     B, T, d, H, KV = shape
     hd = d // H
@@ -62,6 +62,28 @@ def test_bf16_block(art, shape):
     out = run_block(art, W, x, 0, H=H, KV=KV, rope_base=10000.0)
     ref = A.block(x, W["Wq"], W["Wk"], W["Wv"], W["Wo"], H=H, KV=KV, rope_base=10000.0)
     assert_close(out, ref, torch.bfloat16, f"bf16 block {shape}")
+
+
+@pytest.mark.parametrize("shape", [(1, 300, 256, 4, 4), (1, 300, 320, 5, 5), (2, 512, 1024, 8, 2)])
+def test_block_projections_on_cta_pairs_equal_one_sm(art, shape, monkeypatch):
+    """The projection GEMM on CTA pairs (256-row tiles, each SM staging half of the weights'
+    columns) gives the same bits as on one SM per 128-row tile. The shapes have a last row
+    tile whose second half lies past M (300 rows) and column tiles whose second half lies
+    partly or wholly past N (QKV 960 and Wo 320 columns)."""
+    B, T, d, H, KV = shape
+    hd = d // H
+    g = torch.Generator().manual_seed(37)
+    x = workloads.normal((B, T, d), 0, torch.bfloat16, g)
+    W = {n: (torch.randn(*s, generator=g) / np.sqrt(d)).to(torch.bfloat16)
+         for n, s in (("Wq", (d, H * hd)), ("Wk", (d, KV * hd)), ("Wv", (d, KV * hd)),
+                      ("Wo", (H * hd, d)))}
+    pair = run_block(art, W, x, 0, H=H, KV=KV, rope_base=10000.0)
+    torch.cuda.synchronize()
+    monkeypatch.setenv("ATTN_TEST_GEMM_SINGLE", "1")
+    one = run_block(art, W, x, 0, H=H, KV=KV, rope_base=10000.0)
+    torch.cuda.synchronize()
+    assert art.attn_sync_status() == 0
+    assert torch.equal(pair, one)
 
 
 def sampled_rows(T: int, seed: int) -> np.ndarray:
