@@ -12,7 +12,9 @@
 // 128 x 256 tile would need all four W boxes in its own shared memory per stage: the MMA reads
 // of A and W plus the TMA writes (96 KB per stage) exceed what shared memory delivers at the
 // tensor rate, so one-SM tiles stall on it. The one-SM form (M <= 128) keeps four stages of A
-// and four W boxes. In both, warp 4 issues the TMA loads (the pair's both count on CTA 0's
+// and four W boxes. When the last round of pair tiles would keep at most half of the pairs
+// busy, its tiles are cut into two 128-column halves (M=256, N=128 MMAs) so that it takes about
+// half as long. In both forms, warp 4 issues the TMA loads (the pair's both count on CTA 0's
 // barrier), warp 5 allocates TMEM and issues the MMAs into one of two 256-column accumulators,
 // and warps 0-3 read the other accumulator back (one TMEM lane = one row of C per thread) and
 // store bf16: a tile's epilogue overlaps the next tile's MMAs. Rows and columns past M, N are
@@ -23,8 +25,9 @@
 //
 // Epilogues (GemmEpilogue): a store, optionally with each row scaled (the fused block's
 // 1/RMS), one segment's heads turned pairwise by the (cos, sin) table of the row's position
-// (the keys: a 32-column chunk lies in one head, since hd is 64 or 128 and tiles start at
-// multiples of 256), and segments copied into a KV cache; or C = A W plus a residual.
+// (the keys: a 32-column chunk lies in one head, since hd is 64 or 128 and tiles and half-width
+// items start at multiples of 128), and segments copied into a KV cache; or C = A W plus a
+// residual.
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
@@ -60,6 +63,7 @@ struct GCfg {
   static constexpr int OFF_BAR = NS * STAGE;
   static constexpr int SMEM = OFF_BAR + (2 * NS + 5) * 8 + 16 + 1024;
   static constexpr uint32_t IDESC = idesc_bf16_f32(ROWS, BN, 0, 1);
+  static constexpr uint32_t IDESC_HALF = idesc_bf16_f32(ROWS, BN / 2, 0, 1);  // a 128-column item
 };
 static_assert(GCfg<true>::SMEM <= 227 * 1024 && GCfg<false>::SMEM <= 227 * 1024, "shared memory");
 
@@ -74,6 +78,22 @@ struct GemmArgs {
   int* status;
   GemmEpilogue ep;
 };
+
+// The work of a launch: tiles in rounds over the CTAs (pairs). In the pair form, when the last
+// round would keep at most half of the pairs busy, its tiles are cut into two 128-column halves
+// (items), so that it ends in about half the time. Item idx: rows m0.., columns gn0.., width w.
+struct Item {
+  int m0, gn0, w;
+};
+__device__ __forceinline__ Item item_of(int idx, int F, int ntn, int rows) {
+  const int tile = idx < F ? idx : F + (idx - F) / 2;
+  const int half = idx < F ? 0 : ((idx - F) & 1) + 1;  // 0: whole tile, 1 or 2: its halves
+  Item it;
+  it.m0 = (tile / ntn) * rows;
+  it.gn0 = (tile % ntn) * BN + (half == 2 ? BN / 2 : 0);
+  it.w = half ? BN / 2 : BN;
+  return it;
+}
 
 __device__ __forceinline__ void store32(__nv_bfloat16* dst, const float (&v)[32]) {
 #pragma unroll
@@ -107,6 +127,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int cid = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int ncta = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int ntn = (g.N + BN - 1) / BN, ntiles = ntn * ((g.M + C::ROWS - 1) / C::ROWS);
+  const int rem = ntiles % ncta;
+  const bool split = PAIR && rem > 0 && 2 * rem <= ncta;
+  const int F = split ? ntiles - rem : ntiles;   // whole tiles
+  const int nitems = split ? F + 2 * rem : ntiles;
   const int nk = (g.K + BK - 1) / BK;
   // the segment of a column of the launch
   auto seg_of = [&](int col) {
@@ -151,23 +175,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (g.nseg > 1) tma_prefetch(&tmW1);
       if (g.nseg > 2) tma_prefetch(&tmW2);
       int u = 0;  // ring uses so far
-      for (int tile = cid; tile < ntiles && !*abort_flag; tile += ncta) {
-        const int gn0 = (tile % ntn) * BN, m0 = (tile / ntn) * C::ROWS;
-        // this CTA's rows of A and columns of W; boxes that start past M or N are not loaded
-        // (those rows and columns of C are not stored)
-        const int am0 = m0 + (int)rank * BM, bn0 = gn0 + (int)rank * C::B_COLS;
+      for (int idx = cid; idx < nitems && !*abort_flag; idx += ncta) {
+        const Item itm = item_of(idx, F, ntn, C::ROWS);
+        const int gn0 = itm.gn0, m0 = itm.m0;
+        // this CTA's rows of A and columns of W (half of the item's in the pair form); boxes
+        // that start past M or N are not loaded (those rows and columns of C are not stored)
+        const int cw = PAIR ? itm.w / 2 : itm.w;
+        const int am0 = m0 + (int)rank * BM, bn0 = gn0 + (int)rank * cw;
         const bool a_in = am0 < g.M;
-        const int nbv = max(0, min(C::B_COLS / 64, (g.N - bn0 + 63) / 64));
+        const int nbv = max(0, min(cw / 64, (g.N - bn0 + 63) / 64));
         // the bytes the stage's barrier counts: this CTA's, or (PAIR, on rank 0) both CTAs'
         uint32_t bytes = (a_in ? A_BYTES : 0) + nbv * (BK * 128);
         if (PAIR) {
-          const int pbv = max(0, min(C::B_COLS / 64, (g.N - (gn0 + C::B_COLS) + 63) / 64));
+          const int pbv = max(0, min(cw / 64, (g.N - (gn0 + cw) + 63) / 64));
           bytes += (m0 + BM < g.M ? A_BYTES : 0) + pbv * (BK * 128);  // (used on rank 0 only)
         }
-        // the tile's W map, chosen once when this CTA's columns lie in one segment (choosing it
+        // the item's W map, chosen once when this CTA's columns lie in one segment (choosing it
         // per box costs ~10% of the GEMM); per box only for columns across a narrow segment
         const int sgt = seg_of(bn0 < g.N ? bn0 : g.N - 1);
-        const bool one_seg = sgt == seg_of(min(bn0 + C::B_COLS, g.N) - 1);
+        const bool one_seg = sgt == seg_of(min(bn0 + cw, g.N) - 1);
         const CUtensorMap* tmWt = sgt == 0 ? &tmW0 : (sgt == 1 ? &tmW1 : &tmW2);
         const int lc0 = bn0 - (sgt == 0 ? 0 : g.seg_end[sgt - 1]);
         for (int kb = 0; kb < nk; ++kb, ++u) {
@@ -204,8 +230,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint64_t dA = smem_desc_sw128(smem_u32(smem), 16, 1024);
       const uint64_t dW = smem_desc_sw128(smem_u32(smem + A_BYTES), BK * 128, 1024);
       int u = 0, i = 0;  // ring uses and tiles so far
-      for (int tile = cid; tile < ntiles; tile += ncta, ++i) {
-        // accumulator i % 2, free once the epilogue (of both CTAs) has read the tile two before
+      for (int idx = cid; idx < nitems; idx += ncta, ++i) {
+        const uint32_t idesc = item_of(idx, F, ntn, C::ROWS).w == BN ? C::IDESC : C::IDESC_HALF;
+        // accumulator i % 2, free once the epilogue (of both CTAs) has read the item two before
         const int ab = i & 1;
         if (!mbar_wait(acc_empty + ab, ((i >> 1) & 1) ^ 1, abort_flag, g.status, WAIT_LIMIT_NS)) break;
         tc_fence_after();
@@ -224,9 +251,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint64_t a = dA + so + (uint64_t)((kk * 32) >> 4), b = dW + so + (uint64_t)((kk * 16 * 128) >> 4);
             const uint32_t acc_in = (kb > 0 || kk > 0) ? 1u : 0u;
             if (PAIR)
-              umma_ss_pair(acc, a, b, C::IDESC, acc_in);
+              umma_ss_pair(acc, a, b, idesc, acc_in);
             else
-              umma_ss(acc, a, b, C::IDESC, acc_in);
+              umma_ss(acc, a, b, idesc, acc_in);
           }
           if (PAIR)
             umma_commit_pair(empty + st, 0x3);  // the stage is free in both CTAs
@@ -250,8 +277,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // tile after tile, while the MMAs of the next tile fill the other accumulator
     const uint32_t ae = PAIR ? cluster_addr(acc_empty, 0) : 0u;
     int it = 0;
-    for (int tile = cid; tile < ntiles; tile += ncta, ++it) {
-      const int gn0 = (tile % ntn) * BN, m0 = (tile / ntn) * C::ROWS + (int)rank * BM;
+    for (int idx = cid; idx < nitems; idx += ncta, ++it) {
+      const Item itm = item_of(idx, F, ntn, C::ROWS);
+      const int gn0 = itm.gn0, m0 = itm.m0 + (int)rank * BM;
       const int ab = it & 1;
       if (!mbar_wait(acc_full + ab, (it >> 1) & 1, abort_flag, g.status, WAIT_LIMIT_NS)) break;
       tc_fence_after();
@@ -259,7 +287,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t t = tmem + ab * BN + ((uint32_t)(warp * 32) << 16);
       const float rs = (g.ep.mode == 0 && g.ep.row_scale && row < g.M) ? g.ep.row_scale[row] : 1.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = 0; c0 < itm.w; c0 += 32) {
         float v[32];
         tmem_ld32(t + c0, v);
         tmem_wait_ld();
@@ -470,7 +498,13 @@ cudaError_t launch_gemm_tc_multi(const void* A, int nseg, const void* const* Ws,
   if (pairs > 0) {
     const long long tiles = ntn * ((M + 2 * BM - 1) / (2 * BM));
     if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
-    const int ncl = tiles < pairs ? (int)tiles : pairs;
+    int ncl = tiles < pairs ? (int)tiles : pairs;
+    // Test hook: ATTN_TEST_GEMM_CLUSTERS (1..the device's count) fixes the number of pairs, so
+    // that small problems also run several rounds and a last round cut into half-width items.
+    if (const char* env = std::getenv("ATTN_TEST_GEMM_CLUSTERS")) {
+      const int nc = std::atoi(env);
+      if (nc >= 1 && nc <= pairs) ncl = (int)std::min<long long>(nc, tiles);
+    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;

@@ -64,12 +64,19 @@ def test_bf16_block(art, shape):
     assert_close(out, ref, torch.bfloat16, f"bf16 block {shape}")
 
 
+@pytest.mark.parametrize("clusters", [None, 3, 6, 7])
 @pytest.mark.parametrize("shape", [(1, 300, 256, 4, 4), (1, 300, 320, 5, 5), (2, 512, 1024, 8, 2)])
-def test_block_projections_on_cta_pairs_equal_one_sm(art, shape, monkeypatch):
+def test_block_projections_on_cta_pairs_equal_one_sm(art, shape, clusters, monkeypatch):
     """The projection GEMM on CTA pairs (256-row tiles, each SM staging half of the weights'
     columns) gives the same bits as on one SM per 128-row tile. The shapes have a last row
     tile whose second half lies past M (300 rows) and column tiles whose second half lies
-    partly or wholly past N (QKV 960 and Wo 320 columns)."""
+    partly or wholly past N (QKV 960 and Wo 320 columns). A fixed number of pairs (a test
+    hook) gives several rounds and, where the last round would keep at most half of the pairs
+    busy, a last round of half-width items (e.g. 320 columns on 3 pairs: the second row pair's
+    last tile cut into columns 256-383 and 384-511, the latter wholly past N; QKV 960 columns
+    on 6 pairs: 768-895 and 896-1023, partly past N; QKV 1536 columns on 7 pairs)."""
+    if clusters is not None:
+        monkeypatch.setenv("ATTN_TEST_GEMM_CLUSTERS", str(clusters))
     B, T, d, H, KV = shape
     hd = d // H
     g = torch.Generator().manual_seed(37)
@@ -79,6 +86,7 @@ def test_block_projections_on_cta_pairs_equal_one_sm(art, shape, monkeypatch):
                       ("Wo", (H * hd, d)))}
     pair = run_block(art, W, x, 0, H=H, KV=KV, rope_base=10000.0)
     torch.cuda.synchronize()
+    monkeypatch.delenv("ATTN_TEST_GEMM_CLUSTERS", raising=False)
     monkeypatch.setenv("ATTN_TEST_GEMM_SINGLE", "1")
     one = run_block(art, W, x, 0, H=H, KV=KV, rope_base=10000.0)
     torch.cuda.synchronize()
