@@ -316,3 +316,60 @@ def test_binding_rejects_mismatched_shapes(lib):
                                torch.zeros(H, 64, hd + 2, dtype=bf), sl, sl)
     with pytest.raises(ValueError, match="pos"):
         art.attn_kv_append(dq[:, :KV], dq[:, :KV], kc, kc, torch.zeros(B + 1, dtype=torch.int32))
+
+
+def _host_plan_bytes(B, T, H, KV, hd, rope_base, dtype):
+    """The host-buffer prefill's device scratch, restated: the slices (runs of at most eight
+    groups of whole sequences when B >= 4; else one sequence and the largest key/value-head
+    group giving 4 to 16 slices), the last slice cut into a slice per sequence and halving head
+    groups; per slice dense q, k, v, out and lse (each rounded to 256 bytes), plus the rotation
+    scratch of the largest slice (bf16, hd 64/128, RoPE only)."""
+    r256 = lambda n: (n + 255) // 256 * 256
+    es = 4 if dtype == 0 else 2
+    G = H // KV
+    sl = []
+    if B >= 4:
+        runs = min(B, 8)
+        nbs = (B + runs - 1) // runs
+        sl = [(b0, min(nbs, B - b0), 0, KV) for b0 in range(0, B, nbs)]
+    else:
+        ng = KV
+        for g in range(KV, 0, -1):
+            if KV % g == 0 and B * (KV // g) >= 4:
+                if B * (KV // g) <= 16:
+                    ng = g
+                break
+        sl = [(b, 1, g0, ng) for b in range(B) for g0 in range(0, KV, ng)]
+    b0, nb, g0, ng = sl.pop()
+    if nb > 1:
+        sl.append((b0, nb - 1, 0, KV))
+        b0, nb, g0, ng = b0 + nb - 1, 1, 0, KV
+    rem = ng
+    while rem > 1:
+        part = (rem + 1) // 2
+        sl.append((b0, 1, g0, part))
+        g0 += part
+        rem -= part
+    if rem == 1:
+        sl.append((b0, 1, g0, 1))
+    total = 0
+    rot = 0
+    for (_, nb, _, ng) in sl:
+        q = r256(nb * T * ng * G * hd * es)
+        kv = r256(nb * T * ng * hd * es)
+        lse = r256(nb * ng * G * T * 4)
+        total += 2 * q + 2 * kv + lse
+        if dtype == 1 and hd in (64, 128) and rope_base > 0:
+            rot = max(rot, nb * T * ng * hd * 2)
+    return total + r256(rot), len(sl)
+
+
+@pytest.mark.parametrize("shape", [(2, 4096, 32, 8, 128, 5e5, 1), (1, 257, 8, 2, 128, 5e5, 1),
+                                   (3, 130, 8, 1, 128, 1e4, 1), (5, 200, 4, 2, 64, 0.0, 1),
+                                   (18, 40, 4, 4, 128, 1e4, 0), (1, 90, 12, 4, 64, 1e4, 0),
+                                   (2, 300, 16, 8, 128, 1e4, 1), (1, 64, 7, 7, 64, 1e4, 1)])
+def test_prefill_host_workspace_follows_the_slice_plan(lib, shape):
+    B, T, H, KV, hd, base, dtype = shape
+    want, nslices = _host_plan_bytes(B, T, H, KV, hd, base, dtype)
+    assert nslices <= 32
+    assert lib.attn_prefill_host_workspace_size(B, T, H, KV, hd, base, dtype) == want
